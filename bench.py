@@ -1,0 +1,492 @@
+#!/usr/bin/env python
+"""Benchmark of the smoothed W8A8 linear layer (SmoothQuant hot path) on B200.
+
+One step = one pass of the whole path over one batch of synthetic input:
+calibration absmax (LayerNorm-fused when a LayerNorm precedes), smoothing
+factors (eq. (4)), weight + LayerNorm fold with per-output-channel INT8,
+the fused LayerNorm + smoothing + INT8 activation quantizer, and the INT8
+tcgen05 GEMM with the dequantizing epilogue.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
+                    [--impl reference]
+
+`value` is whole-job throughput in TOPS = 2*M*N*K per step (all ranks) over
+the device time of the timed steps (CUDA events on the launching stream, max
+over ranks); L2 is flushed (a 256 MiB write) before every timed step and the
+flush is outside the timed events.  Inputs are resident in HBM before timing.
+`e2e` is the same metric through the public Python API with pinned host
+buffers: every step copies its inputs host->device and its output back.
+`--impl reference` times the CPU oracle (tests-only code) on bounded samples
+of the same workload, each step extrapolated linearly to the full workload.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import synth  # noqa: E402
+
+METRIC = "W8A8 smoothed-linear TOPS & % INT8 peak; small-M HBM GB/s (1×B200)"
+DEFAULT_WORKLOAD = "opt6.7b_qkv_t2048"
+FLUSH_BYTES = 256 << 20
+# INT8 dense peak = measured bf16 dense peak x the nominal int8:bf16 ratio
+# (4.5 POPS : 2.25 PFLOP/s = 2).
+INT8_PER_BF16 = 2.0
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
+    ap.add_argument("--linear", default=None, help="linear of the workload (default: first)")
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--e2e-steps", type=int, default=20)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    return ap.parse_args()
+
+
+def pick_linear(args):
+    wl = synth.workloads()[args.workload]
+    lin = wl.linears[0]
+    if args.linear:
+        lin = next(l for l in wl.linears if l.name == args.linear)
+    return wl, lin
+
+
+def config_of(wl, lin, world):
+    return {
+        "workload": wl.name,
+        "linear": lin.name,
+        "M": lin.T, "N": lin.N, "K": lin.K, "T_cal": lin.T_cal,
+        "layernorm": lin.ln, "alpha": lin.alpha,
+        "act_quant": "per-token dynamic" if lin.per_token else "per-tensor static",
+        "io_dtype": lin.dtype,
+        "l2": "flushed before every timed step (256 MiB write, outside the timed events)",
+        "parallelism": f"replicas x{world}",
+    }
+
+
+# ---------------------------------------------------------------- clocks
+class ClockSampler:
+    """Samples SM clock and throttle reasons with NVML while the timed region runs."""
+
+    REASONS = {
+        0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap",
+        0x8: "hw_slowdown", 0x20: "sw_thermal_slowdown", 0x40: "hw_thermal_slowdown",
+        0x80: "hw_power_brake_slowdown", 0x100: "display_clock_setting",
+    }
+
+    def __init__(self, index):
+        self.samples = []
+        self.reasons = set()
+        self.max_mhz = None
+        self._stop = threading.Event()
+        self._ok = False
+        try:
+            import pynvml
+
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            self.h = pynvml.nvmlDeviceGetHandleByIndex(index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+            self._ok = True
+        except Exception:  # noqa: BLE001 - clocks are reported as unavailable
+            self._ok = False
+
+    def _run(self):
+        while not self._stop.is_set():
+            try:
+                self.samples.append(self.nv.nvmlDeviceGetClockInfo(self.h, self.nv.NVML_CLOCK_SM))
+                r = self.nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+                for bit, name in self.REASONS.items():
+                    if r & bit and name != "gpu_idle":
+                        self.reasons.add(name)
+            except Exception:  # noqa: BLE001
+                pass
+            time.sleep(0.02)
+
+    def __enter__(self):
+        if self._ok:
+            self.t = threading.Thread(target=self._run, daemon=True)
+            self.t.start()
+        return self
+
+    def __exit__(self, *a):
+        if self._ok:
+            self._stop.set()
+            self.t.join()
+
+    def summary(self):
+        if not self._ok or not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": ["unavailable"]}
+        return {"sm_mhz": statistics.median(self.samples), "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(self.reasons), "samples": len(self.samples)}
+
+
+# ---------------------------------------------------------------- our arm
+class Layer:
+    """Device buffers of one smoothed linear and the five calls of one step."""
+
+    def __init__(self, sq, torch, lin, d, dev):
+        self.sq, self.torch, self.lin = sq, torch, lin
+        f32, bf16 = torch.float32, torch.bfloat16
+        io = bf16 if lin.dtype == "bf16" else f32
+        K, N, M, Tc = lin.K, lin.N, lin.T, lin.T_cal
+        self.io = io
+
+        def t(a):
+            if a is None:
+                return None
+            if a.dtype == np.uint16:
+                return torch.from_numpy(a.view(np.int16)).view(bf16).to(dev)
+            return torch.from_numpy(a).to(dev)
+
+        self.x_cal, self.x, self.w = t(d["x_cal"]), t(d["x"]), t(d["w"])
+        self.gamma, self.beta = t(d["gamma"]), t(d["beta"])
+        self.amax = torch.empty(K, dtype=f32, device=dev)
+        self.s = torch.empty(K, dtype=f32, device=dev)
+        self.inv_s = torch.empty(K, dtype=f32, device=dev)
+        self.dA = torch.empty(1, dtype=f32, device=dev)
+        self.wq = torch.empty((N, K), dtype=torch.int8, device=dev)
+        self.ws = torch.empty(N, dtype=f32, device=dev)
+        self.g2 = torch.empty(K, dtype=f32, device=dev) if lin.ln else None
+        self.b2 = torch.empty(K, dtype=f32, device=dev) if lin.ln else None
+        self.xq = torch.empty((M, K), dtype=torch.int8, device=dev)
+        self.act = torch.empty(M if lin.per_token else 1, dtype=f32, device=dev)
+        self.y = torch.empty((M, N), dtype=io, device=dev)
+        self.workspace = sq.Workspace(dev)
+        self.kernels_per_step = 7
+
+    def step(self, ev=None):
+        sq, L = self.sq, self.lin
+        e = ev or [None] * 6
+
+        def rec(i):
+            if e[i] is not None:
+                e[i].record()
+
+        rec(0)
+        self.amax.zero_()
+        sq.sq_calib_absmax(self.x_cal, self.amax, self.gamma, self.beta, 1e-5)
+        rec(1)
+        sq.sq_smooth_scales(self.amax, self.w, L.alpha, self.s, self.inv_s,
+                            None if L.per_token else self.dA)
+        rec(2)
+        sq.sq_fuse_weights_q8(self.w, self.s, self.wq, self.ws, self.gamma, self.beta,
+                              self.g2, self.b2)
+        rec(3)
+        act = self.act
+        if not L.per_token:
+            act.copy_(self.dA)
+        if L.ln:
+            sq.sq_ln_smooth_quant_act(self.x, self.xq, act, self.g2, self.b2, 1e-5,
+                                      per_token=L.per_token)
+        else:
+            sq.sq_ln_smooth_quant_act(self.x, self.xq, act, inv_s=self.inv_s,
+                                      per_token=L.per_token)
+        rec(4)
+        sq.sq_gemm_w8a8(self.xq, self.wq, act, self.ws, self.y, per_token=L.per_token,
+                        workspace=self.workspace)
+        rec(5)
+
+
+def algorithmic_bytes(lin):
+    """Bytes each step reads/writes once (the per-kernel roofline numerators)."""
+    b = 2 if lin.dtype == "bf16" else 4
+    M, N, K, Tc = lin.T, lin.N, lin.K, lin.T_cal
+    return {
+        "calib_absmax": Tc * K * b + 4 * K + (8 * K if lin.ln else 0),
+        "smooth_scales": N * K * b + 12 * K,
+        "fuse_weights_q8": N * K * b + N * K + 4 * N + 4 * K + (16 * K if lin.ln else 0),
+        "ln_smooth_quant_act": M * K * b + M * K + 4 * M + (8 * K if lin.ln else 4 * K),
+        "gemm_w8a8": M * K + N * K + M * N * b + 4 * N + 4 * M,
+    }
+
+
+def run_ours(args):
+    import torch
+    import torch.distributed as dist
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world != args.gpus:
+        raise SystemExit(f"--gpus {args.gpus} but WORLD_SIZE={world}")
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        from datetime import timedelta
+
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120),
+                                device_id=dev)
+    import w8a8_int8_gemm_calib_b200 as sq
+
+    wl, lin = pick_linear(args)
+    d = synth.make_linear_inputs(lin)
+    layer = Layer(sq, torch, lin, d, dev)
+    flush = torch.empty(FLUSH_BYTES // 4, dtype=torch.int32, device=dev)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+
+    for _ in range(max(3, args.warmup)):
+        layer.step()
+    sq.sq_sync_status()
+    barrier()
+
+    K = args.steps
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(6)] for _ in range(K)]
+    clocks = ClockSampler(torch.cuda.current_device())
+    with clocks:
+        barrier()
+        for i in range(K):
+            flush.fill_(i)
+            layer.step(evs[i])
+        barrier()
+    sq.sq_sync_status()
+    names = ["calib_absmax", "smooth_scales", "fuse_weights_q8", "ln_smooth_quant_act",
+             "gemm_w8a8"]
+    per = {n: [] for n in names}
+    step_ms = []
+    for e in evs:
+        for j, n in enumerate(names):
+            per[n].append(e[j].elapsed_time(e[j + 1]))
+        step_ms.append(e[0].elapsed_time(e[5]))
+    total_ms = float(sum(step_ms))
+    if world > 1:
+        t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        total_ms = float(t.item())
+    ops = 2.0 * lin.T * lin.N * lin.K
+    value = world * ops * K / (total_ms * 1e-3) / 1e12
+
+    # ---- e2e through the public API with pinned host buffers
+    e2e = run_e2e(sq, torch, layer, lin, d, dev, args.e2e_steps, world, barrier)
+
+    peaks, peak_kind = load_peaks()
+    bf16_peak = peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"])
+    int8_peak = bf16_peak * INT8_PER_BF16
+    gemm_ms = statistics.mean(per["gemm_w8a8"])
+    gemm_tops = ops / (gemm_ms * 1e-3) / 1e12
+    ab = algorithmic_bytes(lin)
+    hbm = peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"])
+    kernels = {}
+    for n in names:
+        ms = statistics.mean(per[n])
+        k = {"ms": round(ms, 5), "gbs": round(ab[n] / (ms * 1e-3) / 1e9, 1),
+             "hbm_frac": round(ab[n] / (ms * 1e-3) / 1e9 / hbm, 3)}
+        if n == "gemm_w8a8":
+            k["tops"] = round(gemm_tops, 1)
+            k["int8_frac"] = round(gemm_tops / int8_peak, 3)
+        kernels[n] = k
+    line = {
+        "metric": METRIC,
+        "value": round(value, 2),
+        "unit": "TOPS",
+        "n_gpus": world,
+        "steps": K,
+        "warmup": max(3, args.warmup),
+        "ms_per_step": round(total_ms / K, 5),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "int8",
+        "data": "synthetic (seeded outlier-structured activations, random-init weights)",
+        "config": config_of(wl, lin, world),
+        "roofline": {
+            "bound": "tensor",
+            "kernel": "gemm_w8a8 (tcgen05.mma kind::i8)",
+            "achieved": round(gemm_tops, 1),
+            "peak": round(int8_peak, 1),
+            "unit": "TFLOP/s",
+            "frac": round(gemm_tops / int8_peak, 4),
+            "traffic": None,
+            "peak_note": f"int8 dense = {peak_kind} bf16 burst {bf16_peak} TFLOP/s x 2 "
+                         "(nominal int8:bf16 ratio); 'TFLOP/s' here counts int8 ops",
+        },
+        "kernels": kernels,
+        "e2e": e2e,
+        "gpu_launches": layer.kernels_per_step * K,
+        "clocks": clocks.summary(),
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(lin, d)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
+def run_e2e(sq, torch, layer, lin, d, dev, steps, world, barrier):
+    """Same step through the public API, inputs copied from pinned host memory
+    every step and the output read back."""
+    def pinned(a):
+        if a is None:
+            return None
+        t = (torch.from_numpy(a.view(np.int16)).view(torch.bfloat16) if a.dtype == np.uint16
+             else torch.from_numpy(a))
+        return t.pin_memory()
+
+    hx_cal, hx, hw = pinned(d["x_cal"]), pinned(d["x"]), pinned(d["w"])
+    hg, hb = pinned(d["gamma"]), pinned(d["beta"])
+    hy = torch.empty(layer.y.shape, dtype=layer.y.dtype).pin_memory()
+    h2d = sum(t.numel() * t.element_size() for t in (hx_cal, hx, hw, hg, hb) if t is not None)
+    d2h = hy.numel() * hy.element_size()
+
+    def one():
+        layer.x_cal.copy_(hx_cal, non_blocking=True)
+        layer.x.copy_(hx, non_blocking=True)
+        layer.w.copy_(hw, non_blocking=True)
+        if hg is not None:
+            layer.gamma.copy_(hg, non_blocking=True)
+            layer.beta.copy_(hb, non_blocking=True)
+        layer.step()
+        hy.copy_(layer.y, non_blocking=True)
+
+    for _ in range(2):
+        one()
+    barrier()
+    s = torch.cuda.Event(enable_timing=True)
+    e = torch.cuda.Event(enable_timing=True)
+    s.record()
+    for _ in range(steps):
+        one()
+    e.record()
+    barrier()
+    ms = s.elapsed_time(e) / steps
+    if world > 1:
+        import torch.distributed as dist
+
+        t = torch.tensor([ms], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+    ops = 2.0 * lin.T * lin.N * lin.K
+    return {"value": round(world * ops / (ms * 1e-3) / 1e12, 3), "unit": "TOPS",
+            "ms_per_step": round(ms, 4), "h2d_bytes_per_step": int(h2d),
+            "d2h_bytes_per_step": int(d2h)}
+
+
+# ---------------------------------------------------------------- CPU oracle
+def oracle_step_sample(lin, d, frac_tokens, gemm_rows, frac_w):
+    """Time the oracle on a bounded sample of each step and extrapolate each
+    step linearly in the sampled dimension.  Returns (seconds_full, sample)."""
+    import oracle
+
+    oracle.build()
+    Tc = max(1, int(lin.T_cal * frac_tokens))
+    Tq = max(1, int(lin.T * frac_tokens))
+    Nw = max(1, int(lin.N * frac_w))
+    t = {}
+    t0 = time.perf_counter()
+    amax = oracle.calib_absmax(d["x_cal"][:Tc], d["gamma"], d["beta"], 1e-5)
+    t["calib"] = (time.perf_counter() - t0) * lin.T_cal / Tc
+    t0 = time.perf_counter()
+    aw = oracle.weight_colmax(d["w"][:Nw])
+    s, inv_s = oracle.smooth_scales(amax, aw, lin.alpha)
+    dA = oracle.static_delta(amax, s)
+    t["scales"] = (time.perf_counter() - t0) * lin.N / Nw
+    t0 = time.perf_counter()
+    wq, ws = oracle.fuse_weights_q8(d["w"][:Nw], s)
+    if lin.ln:
+        g2, b2 = oracle.fold_ln(d["gamma"], d["beta"], s)
+    t["fuse"] = (time.perf_counter() - t0) * lin.N / Nw
+    t0 = time.perf_counter()
+    if lin.ln:
+        xq, act, _ = oracle.quant_act(d["x"][:Tq], g2, b2, 1e-5, per_token=lin.per_token,
+                                      static_delta=dA)
+    else:
+        xq, act, _ = oracle.quant_act(d["x"][:Tq], inv_s=inv_s, per_token=lin.per_token,
+                                      static_delta=dA)
+    t["quant"] = (time.perf_counter() - t0) * lin.T / Tq
+    R = max(1, min(gemm_rows, Tq))
+    t0 = time.perf_counter()
+    oracle.gemm_w8a8(xq[:R], wq, act[:R] if lin.per_token else act, ws,
+                     per_token=lin.per_token, out_bf16=(lin.dtype == "bf16"))
+    t["gemm"] = (time.perf_counter() - t0) * (lin.T / R) * (lin.N / Nw)
+    sample = (f"oracle (single-threaded C) on {Tc}/{lin.T_cal} calibration tokens, "
+              f"{Nw}/{lin.N} weight rows, {Tq}/{lin.T} runtime tokens and a {R}x{Nw}x{lin.K} "
+              f"GEMM; each step extrapolated linearly to the full workload")
+    return sum(t.values()), t, sample
+
+
+def cpu_baseline(lin, d):
+    # about 10-20 s of single-core work on the opt6.7b workload
+    secs, parts, sample = oracle_step_sample(lin, d, 1 / 16, 8, 1 / 4)
+    ops = 2.0 * lin.T * lin.N * lin.K
+    return {"value": round(ops / secs / 1e12, 6), "unit": "TOPS", "cores": 1,
+            "kind": "oracle", "sample": sample,
+            "seconds_per_step_extrapolated": round(secs, 2),
+            "parts_s": {k: round(v, 3) for k, v in parts.items()}}
+
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    if rank != 0:
+        return
+    wl, lin = pick_linear(args)
+    d = synth.make_linear_inputs(lin)
+    vals = []
+    for _ in range(max(3, args.warmup) if False else 0):
+        pass
+    for _ in range(max(1, min(args.warmup, 1))):
+        oracle_step_sample(lin, d, 1 / 64, 2, 1 / 16)
+    secs_all = []
+    sample = ""
+    for _ in range(args.steps if args.steps <= 5 else 5):
+        secs, _, sample = oracle_step_sample(lin, d, 1 / 64, 2, 1 / 16)
+        secs_all.append(secs)
+    ops = 2.0 * lin.T * lin.N * lin.K
+    total = sum(secs_all)
+    value = ops * len(secs_all) / total / 1e12
+    line = {
+        "metric": METRIC, "value": round(value, 6), "unit": "TOPS", "impl": "reference",
+        "n_gpus": world, "steps": len(secs_all), "warmup": 1,
+        "ms_per_step": round(total / len(secs_all) * 1e3, 3),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "int8",
+        "data": "synthetic (seeded outlier-structured activations, random-init weights)",
+        "config": config_of(wl, lin, world),
+        "cpu_baseline": {"value": round(value, 6), "unit": "TOPS", "cores": 1, "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": round(value, 6), "unit": "TOPS", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    args = parse()
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

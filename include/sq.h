@@ -1,0 +1,228 @@
+/*
+ * sq.h -- C ABI of the B200 (sm_100a) smoothed W8A8 linear layer.
+ *
+ * The layer is SmoothQuant's: an activation absmax over calibration tokens,
+ * the smoothing factors of eq. (4), an offline fold of those factors into the
+ * weights (then per-output-channel symmetric INT8) and into the preceding
+ * LayerNorm, a runtime fused LayerNorm + smoothing + symmetric INT8
+ * activation quantizer, and an INT8 x INT8 -> INT32 GEMM on the tcgen05 tensor
+ * cores whose epilogue dequantizes by act_scale[token] * w_scale[out].
+ *
+ * Sources, cited by tag below:
+ *   [explainer] "SmoothQuant 如何解决激活量化难题？为什么适合 W8A8？"
+ *   [review]    "SmoothQuant：大型语言模型的精准高效训练后量化 — 深度技术评审"
+ *   [embedded]  "嵌入式 SLM 动态权重量化：SmoothQuant 激活异常值迁移与 INT8 部署实战"
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ * Memory.   Every tensor pointer is DEVICE memory owned by the caller,
+ *           contiguous, row-major, and 16-byte aligned.  The library
+ *           allocates no device memory; the only library-owned device state
+ *           is one status word per device (a static __device__ variable).
+ * Layouts.  X is [T,K] (token, input channel).  W and Wq are [N,K]
+ *           (output channel, input channel), i.e. K-major, the transpose of
+ *           the review's W in Y = XW.  Y is [M,N].
+ * Shapes.   K (the input width) must be a multiple of 16 in [16, 133136];
+ *           the upper bound keeps 127*127*K below 2^31 so the INT32
+ *           accumulators cannot overflow.  T, M or N equal to 0 is an empty
+ *           problem: the call returns SQ_OK and launches nothing.  Negative
+ *           sizes are SQ_ERR_SHAPE.
+ * Streams.  Work is enqueued on `stream` (NULL = the legacy default stream)
+ *           and every call is asynchronous.  Argument checks run on the host
+ *           before anything is enqueued: on any error nothing is launched
+ *           and the outputs are untouched.
+ * Errors.   A launch failure returns SQ_ERR_CUDA.  Faults detected on the
+ *           device (a bounded wait that ran out) are recorded in the device
+ *           status word and reported by sq_sync_status().  sq_last_error()
+ *           gives a one-line description of the last host-side error on the
+ *           calling thread.
+ * Numerics. The fp32 operations of every step run in a fixed order with one
+ *           IEEE rounding each (no contraction into FMA except where stated),
+ *           so integer codes, scales and INT32 accumulators are reproducible
+ *           bit for bit: Delta(a) = max(a, 1e-7f) / 127; Q(v; Delta) =
+ *           clamp(round_half_even(v * (1/Delta)), -127, 127), NaN -> 0.
+ * Threads.  The entry points keep no host state between calls and may be
+ *           called from several host threads at once.
+ */
+#ifndef SQ_H
+#define SQ_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  SQ_OK = 0,
+  SQ_ERR_INVALID_ARG = 1, /* NULL where a tensor is required, bad enum, alpha outside [0,1] */
+  SQ_ERR_SHAPE = 2,       /* K not a multiple of 16 or outside [16,133136]; negative size */
+  SQ_ERR_ALIGN = 3,       /* a tensor pointer is not 16-byte aligned */
+  SQ_ERR_DTYPE = 4,       /* unsupported element type for this argument */
+  SQ_ERR_UNSUPPORTED = 5, /* no sm_100 device, or a size this build cannot serve */
+  SQ_ERR_CUDA = 6,        /* a CUDA runtime call failed */
+  SQ_ERR_TIMEOUT = 7,     /* device side: a bounded wait ran out (from sq_sync_status) */
+  SQ_ERR_WORKSPACE = 8    /* workspace NULL or smaller than sq_gemm_workspace_bytes() */
+} sq_status;
+
+typedef enum { SQ_F32 = 0, SQ_BF16 = 1 } sq_dtype;
+
+/* Activation quantization granularity ([review] §2.5, §2.6 Fig. 3, §6.3):
+ * per-tensor with a static step fixed at calibration (SmoothQuant-O3), or
+ * per-token with a step computed from each token's peak at run time (O1). */
+typedef enum {
+  SQ_ACT_PER_TENSOR_STATIC = 0,
+  SQ_ACT_PER_TOKEN_DYNAMIC = 1
+} sq_act_gran;
+
+typedef struct CUstream_st* sq_stream; /* a cudaStream_t */
+
+/*
+ * sq_calib_absmax -- per-input-channel activation peak over calibration
+ * tokens ([explainer] §四: record each input channel's activation peak on a
+ * calibration set; [review] §5.3: max|X_j| in eq. (4)).
+ *
+ *   amax[k] = max(amax[k], max_t |f(X)[t,k]|)
+ *
+ * f is the identity when ln_gamma is NULL.  Otherwise f is the LayerNorm that
+ * precedes the linear, with the ORIGINAL (unfolded) parameters:
+ * f(X)[t,k] = ((X[t,k] - mu_t) * rstd_t) * gamma[k] + beta[k], mu_t and the
+ * variance summed in the library's fixed order (128 slots of 8-element
+ * chunks), rstd_t = 1 / sqrt(var_t + ln_eps).  ln_beta may be NULL (= 0).
+ *
+ *   x      [T,K] of type xt (SQ_F32 or SQ_BF16), read only.
+ *   amax   [K] fp32, read and updated in place (a running maximum): zero it
+ *          before the first batch; calling again with the next batch of
+ *          tokens continues the same statistic.
+ * Values must be finite.
+ */
+sq_status sq_calib_absmax(const void* x, sq_dtype xt, int64_t T, int64_t K,
+                          const float* ln_gamma, const float* ln_beta,
+                          float ln_eps, float* amax, sq_stream stream);
+
+/*
+ * sq_smooth_scales -- smoothing factors of eq. (4) ([review] §5.3;
+ * [explainer] §三):
+ *
+ *   s_k = max|X_k|^alpha / max|W_k|^(1-alpha)
+ *
+ * max|W_k| = max_n |W[n,k]| is computed here from w [N,K] (type wt) and
+ * floored at 1e-7; the ratio is evaluated in fp64 (alpha = 0.5 with square
+ * roots, alpha in {0,1} without pow) and rounded once to fp32, then
+ * s_k = max(s_k, 1e-4f) and inv_s_k = 1/s_k (fp32 division).
+ *
+ *   amax_x            [K] fp32 calibration peaks (from sq_calib_absmax).
+ *   s, inv_s          [K] fp32 outputs.  s is also used as scratch.
+ *   act_delta_static  [1] fp32 output or NULL: the static per-tensor step of
+ *                     the smoothed activation, Delta(max_k amax_x[k]/s_k)
+ *                     (the calibration peak of X diag(s)^-1, [review] §6.4).
+ *   alpha             migration strength in [0, 1].
+ */
+sq_status sq_smooth_scales(const float* amax_x, const void* w, sq_dtype wt,
+                           int64_t N, int64_t K, float alpha, float* s,
+                           float* inv_s, float* act_delta_static,
+                           sq_stream stream);
+
+/*
+ * sq_fuse_weights_q8 -- offline fold of s ([embedded] §二; [review] §5.1
+ * eq. (3), §5.5):
+ *
+ *   W_hat[n,k] = W[n,k] * s_k                     (fp32)
+ *   w_scale[n] = Delta(max_k |W_hat[n,k]|)        (per output channel)
+ *   wq[n,k]    = Q(W_hat[n,k]; w_scale[n])        (int8, K-major)
+ *   gamma_out  = gamma / s,  beta_out = beta / s  (LayerNorm fold)
+ *
+ *   w      [N,K] type wt; s [K] fp32; wq [N,K] int8 out; w_scale [N] fp32 out.
+ *   gamma/gamma_out and beta/beta_out are optional pairs ([K] fp32 each):
+ *   a pair is folded when both of its pointers are non-NULL.
+ */
+sq_status sq_fuse_weights_q8(const void* w, sq_dtype wt, int64_t N, int64_t K,
+                             const float* s, int8_t* wq, float* w_scale,
+                             const float* gamma, const float* beta,
+                             float* gamma_out, float* beta_out,
+                             sq_stream stream);
+
+/*
+ * sq_ln_smooth_quant_act -- runtime fused LayerNorm + smoothing + symmetric
+ * INT8 activation quantizer ([embedded] §二: the modified LayerNorm emits the
+ * smoothed activation, which is quantized per tensor and fed to the INT8
+ * GEMM; [review] §2.2, §2.5, §2.6, §6.3).
+ *
+ *   y = LN(x) with the folded gamma_s, beta_s (same order as sq_calib_absmax)
+ *       when gamma_s != NULL, else y = x * inv_s (inv_s NULL: y = x);
+ *   SQ_ACT_PER_TOKEN_DYNAMIC: act_scale[t] = Delta(max_k |y[t,k]|) (output,
+ *       [T] fp32), xq[t,k] = Q(y[t,k]; act_scale[t]);
+ *   SQ_ACT_PER_TENSOR_STATIC: act_scale[0] is the calibrated step (input),
+ *       xq[t,k] = Q(y[t,k]; act_scale[0]); values above it saturate.
+ *
+ *   x [T,K] type xt; xq [T,K] int8 out.
+ *   n_clipped: NULL, or an int64 counter in device memory to which the number
+ *   of saturated codes is ADDED (the saturation rate of a static scale).
+ */
+sq_status sq_ln_smooth_quant_act(const void* x, sq_dtype xt, int64_t T,
+                                 int64_t K, const float* gamma_s,
+                                 const float* beta_s, float ln_eps,
+                                 const float* inv_s, sq_act_gran gran,
+                                 float* act_scale, int8_t* xq,
+                                 int64_t* n_clipped, sq_stream stream);
+
+/*
+ * sq_gemm_workspace_bytes -- device scratch sq_gemm_w8a8 needs for this
+ * shape (0 when it needs none).  The small-M (decode) path splits K across
+ * SMs and reduces exact INT32 partial sums in the workspace.
+ */
+size_t sq_gemm_workspace_bytes(int64_t M, int64_t N, int64_t K);
+
+/*
+ * sq_gemm_w8a8 -- INT8 GEMM with dequantizing epilogue ([review] §2.6 Fig. 3:
+ * scales only on the outer dimensions; [embedded] §三: integer inner product,
+ * then one float rescale per output):
+ *
+ *   acc[t,n] = sum_k xq[t,k] * wq[n,k]                 (exact INT32)
+ *   y[t,n]   = (float)acc[t,n] * (as_t * w_scale[n])   (fp32, RNE)
+ *   as_t     = act_scale[t] if act_per_token else act_scale[0]
+ *
+ *   xq [M,K] int8; wq [N,K] int8; w_scale [N] fp32;
+ *   y  [M,N] of type yt (SQ_F32, or SQ_BF16 = RNE of the fp32 value);
+ *   acc_out: NULL, or [M,N] int32 that receives the accumulators.
+ *   workspace: at least sq_gemm_workspace_bytes(M,N,K) bytes of device
+ *   memory (may be NULL when that is 0).  It must be ZERO-FILLED before its
+ *   first use; every call that completes without a device error leaves it
+ *   zero-filled again.  Two calls that share a workspace must not run
+ *   concurrently.
+ */
+sq_status sq_gemm_w8a8(const int8_t* xq, const int8_t* wq, int64_t M,
+                       int64_t N, int64_t K, const float* act_scale,
+                       int act_per_token, const float* w_scale, void* y,
+                       sq_dtype yt, int32_t* acc_out, void* workspace,
+                       size_t workspace_bytes, sq_stream stream);
+
+/*
+ * sq_sync_status -- synchronize `stream`, then return and clear the status
+ * word of the current device: SQ_OK, or SQ_ERR_TIMEOUT when a kernel gave up
+ * a bounded wait (its outputs are then undefined, and a GEMM workspace it
+ * used must be zero-filled again), or SQ_ERR_CUDA when the synchronization
+ * itself failed.
+ */
+sq_status sq_sync_status(sq_stream stream);
+
+/* Static description of a status code (never NULL). */
+const char* sq_status_string(sq_status st);
+
+/* Description of the last host-side error on the calling thread ("" if none). */
+const char* sq_last_error(void);
+
+/*
+ * sq_selftest_bounded_wait -- exercises the device-side timeout path without
+ * any fault: launches one CTA that waits on an mbarrier nothing arrives at,
+ * with a wait limit of `limit_ns` nanoseconds (1 .. 10^9).  The wait runs out,
+ * the kernel records SQ_ERR_TIMEOUT in the status word and returns normally;
+ * sq_sync_status() then reports it.  Used by the fault-detection tests.
+ */
+sq_status sq_selftest_bounded_wait(int64_t limit_ns, sq_stream stream);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* SQ_H */

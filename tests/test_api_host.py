@@ -1,0 +1,134 @@
+"""Host-side checks of the C ABI: the library loads, exports every entry point
+include/sq.h declares, and rejects bad arguments before anything reaches the
+GPU (no device is needed: every call here fails or is empty before the
+first CUDA call)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from w8a8_int8_gemm_calib_b200 import _lib
+
+    return _lib
+
+
+def declared_functions():
+    src = open(os.path.join(ROOT, "include", "sq.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(sq_[a-z0-9_]+)\s*\(", src)))
+
+
+def test_exports_every_declared_symbol(lib):
+    names = declared_functions()
+    assert "sq_gemm_w8a8" in names and len(names) >= 10
+    raw = ctypes.CDLL(lib.LIB_PATH)
+    for n in names:
+        assert hasattr(raw, n), f"{n} declared in include/sq.h but not exported"
+    assert set(names) == set(lib.EXPORTS)
+
+
+def test_status_strings(lib):
+    for code in range(9):
+        assert lib.status_string(code).startswith("SQ_")
+    assert lib.status_string(42) == "SQ_ERR_UNKNOWN"
+
+
+# fake, never dereferenced device addresses
+A = 1 << 20
+A2 = (1 << 20) + 4096
+MIS = (1 << 20) + 8
+
+
+def test_calib_absmax_checks(lib):
+    L = lib.lib
+    assert L.sq_calib_absmax(A, 1, 10, 17, None, None, 1e-5, A2, None) == lib.SQ_ERR_SHAPE
+    assert L.sq_calib_absmax(A, 1, 10, 0, None, None, 1e-5, A2, None) == lib.SQ_ERR_SHAPE
+    assert L.sq_calib_absmax(A, 1, 10, 133152, None, None, 1e-5, A2, None) == lib.SQ_ERR_SHAPE
+    assert L.sq_calib_absmax(A, 1, -1, 16, None, None, 1e-5, A2, None) == lib.SQ_ERR_SHAPE
+    assert L.sq_calib_absmax(A, 7, 10, 16, None, None, 1e-5, A2, None) == lib.SQ_ERR_DTYPE
+    assert L.sq_calib_absmax(None, 1, 10, 16, None, None, 1e-5, A2, None) == lib.SQ_ERR_INVALID_ARG
+    assert L.sq_calib_absmax(MIS, 1, 10, 16, None, None, 1e-5, A2, None) == lib.SQ_ERR_ALIGN
+    assert L.sq_calib_absmax(A, 1, 10, 16, None, A2, 1e-5, A2, None) == lib.SQ_ERR_INVALID_ARG
+    assert L.sq_calib_absmax(A, 1, 10, 16, A2, None, -1.0, A2, None) == lib.SQ_ERR_INVALID_ARG
+    assert "multiple of 16" in (L.sq_calib_absmax(A, 1, 1, 24, None, None, 0, A2, None)
+                                and lib.last_error())
+    # empty problem: nothing to do, nothing launched
+    assert L.sq_calib_absmax(A, 1, 0, 16, None, None, 1e-5, A2, None) == lib.SQ_OK
+
+
+def test_smooth_scales_checks(lib):
+    L = lib.lib
+    for bad_alpha in (-0.1, 1.5, float("nan")):
+        assert L.sq_smooth_scales(A, A, 1, 4, 16, bad_alpha, A2, A2, None, None) == \
+            lib.SQ_ERR_INVALID_ARG
+    assert L.sq_smooth_scales(A, A, 1, 4, 20, 0.5, A2, A2, None, None) == lib.SQ_ERR_SHAPE
+    assert L.sq_smooth_scales(A, A, 1, 4, 16, 0.5, None, A2, None, None) == lib.SQ_ERR_INVALID_ARG
+    assert L.sq_smooth_scales(A, A, 1, 4, 16, 0.5, A2, A2, MIS, None) == lib.SQ_ERR_ALIGN
+
+
+def test_fuse_weights_checks(lib):
+    L = lib.lib
+    assert L.sq_fuse_weights_q8(A, 1, 4, 16, None, A2, A2, None, None, None, None, None) == \
+        lib.SQ_ERR_INVALID_ARG
+    assert L.sq_fuse_weights_q8(A, 1, 4, 16, A, None, A2, None, None, None, None, None) == \
+        lib.SQ_ERR_INVALID_ARG
+    assert L.sq_fuse_weights_q8(A, 1, -4, 16, A, A2, A2, None, None, None, None, None) == \
+        lib.SQ_ERR_SHAPE
+    assert L.sq_fuse_weights_q8(A, 1, 4, 16, A, A2, A2, MIS, None, None, None, None) == \
+        lib.SQ_ERR_ALIGN
+
+
+def test_quant_act_checks(lib):
+    L = lib.lib
+    assert L.sq_ln_smooth_quant_act(A, 1, 4, 16, None, None, 1e-5, None, 9, A2, A2, None,
+                                    None) == lib.SQ_ERR_INVALID_ARG
+    assert L.sq_ln_smooth_quant_act(A, 1, 4, 16, A, None, 1e-5, A2, 1, A2, A2, None,
+                                    None) == lib.SQ_ERR_INVALID_ARG
+    assert L.sq_ln_smooth_quant_act(A, 1, 4, 16, None, None, 1e-5, None, 1, A2, A2, A + 4,
+                                    None) == lib.SQ_ERR_ALIGN
+    assert L.sq_ln_smooth_quant_act(A, 1, 4, 40, None, None, 1e-5, None, 1, A2, A2, None,
+                                    None) == lib.SQ_ERR_SHAPE
+    assert L.sq_ln_smooth_quant_act(A, 1, 0, 16, None, None, 1e-5, None, 1, A2, A2, None,
+                                    None) == lib.SQ_OK
+
+
+def test_gemm_checks(lib):
+    L = lib.lib
+    assert L.sq_gemm_w8a8(A, A, 4, 4, 24, A2, 1, A2, A2, 1, None, None, 0, None) == \
+        lib.SQ_ERR_SHAPE
+    assert L.sq_gemm_w8a8(A, A, 4, 4, 16, A2, 1, A2, A2, 5, None, None, 0, None) == \
+        lib.SQ_ERR_DTYPE
+    assert L.sq_gemm_w8a8(A, None, 4, 4, 16, A2, 1, A2, A2, 1, None, None, 0, None) == \
+        lib.SQ_ERR_INVALID_ARG
+    assert L.sq_gemm_w8a8(A, A, 4, 4, 16, A2, 1, A2, MIS, 1, None, None, 0, None) == \
+        lib.SQ_ERR_ALIGN
+    assert L.sq_gemm_w8a8(A, A, 4, 4, 16, A2, 1, A2, A2, 1, MIS, None, 0, None) == \
+        lib.SQ_ERR_ALIGN
+    assert L.sq_gemm_w8a8(A, A, 0, 4, 16, A2, 1, A2, A2, 1, None, None, 0, None) == lib.SQ_OK
+    assert L.sq_gemm_w8a8(A, A, 4, 0, 16, A2, 1, A2, A2, 1, None, None, 0, None) == lib.SQ_OK
+    assert L.sq_gemm_workspace_bytes(0, 5, 16) == 0
+
+
+def test_selftest_checks(lib):
+    L = lib.lib
+    assert L.sq_selftest_bounded_wait(0, None) == lib.SQ_ERR_INVALID_ARG
+    assert L.sq_selftest_bounded_wait(2_000_000_000, None) == lib.SQ_ERR_INVALID_ARG
+
+
+def test_binding_fails_loudly_without_library(tmp_path, monkeypatch):
+    """The product path has no fallback: a missing .so is an ImportError."""
+    import importlib.util
+
+    from w8a8_int8_gemm_calib_b200 import _lib as real
+
+    spec = importlib.util.spec_from_file_location("sq_lib_copy", real.__file__)
+    mod = importlib.util.module_from_spec(spec)
+    monkeypatch.setattr(os.path, "exists", lambda p: False if p.endswith(".so") else True)
+    with pytest.raises(ImportError):
+        spec.loader.exec_module(mod)

@@ -1,0 +1,102 @@
+"""GPU parity of the tcgen05 INT8 GEMM + dequantizing epilogue against the
+oracle: INT32 accumulators and outputs (fp32 and bf16) bit for bit, on tiny
+ragged shapes, multi-tile shapes with ragged tails, and the int8 extremes."""
+import numpy as np
+import pytest
+
+from tests._util import assert_bits_equal, dev, host
+
+pytestmark = pytest.mark.gpu
+
+torch = pytest.importorskip("torch")
+
+
+@pytest.fixture(scope="module")
+def sq():
+    if not torch.cuda.is_available():
+        pytest.skip("needs a CUDA device")
+    import w8a8_int8_gemm_calib_b200 as m
+
+    return m
+
+
+def _operands(M, N, K, seed):
+    r = np.random.default_rng(seed)
+    xq = r.integers(-127, 128, (M, K)).astype(np.int8)
+    wq = r.integers(-127, 128, (N, K)).astype(np.int8)
+    act = r.uniform(1e-3, 0.1, M).astype(np.float32)
+    ws = r.uniform(1e-4, 1e-2, N).astype(np.float32)
+    return xq, wq, act, ws
+
+
+def _run(sq, xq, wq, act, ws, per_token, out, acc=True, workspace=None):
+    M, N = xq.shape[0], wq.shape[0]
+    y = torch.empty((M, N), dtype=torch.bfloat16 if out == "bf16" else torch.float32,
+                    device="cuda")
+    a = torch.empty((M, N), dtype=torch.int32, device="cuda") if acc else None
+    act_d = dev(act if per_token else act[:1])
+    sq.sq_gemm_w8a8(dev(xq), dev(wq), act_d, dev(ws), y, per_token=per_token, acc_out=a,
+                    workspace=workspace)
+    sq.sq_sync_status()
+    return host(y), (host(a) if acc else None)
+
+
+SHAPES = [(1, 1, 16), (3, 17, 48), (17, 255, 1040), (128, 256, 128), (129, 257, 144),
+          (255, 300, 4096), (1, 4096, 4096), (8, 1000, 2064), (200, 512, 272),
+          (384, 768, 256)]
+
+
+@pytest.mark.parametrize("M,N,K", SHAPES)
+@pytest.mark.parametrize("out", ["f32", "bf16"])
+def test_gemm_small_shapes(sq, orc, M, N, K, out):
+    xq, wq, act, ws = _operands(M, N, K, M * 131 + N * 7 + K)
+    y_want, acc_want = orc.gemm_w8a8(xq, wq, act, ws, per_token=True, out_bf16=(out == "bf16"))
+    y, acc = _run(sq, xq, wq, act, ws, True, out, workspace=sq.Workspace())
+    assert_bits_equal(acc, acc_want, "acc")
+    assert_bits_equal(y, y_want, "y")
+
+
+@pytest.mark.parametrize("out", ["f32", "bf16"])
+def test_gemm_per_tensor_scale(sq, orc, out):
+    M, N, K = 70, 130, 512
+    xq, wq, act, ws = _operands(M, N, K, 99)
+    y_want, acc_want = orc.gemm_w8a8(xq, wq, act[:1], ws, per_token=False,
+                                     out_bf16=(out == "bf16"))
+    y, acc = _run(sq, xq, wq, act, ws, False, out, workspace=sq.Workspace())
+    assert_bits_equal(acc, acc_want, "acc")
+    assert_bits_equal(y, y_want, "y")
+
+
+def test_gemm_extremes(sq, orc):
+    """+-127 everywhere at the largest K of the workloads (20480): the INT32
+    accumulators reach +-330,321,920 exactly."""
+    M, N, K = 130, 260, 20480
+    xq = np.full((M, K), 127, np.int8)
+    wq = np.full((N, K), 127, np.int8)
+    wq[1::2] = -127
+    xq[5, ::2] = -127
+    act = np.full(M, 0.01, np.float32)
+    ws = np.full(N, 0.001, np.float32)
+    y_want, acc_want = orc.gemm_w8a8(xq, wq, act, ws)
+    y, acc = _run(sq, xq, wq, act, ws, True, "f32", workspace=sq.Workspace())
+    assert acc[0, 0] == 330321920 and acc[0, 1] == -330321920
+    assert_bits_equal(acc, acc_want, "acc")
+    assert_bits_equal(y, y_want, "y")
+
+
+def test_gemm_without_acc_dump(sq, orc):
+    M, N, K = 300, 520, 1024
+    xq, wq, act, ws = _operands(M, N, K, 5)
+    y_want, _ = orc.gemm_w8a8(xq, wq, act, ws, out_bf16=True)
+    y, _ = _run(sq, xq, wq, act, ws, True, "bf16", acc=False, workspace=sq.Workspace())
+    assert_bits_equal(y, y_want, "y")
+
+
+def test_gemm_is_deterministic(sq):
+    M, N, K = 515, 1030, 2048
+    xq, wq, act, ws = _operands(M, N, K, 6)
+    ws_buf = sq.Workspace()
+    y1, a1 = _run(sq, xq, wq, act, ws, True, "bf16", workspace=ws_buf)
+    y2, a2 = _run(sq, xq, wq, act, ws, True, "bf16", workspace=ws_buf)
+    assert_bits_equal(a1, a2, "acc rerun")
+    assert_bits_equal(y1, y2, "y rerun")

@@ -1,0 +1,265 @@
+// api.cpp -- the C ABI (include/sq.h): argument checks, then dispatch to the
+// kernel launchers.  Nothing is enqueued when a check fails.
+#include <cuda_runtime.h>
+#include <math.h>
+#include <stdarg.h>
+#include <stdio.h>
+#include <string.h>
+
+#include "sq_internal.h"
+
+namespace sq {
+
+namespace {
+thread_local char g_last_error[512] = "";
+constexpr int64_t kMaxK = 133136;  // 127*127*K < 2^31
+
+bool aligned16(const void* p) { return (((uintptr_t)p) & 15u) == 0; }
+
+sq_status check_dtype(sq_dtype t, const char* what) {
+  if (t != SQ_F32 && t != SQ_BF16) return fail(SQ_ERR_DTYPE, "%s: unknown dtype %d", what, (int)t);
+  return SQ_OK;
+}
+
+sq_status check_k(int64_t K, const char* fn) {
+  if (K < 16 || K > kMaxK || (K % 16) != 0)
+    return fail(SQ_ERR_SHAPE, "%s: K=%lld must be a multiple of 16 in [16, %lld]", fn,
+                (long long)K, (long long)kMaxK);
+  return SQ_OK;
+}
+
+#define SQ_REQ(ptr, fn)                                                                \
+  do {                                                                                 \
+    if (!(ptr)) return fail(SQ_ERR_INVALID_ARG, "%s: %s must not be NULL", fn, #ptr); \
+    if (!aligned16(ptr))                                                               \
+      return fail(SQ_ERR_ALIGN, "%s: %s is not 16-byte aligned", fn, #ptr);          \
+  } while (0)
+#define SQ_OPT(ptr, fn)                                                       \
+  do {                                                                        \
+    if ((ptr) && !aligned16(ptr))                                             \
+      return fail(SQ_ERR_ALIGN, "%s: %s is not 16-byte aligned", fn, #ptr); \
+  } while (0)
+#define SQ_TRY(expr)                 \
+  do {                               \
+    sq_status _st = (expr);          \
+    if (_st != SQ_OK) return _st;    \
+  } while (0)
+
+sq_status cuda_fail(cudaError_t e, const char* fn) {
+  return fail(SQ_ERR_CUDA, "%s: %s", fn, cudaGetErrorString(e));
+}
+
+}  // namespace
+
+sq_status fail(sq_status st, const char* fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(g_last_error, sizeof g_last_error, fmt, ap);
+  va_end(ap);
+  return st;
+}
+
+}  // namespace sq
+
+using namespace sq;
+
+extern "C" {
+
+sq_status sq_calib_absmax(const void* x, sq_dtype xt, int64_t T, int64_t K,
+                          const float* ln_gamma, const float* ln_beta, float ln_eps,
+                          float* amax, sq_stream stream) {
+  const char* fn = "sq_calib_absmax";
+  g_last_error[0] = 0;
+  SQ_TRY(check_dtype(xt, fn));
+  if (T < 0) return fail(SQ_ERR_SHAPE, "%s: T=%lld < 0", fn, (long long)T);
+  SQ_TRY(check_k(K, fn));
+  SQ_REQ(x, fn);
+  SQ_REQ(amax, fn);
+  SQ_OPT(ln_gamma, fn);
+  SQ_OPT(ln_beta, fn);
+  if (ln_beta && !ln_gamma) return fail(SQ_ERR_INVALID_ARG, "%s: ln_beta given without ln_gamma", fn);
+  if (ln_gamma && !(ln_eps >= 0.0f && isfinite(ln_eps)))
+    return fail(SQ_ERR_INVALID_ARG, "%s: ln_eps must be finite and >= 0", fn);
+  if (T == 0) return SQ_OK;
+  cudaStream_t st = (cudaStream_t)stream;
+  cudaError_t e;
+  if (!ln_gamma) {
+    e = launch_colmax(x, xt, T, K, amax, st);
+  } else {
+    RowArgs a{};
+    a.x = x; a.T = T; a.K = K; a.g = ln_gamma; a.b = ln_beta; a.eps = ln_eps;
+    a.colmax = amax;
+    e = launch_row(a, xt, ROW_COLMAX, st);
+  }
+  return e == cudaSuccess ? SQ_OK : cuda_fail(e, fn);
+}
+
+sq_status sq_smooth_scales(const float* amax_x, const void* w, sq_dtype wt, int64_t N, int64_t K,
+                           float alpha, float* s, float* inv_s, float* act_delta_static,
+                           sq_stream stream) {
+  const char* fn = "sq_smooth_scales";
+  g_last_error[0] = 0;
+  SQ_TRY(check_dtype(wt, fn));
+  if (N < 0) return fail(SQ_ERR_SHAPE, "%s: N=%lld < 0", fn, (long long)N);
+  SQ_TRY(check_k(K, fn));
+  if (!(alpha >= 0.0f && alpha <= 1.0f))
+    return fail(SQ_ERR_INVALID_ARG, "%s: alpha=%g must lie in [0, 1]", fn, (double)alpha);
+  SQ_REQ(amax_x, fn);
+  SQ_REQ(s, fn);
+  SQ_REQ(inv_s, fn);
+  SQ_OPT(act_delta_static, fn);
+  if (N > 0) SQ_REQ(w, fn);
+  cudaStream_t st = (cudaStream_t)stream;
+  // s first holds the weight column peaks (running max from 0)
+  cudaError_t e = cudaMemsetAsync(s, 0, (size_t)K * sizeof(float), st);
+  if (e == cudaSuccess && N > 0) e = launch_colmax(w, wt, N, K, s, st);
+  if (e == cudaSuccess) e = launch_scales(amax_x, K, alpha, s, inv_s, act_delta_static, st);
+  return e == cudaSuccess ? SQ_OK : cuda_fail(e, fn);
+}
+
+sq_status sq_fuse_weights_q8(const void* w, sq_dtype wt, int64_t N, int64_t K, const float* s,
+                             int8_t* wq, float* w_scale, const float* gamma, const float* beta,
+                             float* gamma_out, float* beta_out, sq_stream stream) {
+  const char* fn = "sq_fuse_weights_q8";
+  g_last_error[0] = 0;
+  SQ_TRY(check_dtype(wt, fn));
+  if (N < 0) return fail(SQ_ERR_SHAPE, "%s: N=%lld < 0", fn, (long long)N);
+  SQ_TRY(check_k(K, fn));
+  SQ_REQ(s, fn);
+  SQ_OPT(gamma, fn);
+  SQ_OPT(beta, fn);
+  SQ_OPT(gamma_out, fn);
+  SQ_OPT(beta_out, fn);
+  if (N > 0) {
+    SQ_REQ(w, fn);
+    SQ_REQ(wq, fn);
+    SQ_REQ(w_scale, fn);
+  }
+  cudaStream_t st = (cudaStream_t)stream;
+  cudaError_t e = cudaSuccess;
+  if (N > 0) {
+    // W_hat = W * s, then per-row (output channel) dynamic INT8: the same
+    // row quantizer as the activations, with s as the column multiplier
+    RowArgs a{};
+    a.x = w; a.T = N; a.K = K; a.mul = s; a.scale = w_scale; a.q = wq;
+    e = launch_row(a, wt, ROW_DYNAMIC, st);
+  }
+  const bool fold_g = gamma && gamma_out, fold_b = beta && beta_out;
+  if (e == cudaSuccess && (fold_g || fold_b))
+    e = launch_fold_ln(gamma, beta, s, K, fold_g ? gamma_out : nullptr,
+                       fold_b ? beta_out : nullptr, st);
+  return e == cudaSuccess ? SQ_OK : cuda_fail(e, fn);
+}
+
+sq_status sq_ln_smooth_quant_act(const void* x, sq_dtype xt, int64_t T, int64_t K,
+                                 const float* gamma_s, const float* beta_s, float ln_eps,
+                                 const float* inv_s, sq_act_gran gran, float* act_scale,
+                                 int8_t* xq, int64_t* n_clipped, sq_stream stream) {
+  const char* fn = "sq_ln_smooth_quant_act";
+  g_last_error[0] = 0;
+  SQ_TRY(check_dtype(xt, fn));
+  if (gran != SQ_ACT_PER_TENSOR_STATIC && gran != SQ_ACT_PER_TOKEN_DYNAMIC)
+    return fail(SQ_ERR_INVALID_ARG, "%s: unknown granularity %d", fn, (int)gran);
+  if (T < 0) return fail(SQ_ERR_SHAPE, "%s: T=%lld < 0", fn, (long long)T);
+  SQ_TRY(check_k(K, fn));
+  SQ_REQ(x, fn);
+  SQ_REQ(xq, fn);
+  SQ_REQ(act_scale, fn);
+  SQ_OPT(gamma_s, fn);
+  SQ_OPT(beta_s, fn);
+  SQ_OPT(inv_s, fn);
+  if (n_clipped && (((uintptr_t)n_clipped) & 7u))
+    return fail(SQ_ERR_ALIGN, "%s: n_clipped is not 8-byte aligned", fn);
+  if (beta_s && !gamma_s) return fail(SQ_ERR_INVALID_ARG, "%s: beta_s given without gamma_s", fn);
+  if (gamma_s && inv_s)
+    return fail(SQ_ERR_INVALID_ARG, "%s: inv_s is folded into gamma_s/beta_s when a LayerNorm precedes; pass one of them", fn);
+  if (gamma_s && !(ln_eps >= 0.0f && isfinite(ln_eps)))
+    return fail(SQ_ERR_INVALID_ARG, "%s: ln_eps must be finite and >= 0", fn);
+  if (T == 0) return SQ_OK;
+  RowArgs a{};
+  a.x = x; a.T = T; a.K = K; a.g = gamma_s; a.b = beta_s; a.eps = ln_eps; a.mul = inv_s;
+  a.scale = act_scale; a.q = xq; a.n_clipped = (unsigned long long*)n_clipped;
+  cudaError_t e = launch_row(a, xt, gran == SQ_ACT_PER_TOKEN_DYNAMIC ? ROW_DYNAMIC : ROW_STATIC,
+                             (cudaStream_t)stream);
+  return e == cudaSuccess ? SQ_OK : cuda_fail(e, fn);
+}
+
+size_t sq_gemm_workspace_bytes(int64_t M, int64_t N, int64_t K) {
+  if (M <= 0 || N <= 0 || K <= 0) return 0;
+  return gemm_workspace_bytes(M, N, K);
+}
+
+sq_status sq_gemm_w8a8(const int8_t* xq, const int8_t* wq, int64_t M, int64_t N, int64_t K,
+                       const float* act_scale, int act_per_token, const float* w_scale, void* y,
+                       sq_dtype yt, int32_t* acc_out, void* workspace, size_t workspace_bytes,
+                       sq_stream stream) {
+  const char* fn = "sq_gemm_w8a8";
+  g_last_error[0] = 0;
+  SQ_TRY(check_dtype(yt, fn));
+  if (M < 0 || N < 0) return fail(SQ_ERR_SHAPE, "%s: M=%lld N=%lld must be >= 0", fn,
+                                  (long long)M, (long long)N);
+  SQ_TRY(check_k(K, fn));
+  if (M == 0 || N == 0) return SQ_OK;
+  if (M > (int64_t)1 << 31 || N > (int64_t)1 << 31)
+    return fail(SQ_ERR_SHAPE, "%s: M and N must be below 2^31", fn);
+  SQ_REQ(xq, fn);
+  SQ_REQ(wq, fn);
+  SQ_REQ(act_scale, fn);
+  SQ_REQ(w_scale, fn);
+  SQ_REQ(y, fn);
+  SQ_OPT(acc_out, fn);
+  const size_t need = gemm_workspace_bytes(M, N, K);
+  if (need) {
+    if (!workspace || workspace_bytes < need)
+      return fail(SQ_ERR_WORKSPACE, "%s: workspace of %zu bytes needed, %zu given", fn, need,
+                  workspace ? workspace_bytes : (size_t)0);
+    SQ_OPT(workspace, fn);
+  }
+  GemmArgs a{};
+  a.xq = xq; a.wq = wq; a.M = M; a.N = N; a.K = K; a.act_scale = act_scale;
+  a.act_per_token = act_per_token ? 1 : 0; a.w_scale = w_scale; a.y = y; a.yt = yt;
+  a.acc_out = acc_out; a.workspace = workspace; a.workspace_bytes = workspace_bytes;
+  return launch_gemm(a, (cudaStream_t)stream);
+}
+
+sq_status sq_sync_status(sq_stream stream) {
+  g_last_error[0] = 0;
+  cudaError_t e = cudaStreamSynchronize((cudaStream_t)stream);
+  if (e != cudaSuccess) return cuda_fail(e, "sq_sync_status");
+  unsigned int* sw = status_word();
+  if (!sw) return fail(SQ_ERR_CUDA, "sq_sync_status: status word unavailable");
+  unsigned int v = 0;
+  e = cudaMemcpy(&v, sw, sizeof v, cudaMemcpyDeviceToHost);
+  if (e == cudaSuccess && v) e = cudaMemset(sw, 0, sizeof v);
+  if (e != cudaSuccess) return cuda_fail(e, "sq_sync_status");
+  if (v) return fail((sq_status)v, "sq_sync_status: a kernel reported %s",
+                     sq_status_string((sq_status)v));
+  return SQ_OK;
+}
+
+const char* sq_status_string(sq_status s) {
+  switch (s) {
+    case SQ_OK: return "SQ_OK";
+    case SQ_ERR_INVALID_ARG: return "SQ_ERR_INVALID_ARG";
+    case SQ_ERR_SHAPE: return "SQ_ERR_SHAPE";
+    case SQ_ERR_ALIGN: return "SQ_ERR_ALIGN";
+    case SQ_ERR_DTYPE: return "SQ_ERR_DTYPE";
+    case SQ_ERR_UNSUPPORTED: return "SQ_ERR_UNSUPPORTED";
+    case SQ_ERR_CUDA: return "SQ_ERR_CUDA";
+    case SQ_ERR_TIMEOUT: return "SQ_ERR_TIMEOUT";
+    case SQ_ERR_WORKSPACE: return "SQ_ERR_WORKSPACE";
+  }
+  return "SQ_ERR_UNKNOWN";
+}
+
+const char* sq_last_error(void) { return g_last_error; }
+
+sq_status sq_selftest_bounded_wait(int64_t limit_ns, sq_stream stream) {
+  g_last_error[0] = 0;
+  if (limit_ns < 1 || limit_ns > 1000000000)
+    return fail(SQ_ERR_INVALID_ARG, "sq_selftest_bounded_wait: limit_ns must be in [1, 1e9]");
+  cudaError_t e = launch_wait_selftest(limit_ns, (cudaStream_t)stream);
+  return e == cudaSuccess ? SQ_OK : cuda_fail(e, "sq_selftest_bounded_wait");
+}
+
+}  // extern "C"

@@ -1,0 +1,91 @@
+// sq_device.cuh -- small device helpers shared by the kernel files.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace sq {
+
+// Device status codes written to the status word (values of sq_status).
+constexpr unsigned kStatusTimeout = 7u;
+
+__device__ __forceinline__ void set_status(unsigned int* status, unsigned code) {
+  if (status) atomicCAS(status, 0u, code);
+}
+
+// bf16 -> fp32 is exact: the bf16 pattern is the upper half of the fp32 one.
+__device__ __forceinline__ float bf16lo(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float bf16hi(uint32_t w) { return __uint_as_float(w & 0xffff0000u); }
+
+// One 8-element chunk of an fp32 or bf16 row, in its storage form.
+template <typename T> struct Raw8;
+template <> struct Raw8<float> { float4 a, b; };
+template <> struct Raw8<uint16_t> { uint4 a; };
+
+// Streaming (read-once) loads: do not keep the line in L1.
+__device__ __forceinline__ uint4 ld_stream_u4(const void* p) {
+  uint4 r;
+  asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w) : "l"(p));
+  return r;
+}
+
+__device__ __forceinline__ void load_raw(const float* p, Raw8<float>& r) {
+  uint4 a = ld_stream_u4(p), b = ld_stream_u4(p + 4);
+  r.a = make_float4(__uint_as_float(a.x), __uint_as_float(a.y), __uint_as_float(a.z), __uint_as_float(a.w));
+  r.b = make_float4(__uint_as_float(b.x), __uint_as_float(b.y), __uint_as_float(b.z), __uint_as_float(b.w));
+}
+__device__ __forceinline__ void load_raw(const uint16_t* p, Raw8<uint16_t>& r) {
+  r.a = ld_stream_u4(p);
+}
+
+// Cached loads (rows read more than once).
+__device__ __forceinline__ void load_raw_cached(const float* p, Raw8<float>& r) {
+  r.a = __ldg(reinterpret_cast<const float4*>(p));
+  r.b = __ldg(reinterpret_cast<const float4*>(p) + 1);
+}
+__device__ __forceinline__ void load_raw_cached(const uint16_t* p, Raw8<uint16_t>& r) {
+  r.a = __ldg(reinterpret_cast<const uint4*>(p));
+}
+
+__device__ __forceinline__ void unpack(const Raw8<float>& r, float (&v)[8]) {
+  v[0] = r.a.x; v[1] = r.a.y; v[2] = r.a.z; v[3] = r.a.w;
+  v[4] = r.b.x; v[5] = r.b.y; v[6] = r.b.z; v[7] = r.b.w;
+}
+__device__ __forceinline__ void unpack(const Raw8<uint16_t>& r, float (&v)[8]) {
+  v[0] = bf16lo(r.a.x); v[1] = bf16hi(r.a.x);
+  v[2] = bf16lo(r.a.y); v[3] = bf16hi(r.a.y);
+  v[4] = bf16lo(r.a.z); v[5] = bf16hi(r.a.z);
+  v[6] = bf16lo(r.a.w); v[7] = bf16hi(r.a.w);
+}
+
+// 8 consecutive fp32 parameters (gamma, beta, multipliers), L1-cached.
+__device__ __forceinline__ void load8(const float* p, float (&v)[8]) {
+  float4 a = __ldg(reinterpret_cast<const float4*>(p));
+  float4 b = __ldg(reinterpret_cast<const float4*>(p) + 1);
+  v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
+  v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
+}
+
+// Q(y; Delta) given 1/Delta: round half to even (cvt.rni: NaN -> 0,
+// +-inf -> saturated), then clamp to the symmetric range [-127, 127].
+__device__ __forceinline__ int quant_code(float y, float inv, unsigned& clipped) {
+  int q = __float2int_rn(__fmul_rn(y, inv));
+  clipped += (q > 127) | (q < -127);
+  return max(-127, min(127, q));
+}
+
+__device__ __forceinline__ uint32_t pack4(int a, int b, int c, int d) {
+  uint32_t lo = __byte_perm((uint32_t)a, (uint32_t)b, 0x0040);  // a.b0, b.b0 -> bytes 0,1
+  uint32_t hi = __byte_perm((uint32_t)c, (uint32_t)d, 0x0040);
+  return __byte_perm(lo, hi, 0x5410);
+}
+
+// Bounded-wait clock: nanoseconds from the global timer.
+__device__ __forceinline__ uint64_t global_ns() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+
+}  // namespace sq

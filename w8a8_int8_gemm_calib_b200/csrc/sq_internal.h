@@ -1,0 +1,76 @@
+// sq_internal.h -- declarations shared by the C-ABI layer (api.cpp) and the
+// kernel translation units.  Not part of the public interface (include/sq.h).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/sq.h"
+
+namespace sq {
+
+// Device address of the per-device status word (a static __device__
+// variable in status.cu), looked up once per device.  NULL on failure.
+unsigned int* status_word();
+
+// Number of SMs of the current device (cached per device).
+int sm_count();
+
+// Record a one-line host-side error for sq_last_error() and return `st`.
+sq_status fail(sq_status st, const char* fmt, ...);
+
+// ---------------------------------------------------------------- row ops
+// Column absmax: out[k] = max(out[k], max_t |x[t,k]|) (out as fp32 bits,
+// atomic max).  K % 8 == 0.
+cudaError_t launch_colmax(const void* x, sq_dtype xt, int64_t T, int64_t K,
+                          float* out, cudaStream_t st);
+
+enum RowMode { ROW_DYNAMIC = 0, ROW_STATIC = 1, ROW_COLMAX = 2 };
+
+struct RowArgs {
+  const void* x;
+  int64_t T, K;
+  const float* g;      // LayerNorm gamma (NULL: no LayerNorm)
+  const float* b;      // LayerNorm beta (may be NULL)
+  float eps;
+  const float* mul;    // per-column multiplier when there is no LayerNorm (may be NULL)
+  float* scale;        // ROW_DYNAMIC: out [T]; ROW_STATIC: in [1]
+  int8_t* q;           // [T,K] codes out (quantizing modes)
+  unsigned long long* n_clipped;  // may be NULL
+  float* colmax;       // ROW_COLMAX: running max [K] (fp32 bits, atomic max)
+};
+
+cudaError_t launch_row(const RowArgs& a, sq_dtype xt, RowMode mode,
+                       cudaStream_t st);
+
+// s / inv_s from amax_x and the weight column peaks held (as fp32) in s.
+cudaError_t launch_scales(const float* amax_x, int64_t K, float alpha,
+                          float* s, float* inv_s, float* delta_out,
+                          cudaStream_t st);
+
+cudaError_t launch_fold_ln(const float* gamma, const float* beta,
+                           const float* s, int64_t K, float* gamma_out,
+                           float* beta_out, cudaStream_t st);
+
+// ---------------------------------------------------------------- GEMM
+struct GemmArgs {
+  const int8_t* xq;
+  const int8_t* wq;
+  int64_t M, N, K;
+  const float* act_scale;
+  int act_per_token;
+  const float* w_scale;
+  void* y;
+  sq_dtype yt;
+  int32_t* acc_out;
+  void* workspace;
+  size_t workspace_bytes;
+};
+
+size_t gemm_workspace_bytes(int64_t M, int64_t N, int64_t K);
+sq_status launch_gemm(const GemmArgs& a, cudaStream_t st);
+
+// ---------------------------------------------------------------- self test
+cudaError_t launch_wait_selftest(int64_t limit_ns, cudaStream_t st);
+
+}  // namespace sq
