@@ -11,9 +11,10 @@ tcgen05 GEMM with the dequantizing epilogue.
                     [--impl reference]
 
 `value` is whole-job throughput in TOPS = 2*M*N*K per step (all ranks) over
-the device time of the timed steps (CUDA events on the launching stream, max
-over ranks); L2 is flushed (a 256 MiB write) before every timed step and the
-flush is outside the timed events.  Inputs are resident in HBM before timing.
+the device time of the timed steps, max over ranks.  Each step is one replay
+of a CUDA graph of the five calls; event nodes inside the graph time the step
+and each call on the device.  L2 is flushed (a 256 MiB write) before every
+timed step, outside the timed events.  Inputs are resident in HBM.
 `e2e` is the same metric through the public Python API with pinned host
 buffers: every step copies its inputs host->device and its output back.
 `--impl reference` times the CPU oracle (tests-only code) on bounded samples
@@ -85,6 +86,7 @@ def config_of(wl, lin, world):
         "act_quant": "per-token dynamic" if lin.per_token else "per-tensor static",
         "io_dtype": lin.dtype,
         "l2": "flushed before every timed step (256 MiB write, outside the timed events)",
+        "timing": "CUDA graph per step, device events around the step and each call",
         "parallelism": f"replicas x{world}",
     }
 
@@ -257,26 +259,34 @@ def run_ours(args):
     for _ in range(max(3, args.warmup)):
         layer.step()
     sq.sq_sync_status()
+    # one CUDA graph per step: the five calls (seven kernels) replay without
+    # host launch gaps; event nodes inside the graph time each call on the
+    # device
+    names = ["calib_absmax", "smooth_scales", "fuse_weights_q8", "ln_smooth_quant_act",
+             "gemm_w8a8"]
+    evs = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(6)]
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        layer.step(evs)
+    for _ in range(max(3, args.warmup)):
+        graph.replay()
     barrier()
 
     K = args.steps
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(6)] for _ in range(K)]
+    per = {n: [] for n in names}
+    step_ms = []
     clocks = ClockSampler(torch.cuda.current_device())
     with clocks:
         barrier()
         for i in range(K):
-            flush.fill_(i)
-            layer.step(evs[i])
+            flush.fill_(i)  # evicts the previous step's data from L2
+            graph.replay()
+            torch.cuda.synchronize()
+            for j, n in enumerate(names):
+                per[n].append(evs[j].elapsed_time(evs[j + 1]))
+            step_ms.append(evs[0].elapsed_time(evs[5]))
         barrier()
     sq.sq_sync_status()
-    names = ["calib_absmax", "smooth_scales", "fuse_weights_q8", "ln_smooth_quant_act",
-             "gemm_w8a8"]
-    per = {n: [] for n in names}
-    step_ms = []
-    for e in evs:
-        for j, n in enumerate(names):
-            per[n].append(e[j].elapsed_time(e[j + 1]))
-        step_ms.append(e[0].elapsed_time(e[5]))
     total_ms = float(sum(step_ms))
     if world > 1:
         t = torch.tensor([total_ms], dtype=torch.float64, device=dev)

@@ -15,7 +15,7 @@ OBJ = os.path.join(HERE, "_build")
 LIB = os.path.join(HERE, "libsq_b200.so")
 INCLUDE = os.path.join(os.path.dirname(HERE), "include")
 
-SOURCES = ["api.cpp", "status.cu", "rowops.cu", "gemm.cu"]
+SOURCES = ["api.cpp", "status.cu", "rowops.cu", "rowpipe.cu", "gemm.cu"]
 HEADERS = ["sq_internal.h", "sq_device.cuh", "tc_ptx.cuh"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 NVCC_FLAGS = ["-O3", "-std=c++17", "-lineinfo", "-Xcompiler", "-fPIC",

@@ -319,13 +319,17 @@ bool make_tmap(CUtensorMap* m, const void* base, uint64_t inner, uint64_t rows, 
 template <bool BF16>
 cudaError_t launch_tc(const CUtensorMap& ta, const CUtensorMap& tb, const Params& p, int grid,
                       cudaStream_t st) {
-  static std::once_flag once;
-  static cudaError_t attr_err = cudaSuccess;
-  std::call_once(once, [] {
-    attr_err = cudaFuncSetAttribute(gemm_w8a8_tc_kernel<BF16>,
-                                    cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_BYTES);
+  static std::once_flag once[64];
+  static cudaError_t attr_err[64];
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess || dev < 0 || dev >= 64) return e != cudaSuccess ? e : cudaErrorInvalidDevice;
+  std::call_once(once[dev], [&] {
+    attr_err[dev] = cudaFuncSetAttribute(gemm_w8a8_tc_kernel<BF16>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)SMEM_BYTES);
   });
-  if (attr_err != cudaSuccess) return attr_err;
+  if (attr_err[dev] != cudaSuccess) return attr_err[dev];
   gemm_w8a8_tc_kernel<BF16><<<grid, THREADS, SMEM_BYTES, st>>>(ta, tb, p);
   return cudaGetLastError();
 }

@@ -17,6 +17,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <mutex>
+
 #include "sq_device.cuh"
 #include "sq_internal.h"
 
@@ -48,12 +50,13 @@ colmax_kernel(const T* __restrict__ x, int64_t T_, int64_t K, int64_t rows_per_s
   if (live) {
     const T* base = x + chunk * 8;
     int64_t r = r0 + warp;
-    for (; r + 3 * kColWarps < r1; r += 4 * kColWarps) {
-      Raw8<T> raw[4];
+    constexpr int U = sizeof(T) == 2 ? 8 : 4;  // 128 B in flight per thread
+    for (; r + (U - 1) * kColWarps < r1; r += U * kColWarps) {
+      Raw8<T> raw[U];
 #pragma unroll
-      for (int u = 0; u < 4; ++u) load_raw(base + (r + u * kColWarps) * K, raw[u]);
+      for (int u = 0; u < U; ++u) load_raw(base + (r + u * kColWarps) * K, raw[u]);
 #pragma unroll
-      for (int u = 0; u < 4; ++u) {
+      for (int u = 0; u < U; ++u) {
         float v[8];
         unpack(raw[u], v);
 #pragma unroll
@@ -84,9 +87,24 @@ colmax_kernel(const T* __restrict__ x, int64_t T_, int64_t K, int64_t rows_per_s
 cudaError_t launch_colmax(const void* x, sq_dtype xt, int64_t T, int64_t K,
                           float* out, cudaStream_t st) {
   const int64_t strips = (K + 255) / 256;
-  const int64_t target = (int64_t)sm_count() * 8;  // one wave of 256-thread CTAs
+  static std::once_flag once[2][64];
+  static int occ[2][64];
+  int dev = 0;
+  cudaError_t de = cudaGetDevice(&dev);
+  if (de != cudaSuccess || dev < 0 || dev >= 64) return de != cudaSuccess ? de : cudaErrorInvalidDevice;
+  const int ti = xt == SQ_BF16 ? 0 : 1;
+  std::call_once(once[ti][dev], [&] {
+    int n = 0;
+    if (xt == SQ_BF16)
+      cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, colmax_kernel<uint16_t>, kColWarps * 32, 0);
+    else
+      cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, colmax_kernel<float>, kColWarps * 32, 0);
+    occ[ti][dev] = n < 1 ? 1 : n;
+  });
+  const int per_sm = occ[ti][dev];
+  const int64_t target = (int64_t)sm_count() * per_sm;  // one wave of CTAs
   int64_t slabs = (target + strips - 1) / strips;
-  const int64_t min_rows = 4 * kColWarps;           // at least one unrolled step
+  const int64_t min_rows = 8 * kColWarps;               // at least one unrolled step
   int64_t maxslabs = (T + min_rows - 1) / min_rows;
   if (slabs > maxslabs) slabs = maxslabs;
   if (slabs < 1) slabs = 1;
@@ -116,8 +134,11 @@ cudaError_t launch_colmax(const void* x, sq_dtype xt, int64_t T, int64_t K,
 // multiply-add per element, (x - mean)^2 + p, in the same order, / K;
 // rstd = 1 / sqrt(var + eps); y = ((x - mean) * rstd) * g + b.
 //
-// MAXC > 0: the thread's chunks of the row are held in registers (at most
-// MAXC of them).  MAXC == 0: every pass re-reads the row (any K).
+// MAXC > 0: the thread's chunks of a row are held in registers (at most MAXC
+// of them) and the next row's chunks are loaded while the current row is
+// processed.  MAXC == 0: every pass re-reads the row (any K).  PREG: the
+// thread's per-column parameters (gamma/beta, or the multiplier) stay in
+// registers for all its rows.
 constexpr int kSlices = 4;
 constexpr int kSliceThreads = 128;
 constexpr size_t kColmaxSmemMax = 192 * 1024;
@@ -137,13 +158,54 @@ __device__ __forceinline__ float warp_max(float p) {
   return p;
 }
 
-template <typename T, int MAXC, bool LN, int MODE, bool COUNT>
+// Calls f(i, c, v[8]) for every chunk the thread owns, in increasing c.
+template <int MAXC, typename T, typename F>
+__device__ __forceinline__ void for_chunks(const Raw8<T> (&raw)[MAXC > 0 ? MAXC : 1],
+                                           const T* xr, int j, int64_t nchunk, F&& f) {
+  if constexpr (MAXC > 0) {
+#pragma unroll
+    for (int i = 0; i < MAXC; ++i) {
+      const int64_t c = j + (int64_t)i * kSliceThreads;
+      if (c < nchunk) {
+        float v[8];
+        unpack(raw[i], v);
+        f(i, c, v);
+      }
+    }
+  } else {
+    int i = 0;
+    for (int64_t c = j; c < nchunk; c += kSliceThreads, ++i) {
+      Raw8<T> r;
+      load_raw_cached(xr + c * 8, r);
+      float v[8];
+      unpack(r, v);
+      f(i, c, v);
+    }
+  }
+}
+
+template <int MAXC, typename T>
+__device__ __forceinline__ void load_row(Raw8<T> (&raw)[MAXC > 0 ? MAXC : 1], const T* xr, int j,
+                                         int64_t nchunk) {
+  if constexpr (MAXC > 0) {
+#pragma unroll
+    for (int i = 0; i < MAXC; ++i) {
+      const int64_t c = j + (int64_t)i * kSliceThreads;
+      if (c < nchunk) load_raw(xr + c * 8, raw[i]);
+    }
+  }
+}
+
+template <typename T, int MAXC, bool LN, int MODE, bool COUNT, bool PREG, bool PF>
 __global__ void __launch_bounds__(kSlices * kSliceThreads)
 row_kernel(RowArgs a) {
   // [slice][parity][reduction][warp]
   __shared__ float red[kSlices][2][3][4];
-  extern __shared__ unsigned int colmax_s[];  // ROW_COLMAX with MAXC == 0: [K]
+  extern __shared__ unsigned int colmax_s[];  // ROW_COLMAX: per-CTA column peaks [K]
 
+  uint32_t dyn_smem;
+  asm("mov.u32 %0, %%dynamic_smem_size;" : "=r"(dyn_smem));
+  const bool use_smem = dyn_smem > 0;
   const int slice = threadIdx.x / kSliceThreads;
   const int j = threadIdx.x % kSliceThreads;
   const int w = j >> 5, lane = j & 31;
@@ -155,23 +217,58 @@ row_kernel(RowArgs a) {
   const float* __restrict__ mul = a.mul;
   const float kf = (float)K;
 
-  uint32_t dyn_smem;
-  asm("mov.u32 %0, %%dynamic_smem_size;" : "=r"(dyn_smem));
-  const bool use_smem = dyn_smem > 0;
   constexpr int CM = MAXC > 0 ? MAXC : 1;
   constexpr int NCMAX = (MODE == ROW_COLMAX && MAXC > 0) ? CM * 8 : 1;
+  constexpr int NP = PREG ? CM * 8 : 1;
   float cmax[NCMAX];
-  if constexpr (MODE == ROW_COLMAX) {
-    if constexpr (MAXC > 0) {
 #pragma unroll
-      for (int i = 0; i < NCMAX; ++i) cmax[i] = 0.0f;
-    } else {
-      if (use_smem) {
-        for (int64_t k = threadIdx.x; k < K; k += blockDim.x) colmax_s[k] = 0u;
-        __syncthreads();
-      }
+  for (int i = 0; i < NCMAX; ++i) cmax[i] = 0.0f;
+  if constexpr (MODE == ROW_COLMAX) {
+    if (use_smem) {
+      for (int64_t k = threadIdx.x; k < K; k += blockDim.x) colmax_s[k] = 0u;
+      __syncthreads();
     }
   }
+
+  // per-column parameters: LN gamma/beta, or the column multiplier
+  float pg[NP], pb[NP];
+  if constexpr (PREG) {
+#pragma unroll
+    for (int i = 0; i < CM; ++i) {
+      const int64_t c = j + (int64_t)i * kSliceThreads;
+      float t0[8], t1[8];
+#pragma unroll
+      for (int e = 0; e < 8; ++e) { t0[e] = 1.0f; t1[e] = 0.0f; }
+      if (c < nchunk) {
+        if (LN) {
+          load8(g + c * 8, t0);
+          if (b) load8(b + c * 8, t1);
+        } else if (mul) {
+          load8(mul + c * 8, t0);
+        }
+      }
+#pragma unroll
+      for (int e = 0; e < 8; ++e) { pg[i * 8 + e] = t0[e]; pb[i * 8 + e] = t1[e]; }
+    }
+  }
+  // parameters of chunk (i, c) into g8/b8
+  auto params = [&](int i, int64_t c, float (&g8)[8], float (&b8)[8]) {
+    if constexpr (PREG) {
+#pragma unroll
+      for (int e = 0; e < 8; ++e) { g8[e] = pg[i * 8 + e]; b8[e] = pb[i * 8 + e]; }
+    } else {
+      if (LN) {
+        load8(g + c * 8, g8);
+        if (b) load8(b + c * 8, b8);
+        else {
+#pragma unroll
+          for (int e = 0; e < 8; ++e) b8[e] = 0.0f;
+        }
+      } else if (mul) {
+        load8(mul + c * 8, g8);
+      }
+    }
+  };
 
   float static_inv = 0.0f;
   if (MODE == ROW_STATIC) static_inv = __fdiv_rn(1.0f, __ldg(a.scale));
@@ -179,44 +276,24 @@ row_kernel(RowArgs a) {
   int parity = 0;
 
   const int64_t stride = (int64_t)gridDim.x * kSlices;
-  for (int64_t row = (int64_t)blockIdx.x * kSlices + slice; row < a.T; row += stride) {
+  int64_t row = (int64_t)blockIdx.x * kSlices + slice;
+  Raw8<T> cur[CM];
+  if (row < a.T) load_row<MAXC>(cur, x + row * K, j, nchunk);
+  while (row < a.T) {
+    const int64_t nrow = row + stride;
+    Raw8<T> nxt[PF ? CM : 1];
+    if constexpr (PF) {
+      if (nrow < a.T) load_row<MAXC>(nxt, x + nrow * K, j, nchunk);
+    }
     const T* xr = x + row * K;
-    Raw8<T> raw[CM];
-    if constexpr (MAXC > 0) {
-#pragma unroll
-      for (int i = 0; i < CM; ++i) {
-        const int64_t c = j + (int64_t)i * kSliceThreads;
-        if (c < nchunk) load_raw(xr + c * 8, raw[i]);
-      }
-    }
-    // element access for pass p: v[8] of chunk i (MAXC>0) or chunk c (MAXC==0)
-#define SQ_CHUNK_LOOP(BODY)                                                     \
-    if constexpr (MAXC > 0) {                                                   \
-      _Pragma("unroll") for (int i = 0; i < CM; ++i) {                          \
-        const int64_t c = j + (int64_t)i * kSliceThreads;                       \
-        if (c < nchunk) {                                                       \
-          float v[8];                                                           \
-          unpack(raw[i], v);                                                    \
-          BODY                                                                  \
-        }                                                                       \
-      }                                                                         \
-    } else {                                                                    \
-      int i = 0;                                                                \
-      for (int64_t c = j; c < nchunk; c += kSliceThreads, ++i) {                \
-        Raw8<T> r1;                                                             \
-        load_raw_cached(xr + c * 8, r1);                                        \
-        float v[8];                                                             \
-        unpack(r1, v);                                                          \
-        BODY                                                                    \
-      }                                                                         \
-    }
 
     float mu = 0.0f, rstd = 0.0f;
     if constexpr (LN) {
       float p = 0.0f;
-      SQ_CHUNK_LOOP({
-        _Pragma("unroll") for (int e = 0; e < 8; ++e) p = __fadd_rn(p, v[e]);
-      })
+      for_chunks<MAXC>(cur, xr, j, nchunk, [&](int, int64_t, const float (&v)[8]) {
+#pragma unroll
+        for (int e = 0; e < 8; ++e) p = __fadd_rn(p, v[e]);
+      });
       p = warp_sum_butterfly(p);
       if (lane == 0) red[slice][parity][0][w] = p;
       slice_bar(slice);
@@ -224,12 +301,13 @@ row_kernel(RowArgs a) {
                                  __fadd_rn(red[slice][parity][0][1], red[slice][parity][0][3]));
       mu = __fdiv_rn(s0, kf);
       float q = 0.0f;
-      SQ_CHUNK_LOOP({
-        _Pragma("unroll") for (int e = 0; e < 8; ++e) {
+      for_chunks<MAXC>(cur, xr, j, nchunk, [&](int, int64_t, const float (&v)[8]) {
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
           const float d = __fsub_rn(v[e], mu);
           q = __fmaf_rn(d, d, q);
         }
-      })
+      });
       q = warp_sum_butterfly(q);
       if (lane == 0) red[slice][parity][1][w] = q;
       slice_bar(slice);
@@ -238,41 +316,40 @@ row_kernel(RowArgs a) {
       const float var = __fdiv_rn(s1, kf);
       rstd = __fdiv_rn(1.0f, __fsqrt_rn(__fadd_rn(var, a.eps)));
     }
-
-    // y for chunk c, element e (gv/bv/mv hold the parameters of the chunk)
-#define SQ_Y(e) (LN ? __fadd_rn(__fmul_rn(__fmul_rn(__fsub_rn(v[e], mu), rstd), gv[e]), bv[e]) \
-                    : (mul ? __fmul_rn(v[e], mv[e]) : v[e]))
-#define SQ_PARAMS                                                               \
-    float gv[8], bv[8], mv[8];                                                  \
-    if (LN) {                                                                   \
-      load8(g + c * 8, gv);                                                     \
-      if (b) load8(b + c * 8, bv); else { _Pragma("unroll") for (int e = 0; e < 8; ++e) bv[e] = 0.0f; } \
-    } else if (mul) {                                                           \
-      load8(mul + c * 8, mv);                                                   \
-    }
+    // y of element e given the chunk's parameters
+    auto yv = [&](float v, float gq, float bq) -> float {
+      if constexpr (LN) {
+        return __fadd_rn(__fmul_rn(__fmul_rn(__fsub_rn(v, mu), rstd), gq), bq);
+      } else {
+        return mul ? __fmul_rn(v, gq) : v;
+      }
+    };
 
     if constexpr (MODE == ROW_COLMAX) {
-      SQ_CHUNK_LOOP({
-        SQ_PARAMS
-        _Pragma("unroll") for (int e = 0; e < 8; ++e) {
-          const float y = fabsf(SQ_Y(e));
+      for_chunks<MAXC>(cur, xr, j, nchunk, [&](int i, int64_t c, const float (&v)[8]) {
+        float g8[8], b8[8];
+        params(i, c, g8, b8);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          const float y = fabsf(yv(v[e], g8[e], b8[e]));
           if constexpr (MAXC > 0) {
             cmax[i * 8 + e] = fmaxf(cmax[i * 8 + e], y);
-          } else if (use_smem) {
-            atomicMax(&colmax_s[c * 8 + e], __float_as_uint(y));
           } else {
-            atomicMax((unsigned int*)a.colmax + c * 8 + e, __float_as_uint(y));
+            if (use_smem) atomicMax(&colmax_s[c * 8 + e], __float_as_uint(y));
+            else atomicMax((unsigned int*)a.colmax + c * 8 + e, __float_as_uint(y));
           }
         }
-      })
+      });
     } else {
       float inv = static_inv;
-      if (MODE == ROW_DYNAMIC) {
+      if constexpr (MODE == ROW_DYNAMIC) {
         float m = 0.0f;
-        SQ_CHUNK_LOOP({
-          SQ_PARAMS
-          _Pragma("unroll") for (int e = 0; e < 8; ++e) m = fmaxf(m, fabsf(SQ_Y(e)));
-        })
+        for_chunks<MAXC>(cur, xr, j, nchunk, [&](int i, int64_t c, const float (&v)[8]) {
+          float g8[8], b8[8];
+          params(i, c, g8, b8);
+#pragma unroll
+          for (int e = 0; e < 8; ++e) m = fmaxf(m, fabsf(yv(v[e], g8[e], b8[e])));
+        });
         m = warp_max(m);
         if (lane == 0) red[slice][parity][2][w] = m;
         slice_bar(slice);
@@ -283,42 +360,50 @@ row_kernel(RowArgs a) {
         if (j == 0) a.scale[row] = delta;
       }
       int8_t* qr = a.q + row * K;
-      SQ_CHUNK_LOOP({
-        SQ_PARAMS
+      for_chunks<MAXC>(cur, xr, j, nchunk, [&](int i, int64_t c, const float (&v)[8]) {
+        float g8[8], b8[8];
+        params(i, c, g8, b8);
         int q[8];
-        _Pragma("unroll") for (int e = 0; e < 8; ++e) q[e] = quant_code(SQ_Y(e), inv, clipped);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) q[e] = quant_code(yv(v[e], g8[e], b8[e]), inv, clipped);
         uint2 pk;
         pk.x = pack4(q[0], q[1], q[2], q[3]);
         pk.y = pack4(q[4], q[5], q[6], q[7]);
         *reinterpret_cast<uint2*>(qr + c * 8) = pk;
-      })
+      });
     }
-#undef SQ_PARAMS
-#undef SQ_Y
-#undef SQ_CHUNK_LOOP
     parity ^= 1;
+    row = nrow;
+    if constexpr (MAXC > 0) {
+      if constexpr (PF) {
+#pragma unroll
+        for (int i = 0; i < CM; ++i) cur[i] = nxt[i];
+      } else {
+        if (row < a.T) load_row<MAXC>(cur, x + row * K, j, nchunk);
+      }
+    }
   }
 
   if constexpr (MODE == ROW_COLMAX) {
     if constexpr (MAXC > 0) {
-      // slices -> global directly (each slot owns distinct columns within a slice)
+      // the four slices own the same columns: combine them in shared memory
 #pragma unroll
       for (int i = 0; i < CM; ++i) {
         const int64_t c = j + (int64_t)i * kSliceThreads;
         if (c < nchunk) {
 #pragma unroll
           for (int e = 0; e < 8; ++e)
-            atomicMax((unsigned int*)a.colmax + c * 8 + e, __float_as_uint(cmax[i * 8 + e]));
+            atomicMax(&colmax_s[c * 8 + e], __float_as_uint(cmax[i * 8 + e]));
         }
       }
-    } else if (use_smem) {
+    }
+    if (use_smem) {
       __syncthreads();
       for (int64_t k = threadIdx.x; k < K; k += blockDim.x)
         atomicMax((unsigned int*)a.colmax + k, colmax_s[k]);
     }
   }
   if (COUNT && a.n_clipped) {
-    // warp-aggregated count
 #pragma unroll
     for (int o = 16; o >= 1; o >>= 1) clipped += __shfl_xor_sync(0xffffffffu, clipped, o);
     if (lane == 0 && clipped) atomicAdd(a.n_clipped, (unsigned long long)clipped);
@@ -327,59 +412,47 @@ row_kernel(RowArgs a) {
 
 template <typename T, int MAXC, bool LN, int MODE, bool COUNT>
 static cudaError_t launch_row_t(const RowArgs& a, cudaStream_t st) {
-  auto kern = row_kernel<T, MAXC, LN, MODE, COUNT>;
+  constexpr bool kBf16 = sizeof(T) == 2;
+  constexpr bool PF = MAXC > 0 && MAXC <= (kBf16 ? (MODE == ROW_COLMAX ? 4 : 8) : 2);
+  constexpr bool PREG = MAXC > 0 && MAXC <= 4 && MODE != ROW_COLMAX;
+  auto kern = row_kernel<T, MAXC, LN, MODE, COUNT, PREG, PF>;
   size_t smem = 0;
-  if (MODE == ROW_COLMAX && MAXC == 0) {
-    // per-CTA column peaks in shared memory when they fit; beyond that the
-    // kernel updates the global peaks directly
-    const size_t need = (size_t)a.K * sizeof(unsigned int);
-    if (need <= kColmaxSmemMax) {
-      smem = need;
-      cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                           (int)smem);
-      if (e != cudaSuccess) return e;
-    }
-  }
-  int per_sm = 0;
-  cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(
-      &per_sm, kern, kSlices * kSliceThreads, smem);
-  if (e != cudaSuccess) return e;
-  if (per_sm < 1) per_sm = 1;
+  if (MODE == ROW_COLMAX && (size_t)a.K * sizeof(unsigned int) <= kColmaxSmemMax)
+    smem = (size_t)a.K * sizeof(unsigned int);
+  // attribute and occupancy are queried once per instantiation and device
+  // (at the largest shared-memory size this variant ever uses)
+  static std::once_flag once[64];
+  static cudaError_t init_err[64];
+  static int per_sm_cache[64];
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess || dev < 0 || dev >= 64) return e != cudaSuccess ? e : cudaErrorInvalidDevice;
+  std::call_once(once[dev], [&] {
+    const size_t top = MODE == ROW_COLMAX ? kColmaxSmemMax : 0;
+    cudaError_t r = cudaSuccess;
+    if (top) r = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)top);
+    int n = 0;
+    if (r == cudaSuccess)
+      r = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, kern, kSlices * kSliceThreads, top);
+    per_sm_cache[dev] = n < 1 ? 1 : n;
+    init_err[dev] = r;
+  });
+  if (init_err[dev] != cudaSuccess) return init_err[dev];
+  int per_sm = per_sm_cache[dev];
+  // column peaks are flushed once per CTA: one CTA per SM
+  if (MODE == ROW_COLMAX) per_sm = 1;
   int64_t want = (a.T + kSlices - 1) / kSlices;
   int64_t cap = (int64_t)sm_count() * per_sm;
-  if (MODE == ROW_COLMAX) {
-    // fewer, longer-lived CTAs: each flushes K column peaks at the end
-    int64_t rows_each = 16;
-    int64_t lim = (a.T + kSlices * rows_each - 1) / (kSlices * rows_each);
-    if (want > lim) want = lim;
-  }
   int64_t grid = want < cap ? want : cap;
   if (grid < 1) grid = 1;
   kern<<<(unsigned)grid, kSlices * kSliceThreads, smem, st>>>(a);
   return cudaGetLastError();
 }
 
-// Register-cached variants cover K up to 8*128*MAXC; the largest MAXC that
-// compiles without spilling depends on the element type and mode (fp32 chunks
-// take twice the registers of bf16 ones; the column-peak mode also keeps a
-// running maximum per owned element).  Wider rows use the re-reading variant.
+// Rows too wide for the shared-memory pipeline (rowpipe.cu) take the
+// re-reading variant, which serves any K.
 template <typename T, bool LN, int MODE, bool COUNT>
 static cudaError_t dispatch_maxc(const RowArgs& a, cudaStream_t st) {
-  constexpr bool kBf16 = sizeof(T) == 2;
-  constexpr int kMax = MODE == ROW_COLMAX ? (kBf16 ? 8 : 4) : (kBf16 ? 24 : 8);
-  const int64_t per_thread = (a.K / 8 + kSliceThreads - 1) / kSliceThreads;
-  if (per_thread <= 1) return launch_row_t<T, 1, LN, MODE, COUNT>(a, st);
-  if (per_thread <= 2) return launch_row_t<T, 2, LN, MODE, COUNT>(a, st);
-  if (per_thread <= 4) return launch_row_t<T, 4, LN, MODE, COUNT>(a, st);
-  if constexpr (kMax >= 8) {
-    if (per_thread <= 8) return launch_row_t<T, 8, LN, MODE, COUNT>(a, st);
-  }
-  if constexpr (kMax >= 16) {
-    if (per_thread <= 16) return launch_row_t<T, 16, LN, MODE, COUNT>(a, st);
-  }
-  if constexpr (kMax >= 24) {
-    if (per_thread <= 24) return launch_row_t<T, 24, LN, MODE, COUNT>(a, st);
-  }
   return launch_row_t<T, 0, LN, MODE, COUNT>(a, st);
 }
 
@@ -405,6 +478,8 @@ static cudaError_t dispatch_mode(const RowArgs& a, RowMode mode, cudaStream_t st
 }
 
 cudaError_t launch_row(const RowArgs& a, sq_dtype xt, RowMode mode, cudaStream_t st) {
+  if (rowpipe_fits(a.K, xt, mode, a.g != nullptr))
+    return launch_rowpipe(a, xt, mode, st);
   if (xt == SQ_BF16) return dispatch_mode<uint16_t>(a, mode, st);
   return dispatch_mode<float>(a, mode, st);
 }
@@ -412,15 +487,20 @@ cudaError_t launch_row(const RowArgs& a, sq_dtype xt, RowMode mode, cudaStream_t
 // ============================================================ eq. (4)
 // s_k = a^alpha / b^(1-alpha), a = amax_x[k], b = max(max_n |W[n,k]|, 1e-7)
 // in fp64 (alpha = 0.5 via square roots, alpha in {0, 1} without pow), then
-// one rounding to fp32, floored at 1e-4; inv_s = 1/s.  One CTA; it also
-// forms the static activation step Delta(max_k a/s_k).
-__global__ void __launch_bounds__(1024)
+// one rounding to fp32, floored at 1e-4; inv_s = 1/s.  Each CTA also forms
+// Delta(max over its channels of a/s_k) and raises delta_out to it with an
+// atomic max on the (non-negative) fp32 bits: Delta is non-decreasing in its
+// argument, so the maximum over CTAs is Delta of the maximum over channels.
+constexpr int kScaleThreads = 256;
+
+__global__ void __launch_bounds__(kScaleThreads)
 scales_kernel(const float* __restrict__ amax_x, int64_t K, float alpha,
-              float* s, float* __restrict__ inv_s, float* __restrict__ delta_out) {
-  __shared__ float wmax[32];
+              float* s, float* __restrict__ inv_s, unsigned int* __restrict__ delta_out) {
+  __shared__ float wmax[kScaleThreads / 32];
   float lmax = 0.0f;
   const double al = (double)alpha;
-  for (int64_t k = threadIdx.x; k < K; k += blockDim.x) {
+  for (int64_t k = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; k < K;
+       k += (int64_t)gridDim.x * blockDim.x) {
     const float a = amax_x[k];
     const float bw = fmaxf(s[k], 1e-7f);  // s holds the weight column peak on entry
     const double ad = (double)a, bd = (double)bw;
@@ -446,14 +526,22 @@ scales_kernel(const float* __restrict__ amax_x, int64_t K, float alpha,
     if (threadIdx.x < 32) {
       float v = threadIdx.x < (blockDim.x >> 5) ? wmax[threadIdx.x] : 0.0f;
       v = warp_max(v);
-      if (threadIdx.x == 0) delta_out[0] = __fdiv_rn(fmaxf(v, 1e-7f), 127.0f);
+      if (threadIdx.x == 0)
+        atomicMax(delta_out, __float_as_uint(__fdiv_rn(fmaxf(v, 1e-7f), 127.0f)));
     }
   }
 }
 
-cudaError_t launch_scales(const float* amax_x, int64_t K, float alpha, float* s,
-                          float* inv_s, float* delta_out, cudaStream_t st) {
-  scales_kernel<<<1, 1024, 0, st>>>(amax_x, K, alpha, s, inv_s, delta_out);
+cudaError_t launch_scales(const float* amax_x, int64_t K, float alpha, float* s, float* inv_s,
+                          float* delta_out, cudaStream_t st) {
+  if (delta_out) {
+    cudaError_t e = cudaMemsetAsync(delta_out, 0, sizeof(float), st);
+    if (e != cudaSuccess) return e;
+  }
+  int64_t blocks = (K + kScaleThreads - 1) / kScaleThreads;
+  if (blocks > 4 * (int64_t)sm_count()) blocks = 4 * (int64_t)sm_count();
+  scales_kernel<<<(unsigned)blocks, kScaleThreads, 0, st>>>(amax_x, K, alpha, s, inv_s,
+                                                           (unsigned int*)delta_out);
   return cudaGetLastError();
 }
 

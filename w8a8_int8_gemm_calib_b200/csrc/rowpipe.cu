@@ -1,0 +1,558 @@
+// rowpipe.cu -- the row-wise HBM-bound steps of the smoothed W8A8 linear
+// layer as a TMA bulk-copy pipeline on sm_100a: the LayerNorm-fused
+// calibration peak, the per-output-channel weight quantizer (W * s), and the
+// runtime fused LayerNorm + smoothing + symmetric INT8 activation quantizer.
+//
+// Sources:
+//   [review]   "SmoothQuant：大型语言模型的精准高效训练后量化 — 深度技术评审"
+//              §2.2 (symmetric quantizer, step max|X|/127, round to nearest),
+//              §2.5-2.6 (static per-tensor / dynamic per-token steps), §5.5
+//   [embedded] "嵌入式 SLM 动态权重量化：SmoothQuant 激活异常值迁移与 INT8 部署实战"
+//              §二 (modified LayerNorm with gamma/s, beta/s feeding the INT8
+//              quantizer; W * diag(s) with static per-channel INT8)
+//
+// Design.  One CTA per SM: a producer warp streams whole rows (contiguous
+// K-element runs) from HBM into a ring of shared-memory row slots with 1-D
+// bulk copies completing on mbarriers, up to 16 rows ahead; four 128-thread
+// slices consume the rows.  Slot j = 32*w + l of a slice owns the 8-element
+// chunks c = j, j+128, ... of the row, which fixes the LayerNorm reduction
+// order (see rowops.cu; both files implement the same order).  Per-column
+// parameters (gamma, beta, or the column multiplier) are staged in shared
+// memory once per CTA.  Every mbarrier wait is bounded.
+//
+// Rounding: r = y * (1/Delta) is clamped to [-127, 127] (NaN -> 0) and
+// 1.5 * 2^23 is added: the fp32 addition rounds r to the nearest integer, ties
+// to even, and the low byte of the sum's bit pattern is the two's-complement
+// code (the constant's low byte is zero).  This equals round-half-even then
+// clamp, without the quarter-rate float-to-int conversion.
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include <mutex>
+
+#include "sq_device.cuh"
+#include "sq_internal.h"
+#include "tc_ptx.cuh"
+
+namespace sq {
+
+namespace {
+
+constexpr int kConsumers = 512;        // consumer threads per CTA
+constexpr int kThreads = kConsumers + 32;
+constexpr int kMaxSlots = 16;
+constexpr size_t kSmemBudget = 200 * 1024;
+constexpr uint32_t kCopyPiece = 32768;
+constexpr uint64_t kWaitNs = 2000000000ull;
+constexpr uint64_t kDrainNs = 1000000000ull;
+constexpr float kRoundMagic = 12582912.0f;  // 1.5 * 2^23
+
+struct Pipe {
+  RowArgs a;
+  int64_t rows_per_cta;
+  uint32_t row_bytes;
+  int slots;
+  int count;  // accumulate n_clipped
+  unsigned int* status;
+};
+
+template <int ST>
+__device__ __forceinline__ void slice_sync_t(int q) {
+  asm volatile("bar.sync %0, %1;" ::"r"(q + 1), "r"(ST) : "memory");
+}
+// slice-wide AND of v (also a barrier of the slice)
+template <int ST>
+__device__ __forceinline__ bool slice_and_t(int q, bool v) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred p, o;\n\t"
+      "setp.ne.u32 p, %1, 0;\n\t"
+      "bar.red.and.pred o, %2, %3, p;\n\t"
+      "selp.u32 %0, 1, 0, o;\n\t}"
+      : "=r"(r)
+      : "r"((uint32_t)v), "r"(q + 1), "r"(ST)
+      : "memory");
+  return r != 0;
+}
+
+__device__ __forceinline__ float bsum(float p) {
+#pragma unroll
+  for (int o = 16; o >= 1; o >>= 1) p = __fadd_rn(p, __shfl_xor_sync(0xffffffffu, p, o));
+  return p;
+}
+__device__ __forceinline__ float bmax(float p) {
+#pragma unroll
+  for (int o = 16; o >= 1; o >>= 1) p = fmaxf(p, __shfl_xor_sync(0xffffffffu, p, o));
+  return p;
+}
+
+// One chunk of a row in shared memory, in storage form (8 bf16 or 8 fp32).
+template <typename T> struct RawC;
+template <> struct RawC<uint16_t> { uint4 a; };
+template <> struct RawC<float> { uint4 a, b; };
+
+__device__ __forceinline__ void lds_raw(const uint8_t* row, int64_t c, RawC<uint16_t>& r) {
+  r.a = *reinterpret_cast<const uint4*>(row + c * 16);
+}
+__device__ __forceinline__ void lds_raw(const uint8_t* row, int64_t c, RawC<float>& r) {
+  r.a = *reinterpret_cast<const uint4*>(row + c * 32);
+  r.b = *reinterpret_cast<const uint4*>(row + c * 32 + 16);
+}
+__device__ __forceinline__ void unpack8(const RawC<uint16_t>& r, float (&v)[8]) {
+  v[0] = bf16lo(r.a.x); v[1] = bf16hi(r.a.x); v[2] = bf16lo(r.a.y); v[3] = bf16hi(r.a.y);
+  v[4] = bf16lo(r.a.z); v[5] = bf16hi(r.a.z); v[6] = bf16lo(r.a.w); v[7] = bf16hi(r.a.w);
+}
+__device__ __forceinline__ void unpack8(const RawC<float>& r, float (&v)[8]) {
+  v[0] = __uint_as_float(r.a.x); v[1] = __uint_as_float(r.a.y);
+  v[2] = __uint_as_float(r.a.z); v[3] = __uint_as_float(r.a.w);
+  v[4] = __uint_as_float(r.b.x); v[5] = __uint_as_float(r.b.y);
+  v[6] = __uint_as_float(r.b.z); v[7] = __uint_as_float(r.b.w);
+}
+__device__ __forceinline__ void lds8(const float* p, float (&v)[8]) {
+  const float4 a = *reinterpret_cast<const float4*>(p);
+  const float4 b = *reinterpret_cast<const float4*>(p + 4);
+  v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w; v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
+}
+
+// Q(y; Delta) given inv = 1/Delta, as the fp32 whose low byte is the code:
+// general form (any y: NaN -> 0, saturation counted and clamped).
+__device__ __forceinline__ uint32_t qbits(float y, float inv, bool count, unsigned& clipped) {
+  float r = __fmul_rn(y, inv);
+  if (count) clipped += fabsf(r) >= 127.5f;  // rounds outside [-127, 127]
+  r = (r != r) ? 0.0f : r;
+  r = fminf(fmaxf(r, -127.0f), 127.0f);
+  return __float_as_uint(__fadd_rn(r, kRoundMagic));
+}
+// Per-token form for rows whose elements are all finite: |y| <= m and
+// inv = 1/fl(max(m,1e-7)/127) give |y*inv| <= 127*(1+2^-23) < 127.5, so no
+// element can saturate and no clamp is needed.
+__device__ __forceinline__ uint32_t qbits_fast(float y, float inv) {
+  return __float_as_uint(__fadd_rn(__fmul_rn(y, inv), kRoundMagic));
+}
+
+__device__ __forceinline__ void store_codes(int8_t* dst, const uint32_t (&b)[8]) {
+  uint2 pk;
+  pk.x = pack4((int)b[0], (int)b[1], (int)b[2], (int)b[3]);
+  pk.y = pack4((int)b[4], (int)b[5], (int)b[6], (int)b[7]);
+  *reinterpret_cast<uint2*>(dst) = pk;
+}
+
+// Slices of W warps (ST = 32*W threads).  A slice emulates the 128 canonical
+// LayerNorm slots: thread (v, l) -- warp v of the slice, lane l -- walks the
+// chunks c = 32*v + l + ST*i, i = 0, 1, ...; chunk i belongs to slot
+// 32*(v + W*(i mod G)) + l with G = 4/W slot groups per thread, so each slot
+// still accumulates its own chunks in increasing c.  The slot groups are
+// then combined exactly as (r0 + r2) + (r1 + r3).
+template <typename T, int W, int CM, bool LN, int MODE>
+__global__ void __launch_bounds__(kThreads, 1) rowpipe_kernel(const Pipe P) {
+  constexpr int ST = 32 * W;            // threads per slice
+  constexpr int NS = kConsumers / ST;   // slices per CTA
+  constexpr int G = 4 / W;              // slot groups per thread
+  extern __shared__ __align__(128) uint8_t smem[];
+  __shared__ float red[NS][2][3][W];
+  __shared__ int abort_s;
+
+  const RowArgs& a = P.a;
+  const int64_t K = a.K, nchunk = K >> 3;
+  const int S = P.slots;
+  const uint32_t RB = P.row_bytes;
+  uint8_t* ring = smem;
+  float* pg = reinterpret_cast<float*>(smem + (size_t)S * RB);  // gamma or multiplier [K]
+  float* pb = pg + K;                                            // beta [K] (LN)
+  unsigned int* colmax_s = reinterpret_cast<unsigned int*>(LN ? pb + K : pb);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(colmax_s + (MODE == ROW_COLMAX ? K : 0));
+  const uint32_t ring_u32 = tc::smem_u32(ring);
+  auto full_bar = [&](int s) { return tc::smem_u32(bars + s); };
+  auto empty_bar = [&](int s) { return tc::smem_u32(bars + kMaxSlots + s); };
+
+  const int tid = threadIdx.x;
+  const bool has_mul = !LN && a.mul != nullptr;
+  if (tid < kConsumers) {
+    for (int64_t k = tid; k < K; k += kConsumers) {
+      if (LN) {
+        pg[k] = a.g[k];
+        pb[k] = a.b ? a.b[k] : 0.0f;
+      } else if (has_mul) {
+        pg[k] = a.mul[k];
+      }
+      if (MODE == ROW_COLMAX) colmax_s[k] = 0u;
+    }
+  }
+  if (tid == 0) {
+    for (int s = 0; s < S; ++s) {
+      tc::mbar_init(full_bar(s), 1);
+      tc::mbar_init(empty_bar(s), 1);
+    }
+    abort_s = 0;
+    tc::mbar_fence_init();
+  }
+  __syncthreads();
+  volatile int* abort_flag = &abort_s;
+
+  const int64_t r0 = (int64_t)blockIdx.x * P.rows_per_cta;
+  int64_t R = a.T - r0;
+  if (R > P.rows_per_cta) R = P.rows_per_cta;
+  if (R < 0) R = 0;
+  unsigned clipped = 0;
+
+  if (tid >= kConsumers) {
+    // ------------------------------------------------------------ producer
+    if (tid == kConsumers) {
+      uint32_t issued = 0, issued_par = 0;
+      bool ok = true;
+      const uint8_t* src = reinterpret_cast<const uint8_t*>(a.x) + r0 * (int64_t)RB;
+      for (int64_t i = 0; i < R; ++i) {
+        const int s = (int)(i % S);
+        const int64_t u = i / S;
+        if (u > 0 && !tc::mbar_wait(empty_bar(s), (uint32_t)((u - 1) & 1), abort_flag, kWaitNs,
+                                    P.status)) {
+          ok = false;
+          break;
+        }
+        tc::mbar_arrive_expect_tx(full_bar(s), RB);
+        for (uint32_t off = 0; off < RB; off += kCopyPiece) {
+          const uint32_t n = RB - off < kCopyPiece ? RB - off : kCopyPiece;
+          tc::bulk_load(ring_u32 + (uint32_t)s * RB + off, src + i * (int64_t)RB + off, n,
+                        full_bar(s));
+        }
+        issued |= 1u << s;
+        issued_par = (issued_par & ~(1u << s)) | ((uint32_t)(u & 1) << s);
+      }
+      if (!ok) {
+        int never = 0;
+        for (int s = 0; s < S; ++s)
+          if (issued & (1u << s))
+            tc::mbar_wait(full_bar(s), (issued_par >> s) & 1u, &never, kDrainNs, P.status);
+      }
+    }
+  } else {
+    // ------------------------------------------------------------ consumers
+    const int q = tid / ST, j = tid % ST;
+    const int v = j >> 5, lane = j & 31;
+    const float kf = (float)K;
+    constexpr int NC = (MODE == ROW_COLMAX && CM > 0) ? CM * 8 : 1;
+    float cmax[NC];
+#pragma unroll
+    for (int i = 0; i < NC; ++i) cmax[i] = 0.0f;
+    const float static_inv = MODE == ROW_STATIC ? __fdiv_rn(1.0f, __ldg(a.scale)) : 0.0f;
+    const bool count = P.count != 0;
+    int parity = 0;
+    auto chunk_of = [&](int i) -> int64_t { return 32 * v + lane + (int64_t)ST * i; };
+    auto sync = [&]() { slice_sync_t<ST>(q); };
+
+    for (int64_t i = q; i < R; i += NS) {
+      const int s = (int)(i % S);
+      const int64_t u = i / S;
+      bool ok = tc::mbar_wait(full_bar(s), (uint32_t)(u & 1), abort_flag, kWaitNs, P.status);
+      if (!slice_and_t<ST>(q, ok)) break;
+      const uint8_t* rowp = ring + (size_t)s * RB;
+      const int64_t row = r0 + i;
+
+      RawC<T> xr[CM > 0 ? CM : 1];
+      if constexpr (CM > 0) {
+#pragma unroll
+        for (int m = 0; m < CM; ++m)
+          if (chunk_of(m) < nchunk) lds_raw(rowp, chunk_of(m), xr[m]);
+      }
+      // f(m, c, x[8]) over the thread's chunks in increasing c
+      auto for_chunks = [&](auto&& f) {
+        if constexpr (CM > 0) {
+#pragma unroll
+          for (int m = 0; m < CM; ++m) {
+            const int64_t c = chunk_of(m);
+            if (c < nchunk) {
+              float x[8];
+              unpack8(xr[m], x);
+              f(m, c, x);
+            }
+          }
+        } else {
+          int m = 0;
+          for (int64_t c = chunk_of(0); c < nchunk; c += ST, ++m) {
+            RawC<T> r;
+            lds_raw(rowp, c, r);
+            float x[8];
+            unpack8(r, x);
+            f(m, c, x);
+          }
+        }
+      };
+      // exact (r0 + r2) + (r1 + r3) of the per-slot partial sums p[g]
+      auto slot_sum = [&](const float (&p)[G], int which) -> float {
+        float t[G];
+#pragma unroll
+        for (int g = 0; g < G; ++g) t[g] = bsum(p[g]);
+        float mine = t[0];
+        if constexpr (G == 2) mine = __fadd_rn(t[0], t[1]);  // r_v + r_(v+2)
+        if (lane == 0) red[q][parity][which][v] = mine;
+        sync();
+        const float* r = red[q][parity][which];
+        if constexpr (W == 4) return __fadd_rn(__fadd_rn(r[0], r[2]), __fadd_rn(r[1], r[3]));
+        else return __fadd_rn(r[0], r[1]);
+      };
+
+      float mu = 0.0f, rstd = 0.0f;
+      if constexpr (LN) {
+        float p[G];
+#pragma unroll
+        for (int g = 0; g < G; ++g) p[g] = 0.0f;
+        for_chunks([&](int m, int64_t, const float (&x)[8]) {
+#pragma unroll
+          for (int e = 0; e < 8; ++e) p[m % G] = __fadd_rn(p[m % G], x[e]);
+        });
+        mu = __fdiv_rn(slot_sum(p, 0), kf);
+#pragma unroll
+        for (int g = 0; g < G; ++g) p[g] = 0.0f;
+        for_chunks([&](int m, int64_t, const float (&x)[8]) {
+#pragma unroll
+          for (int e = 0; e < 8; ++e) {
+            const float d = __fsub_rn(x[e], mu);
+            p[m % G] = __fmaf_rn(d, d, p[m % G]);
+          }
+        });
+        rstd = __fdiv_rn(1.0f, __fsqrt_rn(__fadd_rn(__fdiv_rn(slot_sum(p, 1), kf), a.eps)));
+      }
+      auto ychunk = [&](int64_t c, const float (&x)[8], float (&y)[8]) {
+        if constexpr (LN) {
+          float g8[8], b8[8];
+          lds8(pg + c * 8, g8);
+          lds8(pb + c * 8, b8);
+#pragma unroll
+          for (int e = 0; e < 8; ++e)
+            y[e] = __fadd_rn(__fmul_rn(__fmul_rn(__fsub_rn(x[e], mu), rstd), g8[e]), b8[e]);
+        } else {
+          if (has_mul) {
+            float m8[8];
+            lds8(pg + c * 8, m8);
+#pragma unroll
+            for (int e = 0; e < 8; ++e) y[e] = __fmul_rn(x[e], m8[e]);
+          } else {
+#pragma unroll
+            for (int e = 0; e < 8; ++e) y[e] = x[e];
+          }
+        }
+      };
+
+      if constexpr (MODE == ROW_COLMAX) {
+        for_chunks([&](int m, int64_t c, const float (&x)[8]) {
+          float y[8];
+          ychunk(c, x, y);
+#pragma unroll
+          for (int e = 0; e < 8; ++e) {
+            if constexpr (CM > 0) {
+              cmax[m * 8 + e] = fmaxf(cmax[m * 8 + e], fabsf(y[e]));
+            } else {
+              atomicMax(&colmax_s[c * 8 + e], __float_as_uint(fabsf(y[e])));
+            }
+          }
+        });
+      } else if constexpr (MODE == ROW_STATIC) {
+        int8_t* qr = a.q + row * K;
+        for_chunks([&](int, int64_t c, const float (&x)[8]) {
+          float y[8];
+          ychunk(c, x, y);
+          uint32_t b[8];
+#pragma unroll
+          for (int e = 0; e < 8; ++e) b[e] = qbits(y[e], static_inv, count, clipped);
+          store_codes(qr + c * 8, b);
+        });
+      } else {
+        // peak of |y| as the maximum of the fp32 bit patterns: exact for
+        // finite values, and any inf/NaN element shows up as a pattern at or
+        // above that of +inf
+        uint32_t mb = 0;
+        for_chunks([&](int, int64_t c, const float (&x)[8]) {
+          float y[8];
+          ychunk(c, x, y);
+#pragma unroll
+          for (int e = 0; e < 8; ++e) mb = max(mb, __float_as_uint(fabsf(y[e])));
+        });
+#pragma unroll
+        for (int o = 16; o >= 1; o >>= 1) mb = max(mb, __shfl_xor_sync(0xffffffffu, mb, o));
+        if (lane == 0) red[q][parity][2][v] = __uint_as_float(mb);
+        sync();
+#pragma unroll
+        for (int t = 0; t < W; ++t) mb = max(mb, __float_as_uint(red[q][parity][2][t]));
+        const bool clean = mb < 0x7f800000u;
+        float mx = __uint_as_float(mb);
+        if (!clean) {
+          // non-finite elements: the peak over the non-NaN values, as fmaxf
+          float m2 = 0.0f;
+          for_chunks([&](int, int64_t c, const float (&x)[8]) {
+            float y[8];
+            ychunk(c, x, y);
+#pragma unroll
+            for (int e = 0; e < 8; ++e) m2 = fmaxf(m2, fabsf(y[e]));
+          });
+          m2 = bmax(m2);
+          sync();  // everyone has read red[..][2] above
+          if (lane == 0) red[q][parity][2][v] = m2;
+          sync();
+#pragma unroll
+          for (int t = 0; t < W; ++t) m2 = fmaxf(m2, red[q][parity][2][t]);
+          mx = m2;
+        }
+        const float delta = __fdiv_rn(fmaxf(mx, 1e-7f), 127.0f);
+        const float inv = __fdiv_rn(1.0f, delta);
+        if (j == 0) a.scale[row] = delta;
+        int8_t* qr = a.q + row * K;
+        if (clean) {
+          for_chunks([&](int, int64_t c, const float (&x)[8]) {
+            float y[8];
+            ychunk(c, x, y);
+            uint32_t b[8];
+#pragma unroll
+            for (int e = 0; e < 8; ++e) b[e] = qbits_fast(y[e], inv);
+            store_codes(qr + c * 8, b);
+          });
+        } else {
+          for_chunks([&](int, int64_t c, const float (&x)[8]) {
+            float y[8];
+            ychunk(c, x, y);
+            uint32_t b[8];
+#pragma unroll
+            for (int e = 0; e < 8; ++e) b[e] = qbits(y[e], inv, count, clipped);
+            store_codes(qr + c * 8, b);
+          });
+        }
+      }
+      sync();  // every thread of the slice is done with the slot
+      if (j == 0) tc::mbar_arrive(empty_bar(s));
+      parity ^= 1;
+    }
+    if constexpr (MODE == ROW_COLMAX && CM > 0) {
+#pragma unroll
+      for (int m = 0; m < CM; ++m) {
+        const int64_t c = chunk_of(m);
+        if (c < nchunk) {
+#pragma unroll
+          for (int e = 0; e < 8; ++e)
+            atomicMax(&colmax_s[c * 8 + e], __float_as_uint(cmax[m * 8 + e]));
+        }
+      }
+    }
+  }
+  __syncthreads();
+  if constexpr (MODE == ROW_COLMAX) {
+    if (tid < kConsumers && R > 0)
+      for (int64_t k = tid; k < K; k += kConsumers)
+        atomicMax(reinterpret_cast<unsigned int*>(a.colmax) + k, colmax_s[k]);
+  }
+  if (P.count && tid < kConsumers) {
+#pragma unroll
+    for (int o = 16; o >= 1; o >>= 1) clipped += __shfl_xor_sync(0xffffffffu, clipped, o);
+    if ((tid & 31) == 0 && clipped) atomicAdd(a.n_clipped, (unsigned long long)clipped);
+  }
+}
+
+// Shared memory after the ring: parameters (gamma and beta, or the column
+// multiplier: the region exists even when no multiplier is given), the
+// per-CTA column peaks (column-peak mode), and the mbarriers.
+size_t fixed_smem(int64_t K, bool ln, RowMode mode) {
+  size_t b = (ln ? 2 : 1) * (size_t)K * 4;
+  if (mode == ROW_COLMAX) b += (size_t)K * 4;
+  return b + 2 * kMaxSlots * 8;
+}
+
+template <typename T, int W, int CM, bool LN, int MODE>
+cudaError_t launch_t(const Pipe& P, size_t smem, int grid, cudaStream_t st) {
+  auto kern = rowpipe_kernel<T, W, CM, LN, MODE>;
+  // the shared-memory limit is raised once per instantiation (and per
+  // device), to the whole budget, so that launches stay free of driver calls
+  static std::once_flag once[64];
+  static cudaError_t attr_err[64];
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess || dev < 0 || dev >= 64) return e != cudaSuccess ? e : cudaErrorInvalidDevice;
+  std::call_once(once[dev], [&] {
+    attr_err[dev] = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)kSmemBudget);
+  });
+  if (attr_err[dev] != cudaSuccess) return attr_err[dev];
+  kern<<<grid, kThreads, smem, st>>>(P);
+  return cudaGetLastError();
+}
+
+// Quantizing modes: 64-thread slices (8 rows in flight per SM); the row is
+// held packed in registers when it spans at most 16 chunks per thread
+// (bf16: 64 registers) or 8 (fp32), else each pass re-reads shared memory.
+template <typename T, bool LN, int MODE>
+cudaError_t dispatch_quant(const Pipe& P, size_t smem, int grid, cudaStream_t st) {
+  constexpr bool kBf16 = sizeof(T) == 2;
+  const int64_t per = (P.a.K / 8 + 63) / 64;
+  if (per <= 2) return launch_t<T, 2, 2, LN, MODE>(P, smem, grid, st);
+  if (per <= 4) return launch_t<T, 2, 4, LN, MODE>(P, smem, grid, st);
+  if (per <= 8) return launch_t<T, 2, 8, LN, MODE>(P, smem, grid, st);
+  if constexpr (kBf16) {
+    if (per <= 12) return launch_t<T, 2, 12, LN, MODE>(P, smem, grid, st);
+    if (per <= 16) return launch_t<T, 2, 16, LN, MODE>(P, smem, grid, st);
+  }
+  return launch_t<T, 2, 0, LN, MODE>(P, smem, grid, st);
+}
+
+// Column-peak mode: 128-thread slices; the running peak of each owned
+// element stays in registers for up to 6 chunks per thread (4 for fp32).
+template <typename T>
+cudaError_t dispatch_colmax(const Pipe& P, size_t smem, int grid, cudaStream_t st) {
+  const int64_t per = (P.a.K / 8 + 127) / 128;
+  if (sizeof(T) == 4 && per > 4) return launch_t<T, 4, 0, true, ROW_COLMAX>(P, smem, grid, st);
+  switch (per) {
+    case 1: return launch_t<T, 4, 1, true, ROW_COLMAX>(P, smem, grid, st);
+    case 2: return launch_t<T, 4, 2, true, ROW_COLMAX>(P, smem, grid, st);
+    case 3: return launch_t<T, 4, 3, true, ROW_COLMAX>(P, smem, grid, st);
+    case 4: return launch_t<T, 4, 4, true, ROW_COLMAX>(P, smem, grid, st);
+    case 5: return launch_t<T, 4, 5, true, ROW_COLMAX>(P, smem, grid, st);
+    case 6: return launch_t<T, 4, 6, true, ROW_COLMAX>(P, smem, grid, st);
+    default: return launch_t<T, 4, 0, true, ROW_COLMAX>(P, smem, grid, st);
+  }
+}
+
+template <typename T>
+cudaError_t dispatch_mode(const Pipe& P, RowMode mode, size_t smem, int grid, cudaStream_t st) {
+  const bool ln = P.a.g != nullptr;
+  switch (mode) {
+    case ROW_DYNAMIC:
+      return ln ? dispatch_quant<T, true, ROW_DYNAMIC>(P, smem, grid, st)
+                : dispatch_quant<T, false, ROW_DYNAMIC>(P, smem, grid, st);
+    case ROW_STATIC:
+      return ln ? dispatch_quant<T, true, ROW_STATIC>(P, smem, grid, st)
+                : dispatch_quant<T, false, ROW_STATIC>(P, smem, grid, st);
+    case ROW_COLMAX:
+      return dispatch_colmax<T>(P, smem, grid, st);
+  }
+  return cudaErrorInvalidValue;
+}
+
+}  // namespace
+
+bool rowpipe_fits(int64_t K, sq_dtype xt, RowMode mode, bool ln) {
+  const size_t rb = (size_t)K * (xt == SQ_BF16 ? 2 : 4);
+  const size_t fixed = fixed_smem(K, ln, mode);
+  return fixed + 2 * rb <= kSmemBudget;
+}
+
+cudaError_t launch_rowpipe(const RowArgs& a, sq_dtype xt, RowMode mode, cudaStream_t st) {
+  const size_t rb = (size_t)a.K * (xt == SQ_BF16 ? 2 : 4);
+  const bool ln = a.g != nullptr;
+  const size_t fixed = fixed_smem(a.K, ln, mode);
+  int slots = (int)((kSmemBudget - fixed) / rb);
+  if (slots > kMaxSlots) slots = kMaxSlots;
+  if (slots < 2) return cudaErrorInvalidValue;
+  unsigned int* sw = status_word();
+  if (!sw) return cudaErrorInvalidDevice;
+  int grid = sm_count();
+  if ((int64_t)grid > a.T) grid = (int)a.T;
+  Pipe P{};
+  P.a = a;
+  P.rows_per_cta = (a.T + grid - 1) / grid;
+  grid = (int)((a.T + P.rows_per_cta - 1) / P.rows_per_cta);
+  P.row_bytes = (uint32_t)rb;
+  P.slots = slots;
+  P.count = a.n_clipped != nullptr;
+  P.status = sw;
+  const size_t smem = (size_t)slots * rb + fixed;
+  return xt == SQ_BF16 ? dispatch_mode<uint16_t>(P, mode, smem, grid, st)
+                       : dispatch_mode<float>(P, mode, smem, grid, st);
+}
+
+}  // namespace sq

@@ -43,6 +43,12 @@ struct RowArgs {
 cudaError_t launch_row(const RowArgs& a, sq_dtype xt, RowMode mode,
                        cudaStream_t st);
 
+// Bulk-copy pipelined variant (rowpipe.cu), used whenever two row slots and
+// the per-column parameters fit in shared memory.
+bool rowpipe_fits(int64_t K, sq_dtype xt, RowMode mode, bool ln);
+cudaError_t launch_rowpipe(const RowArgs& a, sq_dtype xt, RowMode mode,
+                           cudaStream_t st);
+
 // s / inv_s from amax_x and the weight column peaks held (as fp32) in s.
 cudaError_t launch_scales(const float* amax_x, int64_t K, float alpha,
                           float* s, float* inv_s, float* delta_out,
