@@ -150,7 +150,8 @@ sq_status sq_fuse_weights_q8(const void* w, sq_dtype wt, int64_t N, int64_t K,
  * GEMM; [review] §2.2, §2.5, §2.6, §6.3).
  *
  *   y = LN(x) with the folded gamma_s, beta_s (same order as sq_calib_absmax)
- *       when gamma_s != NULL, else y = x * inv_s (inv_s NULL: y = x);
+ *       when gamma_s != NULL (inv_s must then be NULL: s is already folded
+ *       into gamma_s and beta_s), else y = x * inv_s (inv_s NULL: y = x);
  *   SQ_ACT_PER_TOKEN_DYNAMIC: act_scale[t] = Delta(max_k |y[t,k]|) (output,
  *       [T] fp32), xq[t,k] = Q(y[t,k]; act_scale[t]);
  *   SQ_ACT_PER_TENSOR_STATIC: act_scale[0] is the calibrated step (input),
@@ -169,8 +170,11 @@ sq_status sq_ln_smooth_quant_act(const void* x, sq_dtype xt, int64_t T,
 
 /*
  * sq_gemm_workspace_bytes -- device scratch sq_gemm_w8a8 needs for this
- * shape (0 when it needs none).  The small-M (decode) path splits K across
- * SMs and reduces exact INT32 partial sums in the workspace.
+ * shape on the current device (0 when it needs none).  Problems with
+ * M <= 128 tokens take the weight-streaming path, which splits the K loop of
+ * a weight tile across SMs and reduces the exact INT32 partial tiles in the
+ * workspace: 256 bytes per 128 output channels (rounded up to 256) plus
+ * 2 * M * 128 * 4 bytes per SM used.
  */
 size_t sq_gemm_workspace_bytes(int64_t M, int64_t N, int64_t K);
 
@@ -187,10 +191,9 @@ size_t sq_gemm_workspace_bytes(int64_t M, int64_t N, int64_t K);
  *   y  [M,N] of type yt (SQ_F32, or SQ_BF16 = RNE of the fp32 value);
  *   acc_out: NULL, or [M,N] int32 that receives the accumulators.
  *   workspace: at least sq_gemm_workspace_bytes(M,N,K) bytes of device
- *   memory (may be NULL when that is 0).  It must be ZERO-FILLED before its
- *   first use; every call that completes without a device error leaves it
- *   zero-filled again.  Two calls that share a workspace must not run
- *   concurrently.
+ *   memory, 16-byte aligned (may be NULL when that size is 0).  It needs no
+ *   initialization: each call zeroes the part it counts with and overwrites
+ *   the rest.  Calls that share a workspace must not run concurrently.
  */
 sq_status sq_gemm_w8a8(const int8_t* xq, const int8_t* wq, int64_t M,
                        int64_t N, int64_t K, const float* act_scale,
@@ -201,9 +204,8 @@ sq_status sq_gemm_w8a8(const int8_t* xq, const int8_t* wq, int64_t M,
 /*
  * sq_sync_status -- synchronize `stream`, then return and clear the status
  * word of the current device: SQ_OK, or SQ_ERR_TIMEOUT when a kernel gave up
- * a bounded wait (its outputs are then undefined, and a GEMM workspace it
- * used must be zero-filled again), or SQ_ERR_CUDA when the synchronization
- * itself failed.
+ * a bounded wait (its outputs are then undefined), or SQ_ERR_CUDA when the
+ * synchronization itself failed.
  */
 sq_status sq_sync_status(sq_stream stream);
 

@@ -100,3 +100,50 @@ def test_gemm_is_deterministic(sq):
     y2, a2 = _run(sq, xq, wq, act, ws, True, "bf16", workspace=ws_buf)
     assert_bits_equal(a1, a2, "acc rerun")
     assert_bits_equal(y1, y2, "y rerun")
+
+
+# ---------------------------------------------------------------- small M
+# M <= 128 takes the weight-streaming kernel: tokens padded to 8/16/32/64/128
+# as the MMA N dimension, (tile, k-block) units split evenly over the SMs,
+# partial tiles summed exactly by the last CTA to arrive.
+SMALL_SHAPES = [
+    (1, 130, 16), (2, 1000, 12288), (8, 4096, 2064), (9, 300, 4096), (16, 2048, 1040),
+    (17, 777, 8192), (32, 1024, 6144), (33, 260, 144), (64, 3000, 2048), (100, 1536, 4096),
+    (128, 512, 12288), (128, 49152, 256), (5, 128, 20480),
+]
+
+
+@pytest.mark.parametrize("M,N,K", SMALL_SHAPES)
+def test_gemm_small_m_stream_k(sq, orc, M, N, K):
+    xq, wq, act, ws = _operands(M, N, K, M * 7 + N * 3 + K)
+    for out in ("bf16", "f32"):
+        y_want, acc_want = orc.gemm_w8a8(xq, wq, act, ws, per_token=True,
+                                         out_bf16=(out == "bf16"))
+        y, acc = _run(sq, xq, wq, act, ws, True, out, workspace=sq.Workspace())
+        assert_bits_equal(acc, acc_want, f"acc {out}")
+        assert_bits_equal(y, y_want, f"y {out}")
+
+
+def test_gemm_small_m_workspace_reuse(sq, orc):
+    """One workspace buffer reused across shapes, holding garbage from the
+    previous call: the kernel needs no particular initial contents."""
+    wsbuf = torch.full((64 << 20,), 0x5A, dtype=torch.uint8, device="cuda")
+    for (M, N, K) in [(128, 2000, 4096), (3, 50000, 1024), (64, 7000, 2048), (1, 1000, 12288)]:
+        need = sq.sq_gemm_workspace_bytes(M, N, K)
+        assert 0 < need <= wsbuf.numel()
+        xq, wq, act, ws = _operands(M, N, K, M + N + K)
+        y_want, acc_want = orc.gemm_w8a8(xq, wq, act, ws, out_bf16=True)
+        y, acc = _run(sq, xq, wq, act, ws, True, "bf16", workspace=wsbuf)
+        assert_bits_equal(acc, acc_want, "acc reuse")
+        assert_bits_equal(y, y_want, "y reuse")
+
+
+def test_gemm_small_m_rejects_short_workspace(sq):
+    M, N, K = 8, 1024, 1024
+    xq, wq, act, ws = _operands(M, N, K, 1)
+    need = sq.sq_gemm_workspace_bytes(M, N, K)
+    short = torch.empty(need - 16, dtype=torch.uint8, device="cuda")
+    y = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
+    with pytest.raises(sq.SQError) as ei:
+        sq.sq_gemm_w8a8(dev(xq), dev(wq), dev(act), dev(ws), y, workspace=short)
+    assert ei.value.status == 8  # SQ_ERR_WORKSPACE

@@ -93,8 +93,8 @@ def sq_gemm_workspace_bytes(M, N, K) -> int:
 
 
 class Workspace:
-    """Zero-filled device scratch for sq_gemm_w8a8, grown on demand (the GEMM
-    leaves it zero-filled after every call that completes without error)."""
+    """Device scratch for sq_gemm_w8a8, grown on demand.  The GEMM needs no
+    particular contents: each call resets the part it counts with."""
 
     def __init__(self, device=None):
         self.device = device
@@ -104,7 +104,7 @@ class Workspace:
         if nbytes == 0:
             return None
         if self.buf is None or self.buf.numel() < nbytes:
-            self.buf = torch.zeros(nbytes, dtype=torch.uint8, device=self.device or "cuda")
+            self.buf = torch.empty(nbytes, dtype=torch.uint8, device=self.device or "cuda")
         return self.buf
 
 

@@ -285,6 +285,295 @@ gemm_w8a8_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
   }
 }
 
+// ====================================================================== small M
+// Decode-shaped problems (M <= 128 tokens) stream the weights: the operands
+// are swapped so that a 128-row block of Wq fills the MMA's M dimension and
+// the (padded) tokens form its N dimension (NPAD in {8, 16, 32, 64, 128}).
+// The work -- (weight tile, 128-byte k-block) units -- is split evenly over
+// a persistent grid (stream-K): CTA g owns units [g*U/G, (g+1)*U/G).  A tile
+// covered by one CTA is finished in place; otherwise every contributing CTA
+// stores its INT32 partial tile into its own scratch slot, and the last one
+// to arrive (an atomic counter per tile) sums the slots -- exact integer
+// addition in any order -- and runs the epilogue.  No CTA ever waits for
+// another one.
+constexpr int SM_BM = 128;
+constexpr int SM_A_BYTES = SM_BM * BK;
+
+template <int NPAD>
+struct SmallCfg {
+  static constexpr int B_BYTES = NPAD * BK;
+  static constexpr int STAGE = SM_A_BYTES + B_BYTES;
+  static constexpr int STAGES = (200 * 1024) / STAGE > 12 ? 12 : (200 * 1024) / STAGE;
+  static constexpr uint32_t TMEM_COLS = 2 * NPAD < 32 ? 32 : 2 * NPAD;
+  static constexpr int CH = NPAD < 32 ? NPAD : 32;  // accumulator columns per TMEM load
+  static constexpr size_t SMEM = 1024 + (size_t)STAGES * STAGE + 512;
+};
+
+struct SmallParams {
+  int M, N, K;
+  int n_tiles, nk;
+  int64_t units;  // n_tiles * nk
+  int grid;
+  const float* act_scale;
+  int per_token;
+  const float* w_scale;
+  void* y;
+  int32_t* acc;
+  int32_t* slots;           // [grid][2][M][128]
+  unsigned int* counters;   // [n_tiles], zeroed before the launch
+  unsigned int* status;
+};
+
+__device__ __forceinline__ int64_t unit_begin(int64_t g, const SmallParams& p) {
+  return g * p.units / p.grid;
+}
+// the CTA whose range holds unit u
+__device__ __forceinline__ int64_t unit_owner(int64_t u, const SmallParams& p) {
+  return ((u + 1) * p.grid - 1) / p.units;
+}
+
+template <int CH>
+__device__ __forceinline__ void tmem_ld_n(uint32_t taddr, uint32_t (&r)[CH]) {
+  if constexpr (CH == 8) tc::tmem_ld8(taddr, r);
+  else if constexpr (CH == 16) tc::tmem_ld16(taddr, r);
+  else tc::tmem_ld32(taddr, r);
+}
+
+// y[t, n] (and acc[t, n]) for tokens t0 .. t0+CH-1 of output channel n
+template <bool BF16, int CH>
+__device__ __forceinline__ void small_store(const SmallParams& p, int n, int t0, const int32_t (&v)[CH]) {
+  if (n >= p.N) return;
+  const float ws = __ldg(p.w_scale + n);
+#pragma unroll
+  for (int i = 0; i < CH; ++i) {
+    const int t = t0 + i;
+    if (t < p.M) {
+      const float as = __ldg(p.act_scale + (p.per_token ? t : 0));
+      const float y = __fmul_rn(__int2float_rn(v[i]), __fmul_rn(as, ws));
+      const size_t o = (size_t)t * (size_t)p.N + (size_t)n;
+      if (BF16) reinterpret_cast<__nv_bfloat16*>(p.y)[o] = __float2bfloat16_rn(y);
+      else reinterpret_cast<float*>(p.y)[o] = y;
+      if (p.acc) p.acc[o] = v[i];
+    }
+  }
+}
+
+__device__ __forceinline__ void epi_bar() {
+  asm volatile("bar.sync 1, 128;" ::: "memory");
+}
+// AND of v over the 128 epilogue threads (also a barrier among them), so
+// that all four epilogue warps take the same branch
+__device__ __forceinline__ bool epi_and(bool v) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred p, o;\n\t"
+      "setp.ne.u32 p, %1, 0;\n\t"
+      "bar.red.and.pred o, 1, 128, p;\n\t"
+      "selp.u32 %0, 1, 0, o;\n\t}"
+      : "=r"(r)
+      : "r"((uint32_t)v)
+      : "memory");
+  return r != 0;
+}
+
+template <int NPAD, bool BF16>
+__global__ void __launch_bounds__(THREADS, 1)
+gemm_w8a8_smallm_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmX,
+                        const SmallParams p) {
+  using C = SmallCfg<NPAD>;
+  constexpr int S = C::STAGES;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+  uint8_t* sA = smem;
+  uint8_t* sB = smem + S * SM_A_BYTES;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + S * C::STAGE);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * S + 5);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  volatile int* last_flag = reinterpret_cast<volatile int*>(tmem_slot + 2);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  auto full_bar = [&](int s) { return tc::smem_u32(bars + s); };
+  auto empty_bar = [&](int s) { return tc::smem_u32(bars + S + s); };
+  auto tfull_bar = [&](int b) { return tc::smem_u32(bars + 2 * S + b); };
+  auto tempty_bar = [&](int b) { return tc::smem_u32(bars + 2 * S + 2 + b); };
+  const uint32_t drain_bar = tc::smem_u32(bars + 2 * S + 4);
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < S; ++s) {
+      tc::mbar_init(full_bar(s), 1);
+      tc::mbar_init(empty_bar(s), 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      tc::mbar_init(tfull_bar(b), 1);
+      tc::mbar_init(tempty_bar(b), 4);
+    }
+    tc::mbar_init(drain_bar, 1);
+    *abort_flag = 0;
+    tc::mbar_fence_init();
+    tc::tma_prefetch_desc(&tmW);
+    tc::tma_prefetch_desc(&tmX);
+  }
+  if (warp == 1) {
+    tc::tmem_alloc(tc::smem_u32(tmem_slot), C::TMEM_COLS);
+    tc::tmem_relinquish();
+  }
+  tc::tc_fence_before();
+  __syncthreads();
+  tc::tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+  const int64_t ub = unit_begin(blockIdx.x, p), ue = unit_begin(blockIdx.x + 1, p);
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ TMA producer
+    if (tc::elect_one()) {
+      uint32_t stage = 0, phase = 0, issued = 0, issued_par = 0;
+      bool ok = true;
+      for (int64_t u = ub; ok && u < ue;) {
+        const int tile = (int)(u / p.nk);
+        const int kb0 = (int)(u % p.nk);
+        const int kb1 = (int)min((int64_t)p.nk, kb0 + (ue - u));
+        for (int kb = kb0; kb < kb1; ++kb) {
+          if (!tc::mbar_wait(empty_bar(stage), phase ^ 1u, abort_flag, kWaitNs, p.status)) {
+            ok = false;
+            break;
+          }
+          tc::mbar_arrive_expect_tx(full_bar(stage), C::STAGE);
+          tc::tma_load_2d(tc::smem_u32(sA + stage * SM_A_BYTES), &tmW, kb * BK, tile * SM_BM,
+                          full_bar(stage));
+          tc::tma_load_2d(tc::smem_u32(sB + stage * C::B_BYTES), &tmX, kb * BK, 0, full_bar(stage));
+          issued |= 1u << stage;
+          issued_par = (issued_par & ~(1u << stage)) | (phase << stage);
+          if (++stage == S) { stage = 0; phase ^= 1u; }
+        }
+        u += kb1 - kb0;
+      }
+      if (!ok) {
+        int never = 0;
+        for (int s = 0; s < S; ++s)
+          if (issued & (1u << s))
+            tc::mbar_wait(full_bar(s), (issued_par >> s) & 1u, &never, kDrainNs, p.status);
+      }
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (tc::elect_one()) {
+      constexpr uint32_t idesc = tc::idesc_i8(SM_BM, NPAD);
+      uint32_t stage = 0, phase = 0, abuf = 0, aphase = 0;
+      bool ok = true;
+      for (int64_t u = ub; ok && u < ue;) {
+        const int kb0 = (int)(u % p.nk);
+        const int kb1 = (int)min((int64_t)p.nk, kb0 + (ue - u));
+        if (!tc::mbar_wait(tempty_bar(abuf), aphase ^ 1u, abort_flag, kWaitNs, p.status)) break;
+        tc::tc_fence_after();
+        const uint32_t d = tmem_base + abuf * NPAD;
+        for (int kb = kb0; kb < kb1; ++kb) {
+          if (!tc::mbar_wait(full_bar(stage), phase, abort_flag, kWaitNs, p.status)) {
+            ok = false;
+            break;
+          }
+          tc::tc_fence_after();
+          const uint32_t a0 = tc::smem_u32(sA + stage * SM_A_BYTES);
+          const uint32_t b0 = tc::smem_u32(sB + stage * C::B_BYTES);
+#pragma unroll
+          for (int k = 0; k < BK / UK; ++k)
+            tc::mma_i8(d, tc::desc_k_sw128(a0 + k * UK), tc::desc_k_sw128(b0 + k * UK), idesc,
+                       (kb != kb0) || (k != 0));
+          tc::mma_commit(empty_bar(stage));
+          if (++stage == S) { stage = 0; phase ^= 1u; }
+        }
+        if (!ok) break;
+        tc::mma_commit(tfull_bar(abuf));
+        abuf ^= 1u;
+        if (abuf == 0) aphase ^= 1u;
+        u += kb1 - kb0;
+      }
+      tc::mma_commit(drain_bar);
+      int never = 0;
+      tc::mbar_wait(drain_bar, 0, &never, kDrainNs, p.status);
+    }
+    __syncwarp();
+  } else {
+    // ------------------------------------------------------------ epilogue
+    const int quarter = warp & 3;
+    const int rloc = quarter * 32 + lane;  // output channel within the tile
+    uint32_t abuf = 0, aphase = 0;
+    for (int64_t u = ub; u < ue;) {
+      const int tile = (int)(u / p.nk);
+      const int kb0 = (int)(u % p.nk);
+      const int kb1 = (int)min((int64_t)p.nk, kb0 + (ue - u));
+      const bool full = kb0 == 0 && kb1 == p.nk;
+      const int which = u == ub ? 0 : 1;
+      const bool got = tc::mbar_wait(tfull_bar(abuf), aphase, abort_flag, kWaitNs, p.status);
+      if (!epi_and(got)) break;
+      tc::tc_fence_after();
+      const int n = tile * SM_BM + rloc;
+      const uint32_t taddr = tmem_base + abuf * NPAD + ((uint32_t)(quarter * 32) << 16);
+      int32_t* slot = p.slots + ((int64_t)blockIdx.x * 2 + which) * (int64_t)p.M * SM_BM;
+#pragma unroll 1
+      for (int c0 = 0; c0 < NPAD; c0 += C::CH) {
+        uint32_t r[C::CH];
+        tmem_ld_n<C::CH>(taddr + c0, r);
+        tc::tmem_ld_wait();
+        if (full) {
+          int32_t v[C::CH];
+#pragma unroll
+          for (int i = 0; i < C::CH; ++i) v[i] = (int32_t)r[i];
+          small_store<BF16, C::CH>(p, n, c0, v);
+        } else {
+#pragma unroll
+          for (int i = 0; i < C::CH; ++i)
+            if (c0 + i < p.M) slot[(int64_t)(c0 + i) * SM_BM + rloc] = (int32_t)r[i];
+        }
+      }
+      tc::tc_fence_before();
+      __syncwarp();
+      if (lane == 0) tc::mbar_arrive(tempty_bar(abuf));
+      abuf ^= 1u;
+      if (abuf == 0) aphase ^= 1u;
+      if (!full) {
+        // publish the partial tile, then count arrivals; the last one sums
+        const int64_t gf = unit_owner((int64_t)tile * p.nk, p);
+        const int64_t gl = unit_owner((int64_t)tile * p.nk + p.nk - 1, p);
+        __threadfence();
+        epi_bar();
+        if (threadIdx.x == 64) {
+          const unsigned prev = atomicAdd(p.counters + tile, 1u);
+          *last_flag = prev == (unsigned)(gl - gf);
+        }
+        epi_bar();
+        const bool last = *last_flag != 0;
+        epi_bar();  // every thread has read the flag before it is reused
+        if (last) {
+          __threadfence();
+#pragma unroll 1
+          for (int c0 = 0; c0 < p.M; c0 += C::CH) {
+            int32_t v[C::CH];
+#pragma unroll
+            for (int i = 0; i < C::CH; ++i) v[i] = 0;
+            for (int64_t g = gf; g <= gl; ++g) {
+              const int wg = ((int)(unit_begin(g, p) / p.nk) == tile) ? 0 : 1;
+              const int32_t* sl = p.slots + (g * 2 + wg) * (int64_t)p.M * SM_BM;
+#pragma unroll
+              for (int i = 0; i < C::CH; ++i)
+                if (c0 + i < p.M) v[i] += __ldcg(sl + (int64_t)(c0 + i) * SM_BM + rloc);
+            }
+            small_store<BF16, C::CH>(p, n, c0, v);
+          }
+        }
+      }
+      u += kb1 - kb0;
+    }
+  }
+
+  tc::tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc::tc_fence_after();
+    tc::tmem_dealloc(tmem_base, C::TMEM_COLS);
+  }
+}
+
 // ------------------------------------------------------------------ host side
 PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
 std::once_flag g_encode_once;
@@ -334,16 +623,93 @@ cudaError_t launch_tc(const CUtensorMap& ta, const CUtensorMap& tb, const Params
   return cudaGetLastError();
 }
 
+
+constexpr int64_t kSmallMaxM = 128;
+
+int64_t small_grid(int64_t N, int64_t K) {
+  const int64_t units = ((N + SM_BM - 1) / SM_BM) * ((K + BK - 1) / BK);
+  const int64_t g = sm_count();
+  return units < g ? units : g;
+}
+
+// Workspace of the small-M kernel: the per-tile arrival counters first
+// (zeroed by every call), then the partial-tile slots [grid][2][M][128].
+size_t counters_bytes(int64_t N) {
+  const int64_t n_tiles = (N + SM_BM - 1) / SM_BM;
+  return ((size_t)n_tiles * sizeof(unsigned int) + 255) & ~(size_t)255;
+}
+
+size_t gemm_workspace_bytes_impl(int64_t M, int64_t N, int64_t K) {
+  if (M > kSmallMaxM) return 0;
+  const int64_t G = small_grid(N, K);
+  return counters_bytes(N) + (size_t)G * 2 * (size_t)M * SM_BM * sizeof(int32_t);
+}
+
+template <int NPAD, bool BF16>
+cudaError_t launch_small_t(const CUtensorMap& tw, const CUtensorMap& tx, const SmallParams& p,
+                           cudaStream_t st) {
+  static std::once_flag once[64];
+  static cudaError_t attr_err[64];
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess || dev < 0 || dev >= 64) return e != cudaSuccess ? e : cudaErrorInvalidDevice;
+  std::call_once(once[dev], [&] {
+    attr_err[dev] = cudaFuncSetAttribute(gemm_w8a8_smallm_kernel<NPAD, BF16>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)SmallCfg<NPAD>::SMEM);
+  });
+  if (attr_err[dev] != cudaSuccess) return attr_err[dev];
+  gemm_w8a8_smallm_kernel<NPAD, BF16><<<p.grid, THREADS, SmallCfg<NPAD>::SMEM, st>>>(tw, tx, p);
+  return cudaGetLastError();
+}
+
+template <bool BF16>
+cudaError_t launch_small(const GemmArgs& a, const SmallParams& p, cudaStream_t st) {
+  const int npad = a.M <= 8 ? 8 : a.M <= 16 ? 16 : a.M <= 32 ? 32 : a.M <= 64 ? 64 : 128;
+  CUtensorMap tw, tx;
+  if (!make_tmap(&tw, a.wq, (uint64_t)a.K, (uint64_t)a.N, SM_BM) ||
+      !make_tmap(&tx, a.xq, (uint64_t)a.K, (uint64_t)a.M, (uint32_t)npad))
+    return cudaErrorInvalidValue;
+  switch (npad) {
+    case 8: return launch_small_t<8, BF16>(tw, tx, p, st);
+    case 16: return launch_small_t<16, BF16>(tw, tx, p, st);
+    case 32: return launch_small_t<32, BF16>(tw, tx, p, st);
+    case 64: return launch_small_t<64, BF16>(tw, tx, p, st);
+    default: return launch_small_t<128, BF16>(tw, tx, p, st);
+  }
+}
+
 }  // namespace
 
 size_t gemm_workspace_bytes(int64_t M, int64_t N, int64_t K) {
-  (void)M; (void)N; (void)K;
-  return 0;
+  return gemm_workspace_bytes_impl(M, N, K);
 }
 
 sq_status launch_gemm(const GemmArgs& a, cudaStream_t st) {
   unsigned int* sw = status_word();
   if (!sw) return fail(SQ_ERR_CUDA, "sq_gemm_w8a8: device status word unavailable");
+  if (a.M <= kSmallMaxM) {
+    SmallParams p{};
+    p.M = (int)a.M; p.N = (int)a.N; p.K = (int)a.K;
+    p.n_tiles = (int)((a.N + SM_BM - 1) / SM_BM);
+    p.nk = (int)((a.K + BK - 1) / BK);
+    p.units = (int64_t)p.n_tiles * p.nk;
+    p.grid = (int)small_grid(a.N, a.K);
+    p.act_scale = a.act_scale;
+    p.per_token = a.act_per_token;
+    p.w_scale = a.w_scale;
+    p.y = a.y;
+    p.acc = a.acc_out;
+    p.counters = reinterpret_cast<unsigned int*>(a.workspace);
+    p.slots = reinterpret_cast<int32_t*>(reinterpret_cast<uint8_t*>(a.workspace) +
+                                         counters_bytes(a.N));
+    p.status = sw;
+    cudaError_t e = cudaMemsetAsync(a.workspace, 0, counters_bytes(a.N), st);
+    if (e == cudaSuccess)
+      e = a.yt == SQ_BF16 ? launch_small<true>(a, p, st) : launch_small<false>(a, p, st);
+    if (e != cudaSuccess) return fail(SQ_ERR_CUDA, "sq_gemm_w8a8: %s", cudaGetErrorString(e));
+    return SQ_OK;
+  }
   CUtensorMap ta, tb;
   if (!make_tmap(&ta, a.xq, (uint64_t)a.K, (uint64_t)a.M, BM) ||
       !make_tmap(&tb, a.wq, (uint64_t)a.K, (uint64_t)a.N, BN))
