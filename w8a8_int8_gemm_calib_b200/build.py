@@ -1,6 +1,7 @@
 """Build the sm_100a library libsq_b200.so in-tree with nvcc.
 
-Usage: python -m w8a8_int8_gemm_calib_b200.build [--force] [--verbose]
+Usage: python w8a8_int8_gemm_calib_b200/build.py [--force] [--verbose] [--ptxas]
+(run it as a script: importing the package would load the existing library)
 """
 from __future__ import annotations
 
