@@ -202,6 +202,39 @@ sq_status sq_gemm_w8a8(const int8_t* xq, const int8_t* wq, int64_t M,
                        size_t workspace_bytes, sq_stream stream);
 
 /*
+ * sq_gemm_w8a8_noalloc -- sq_gemm_w8a8 for callers that cannot allocate
+ * device memory.  (No counterpart on the pages: this is a property of the
+ * library interface, not of the method.)
+ *
+ * Some callers cannot call cudaMalloc or hand out a workspace: code running
+ * inside an engine or framework that owns every device allocation and
+ * forbids new ones while it executes, or plugin-style hooks whose execute
+ * step receives only its inputs and outputs.  This entry point takes the
+ * same arguments as sq_gemm_w8a8 minus the workspace and allocates nothing
+ * (no cudaMalloc/cudaFree, no allocating library routine): the scratch the
+ * M <= 128 path needs lives in a fixed array of 8 MiB (8,388,608 bytes) of
+ * device memory that the library reserves on every GPU that loads it, held
+ * until the process exits.
+ *
+ *   - Shapes whose sq_gemm_workspace_bytes(M,N,K) exceeds 8 MiB are refused
+ *     with SQ_ERR_WORKSPACE before anything is launched (at 148 SMs that is
+ *     roughly M > 52 tokens on the M <= 128 path); M > 128 needs no scratch
+ *     and is always served.
+ *   - The first call on a device looks up the array's device address with
+ *     cudaGetSymbolAddress, so make that first call before any stream capture
+ *     begins on that device.
+ *   - Every call on a device uses the same array, and each call resets the
+ *     part of it that must start at zero.  Calls whose executions overlap on
+ *     the GPU (different streams, or different host threads) race on it and
+ *     give wrong results: serialize them.
+ */
+sq_status sq_gemm_w8a8_noalloc(const int8_t* xq, const int8_t* wq, int64_t M,
+                               int64_t N, int64_t K, const float* act_scale,
+                               int act_per_token, const float* w_scale,
+                               void* y, sq_dtype yt, int32_t* acc_out,
+                               sq_stream stream);
+
+/*
  * sq_sync_status -- synchronize `stream`, then return and clear the status
  * word of the current device: SQ_OK, or SQ_ERR_TIMEOUT when a kernel gave up
  * a bounded wait (its outputs are then undefined), or SQ_ERR_CUDA when the

@@ -33,7 +33,7 @@ EXPORTS = [
     "sq_calib_absmax", "sq_smooth_scales", "sq_fuse_weights_q8",
     "sq_ln_smooth_quant_act", "sq_gemm_workspace_bytes", "sq_gemm_w8a8",
     "sq_sync_status", "sq_status_string", "sq_last_error",
-    "sq_selftest_bounded_wait",
+    "sq_selftest_bounded_wait", "sq_gemm_w8a8_noalloc",
 ]
 
 
@@ -47,7 +47,7 @@ def _load() -> ctypes.CDLL:
     if not os.path.exists(LIB_PATH):
         raise ImportError(
             f"{LIB_PATH} is missing: build it with "
-            "`python -m w8a8_int8_gemm_calib_b200.build` (nvcc, sm_100a)")
+            "`python w8a8_int8_gemm_calib_b200/build.py` (nvcc, sm_100a)")
     L = ctypes.CDLL(LIB_PATH)
     p, i64, f, i, sz = ctypes.c_void_p, ctypes.c_int64, ctypes.c_float, ctypes.c_int, ctypes.c_size_t
     st = ctypes.c_int
@@ -64,9 +64,10 @@ def _load() -> ctypes.CDLL:
     L.sq_last_error.argtypes = []
     L.sq_last_error.restype = ctypes.c_char_p
     L.sq_selftest_bounded_wait.argtypes = [i64, p]
+    L.sq_gemm_w8a8_noalloc.argtypes = [p, p, i64, i64, i64, p, i, p, p, i, p, p]
     for fn in ("sq_calib_absmax", "sq_smooth_scales", "sq_fuse_weights_q8",
                "sq_ln_smooth_quant_act", "sq_gemm_w8a8", "sq_sync_status",
-               "sq_selftest_bounded_wait"):
+               "sq_selftest_bounded_wait", "sq_gemm_w8a8_noalloc"):
         getattr(L, fn).restype = st
     return L
 

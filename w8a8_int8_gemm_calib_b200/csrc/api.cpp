@@ -222,6 +222,32 @@ sq_status sq_gemm_w8a8(const int8_t* xq, const int8_t* wq, int64_t M, int64_t N,
   return launch_gemm(a, (cudaStream_t)stream);
 }
 
+sq_status sq_gemm_w8a8_noalloc(const int8_t* xq, const int8_t* wq, int64_t M, int64_t N,
+                               int64_t K, const float* act_scale, int act_per_token,
+                               const float* w_scale, void* y, sq_dtype yt, int32_t* acc_out,
+                               sq_stream stream) {
+  const char* fn = "sq_gemm_w8a8_noalloc";
+  g_last_error[0] = 0;
+  SQ_TRY(check_dtype(yt, fn));
+  if (M < 0 || N < 0) return fail(SQ_ERR_SHAPE, "%s: M=%lld N=%lld must be >= 0", fn,
+                                  (long long)M, (long long)N);
+  SQ_TRY(check_k(K, fn));
+  if (M == 0 || N == 0) return SQ_OK;
+  if (M > (int64_t)1 << 31 || N > (int64_t)1 << 31)
+    return fail(SQ_ERR_SHAPE, "%s: M and N must be below 2^31", fn);
+  SQ_REQ(xq, fn);
+  SQ_REQ(wq, fn);
+  SQ_REQ(act_scale, fn);
+  SQ_REQ(w_scale, fn);
+  SQ_REQ(y, fn);
+  SQ_OPT(acc_out, fn);
+  GemmArgs a{};
+  a.xq = xq; a.wq = wq; a.M = M; a.N = N; a.K = K; a.act_scale = act_scale;
+  a.act_per_token = act_per_token ? 1 : 0; a.w_scale = w_scale; a.y = y; a.yt = yt;
+  a.acc_out = acc_out;
+  return launch_gemm_noalloc(a, (cudaStream_t)stream);
+}
+
 sq_status sq_sync_status(sq_stream stream) {
   g_last_error[0] = 0;
   cudaError_t e = cudaStreamSynchronize((cudaStream_t)stream);

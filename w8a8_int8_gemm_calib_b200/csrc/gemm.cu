@@ -685,6 +685,47 @@ size_t gemm_workspace_bytes(int64_t M, int64_t N, int64_t K) {
   return gemm_workspace_bytes_impl(M, N, K);
 }
 
+// Scratch of sq_gemm_w8a8_noalloc: a fixed array in device memory, reserved
+// on every device that loads this library and kept until the process exits.
+// All calls share it.  Host code only sees a stand-in for it, so its device
+// address is looked up (cudaGetSymbolAddress) once per device, with that
+// device current, the first time the entry point runs there.
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoallocScratchBytes];
+
+namespace {
+std::mutex g_noalloc_mu;
+void* g_noalloc_ptr[64] = {};
+}  // namespace
+
+sq_status launch_gemm_noalloc(GemmArgs a, cudaStream_t st) {
+  const size_t need = gemm_workspace_bytes_impl(a.M, a.N, a.K);
+  if (need > kNoallocScratchBytes)
+    return fail(SQ_ERR_WORKSPACE,
+                "sq_gemm_w8a8_noalloc: M=%lld N=%lld K=%lld needs %zu bytes of scratch; the "
+                "static scratch holds %zu (use sq_gemm_w8a8 with a workspace)",
+                (long long)a.M, (long long)a.N, (long long)a.K, need, kNoallocScratchBytes);
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return fail(SQ_ERR_CUDA, "sq_gemm_w8a8_noalloc: %s", cudaGetErrorString(e));
+  if (dev < 0 || dev >= 64) return fail(SQ_ERR_UNSUPPORTED, "sq_gemm_w8a8_noalloc: device %d", dev);
+  void* scratch = nullptr;
+  {
+    std::lock_guard<std::mutex> lk(g_noalloc_mu);
+    if (!g_noalloc_ptr[dev]) {
+      void* ptr = nullptr;
+      e = cudaGetSymbolAddress(&ptr, g_noalloc_scratch);
+      if (e != cudaSuccess || !ptr)
+        return fail(SQ_ERR_CUDA, "sq_gemm_w8a8_noalloc: cudaGetSymbolAddress: %s",
+                    cudaGetErrorString(e));
+      g_noalloc_ptr[dev] = ptr;
+    }
+    scratch = g_noalloc_ptr[dev];
+  }
+  a.workspace = need ? scratch : nullptr;
+  a.workspace_bytes = need ? kNoallocScratchBytes : 0;
+  return launch_gemm(a, st);
+}
+
 sq_status launch_gemm(const GemmArgs& a, cudaStream_t st) {
   unsigned int* sw = status_word();
   if (!sw) return fail(SQ_ERR_CUDA, "sq_gemm_w8a8: device status word unavailable");

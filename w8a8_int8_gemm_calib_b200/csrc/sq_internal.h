@@ -76,6 +76,11 @@ struct GemmArgs {
 size_t gemm_workspace_bytes(int64_t M, int64_t N, int64_t K);
 sq_status launch_gemm(const GemmArgs& a, cudaStream_t st);
 
+// sq_gemm_w8a8_noalloc: the same GEMM with its scratch in a static device
+// array of kNoallocScratchBytes (gemm.cu).
+constexpr size_t kNoallocScratchBytes = (size_t)8 << 20;
+sq_status launch_gemm_noalloc(GemmArgs a, cudaStream_t st);
+
 // ---------------------------------------------------------------- self test
 cudaError_t launch_wait_selftest(int64_t limit_ns, cudaStream_t st);
 
