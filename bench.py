@@ -215,6 +215,24 @@ class Layer:
         rec(5)
 
 
+def max_over_ranks(value: float, world: int, device) -> float:
+    """Largest value over all ranks (every rank gets it).  Used for the timed
+    milliseconds: the job is as slow as its slowest rank."""
+    if world <= 1:
+        return float(value)
+    import torch
+    import torch.distributed as dist
+
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def throughput_tops(ops_per_step: float, steps: int, world: int, max_ms: float) -> float:
+    """Whole-job TOPS: every rank ran `steps` steps of `ops_per_step` ops."""
+    return world * ops_per_step * steps / (max_ms * 1e-3) / 1e12
+
+
 def algorithmic_bytes(lin):
     """Bytes each step reads/writes once (the per-kernel roofline numerators)."""
     b = 2 if lin.dtype == "bf16" else 4
@@ -287,13 +305,9 @@ def run_ours(args):
             step_ms.append(evs[0].elapsed_time(evs[5]))
         barrier()
     sq.sq_sync_status()
-    total_ms = float(sum(step_ms))
-    if world > 1:
-        t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        total_ms = float(t.item())
+    total_ms = max_over_ranks(float(sum(step_ms)), world, dev)
     ops = 2.0 * lin.T * lin.N * lin.K
-    value = world * ops * K / (total_ms * 1e-3) / 1e12
+    value = throughput_tops(ops, K, world, total_ms)
 
     # ---- e2e through the public API with pinned host buffers
     e2e = run_e2e(sq, torch, layer, lin, d, dev, args.e2e_steps, world, barrier)
@@ -389,15 +403,9 @@ def run_e2e(sq, torch, layer, lin, d, dev, steps, world, barrier):
         one()
     e.record()
     barrier()
-    ms = s.elapsed_time(e) / steps
-    if world > 1:
-        import torch.distributed as dist
-
-        t = torch.tensor([ms], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
+    ms = max_over_ranks(s.elapsed_time(e) / steps, world, dev)
     ops = 2.0 * lin.T * lin.N * lin.K
-    return {"value": round(world * ops / (ms * 1e-3) / 1e12, 3), "unit": "TOPS",
+    return {"value": round(throughput_tops(ops, 1, world, ms), 3), "unit": "TOPS",
             "ms_per_step": round(ms, 4), "h2d_bytes_per_step": int(h2d),
             "d2h_bytes_per_step": int(d2h)}
 

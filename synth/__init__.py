@@ -21,23 +21,53 @@ Every tensor has its own PCG64 sub-stream keyed by (seed, tensor name).
 """
 from __future__ import annotations
 
+import concurrent.futures as cf
+import os
 import zlib
 from dataclasses import dataclass, field
 
 import numpy as np
 
+ROWS_PER_BLOCK = 256  # rows drawn per sub-stream (independent of thread count)
 
-def rng_for(seed: int, name: str) -> np.random.Generator:
-    """Independent PCG64 stream for one named tensor of one workload."""
-    return np.random.Generator(np.random.PCG64([seed, zlib.crc32(name.encode())]))
+
+def rng_for(seed: int, name: str, block: int = 0) -> np.random.Generator:
+    """Independent PCG64 stream for one named tensor (and row block) of one
+    workload."""
+    return np.random.Generator(np.random.PCG64([seed, zlib.crc32(name.encode()), block]))
+
+
+def _normal_rows(seed: int, name: str, T: int, K: int) -> np.ndarray:
+    """[T, K] fp32 N(0,1), drawn in blocks of ROWS_PER_BLOCK rows, each from
+    its own sub-stream, on a thread pool (numpy releases the GIL)."""
+    x = np.empty((T, K), dtype=np.float32)
+    nb = (T + ROWS_PER_BLOCK - 1) // ROWS_PER_BLOCK
+
+    def fill(b):
+        r0 = b * ROWS_PER_BLOCK
+        r1 = min(T, r0 + ROWS_PER_BLOCK)
+        rng_for(seed, name, b).standard_normal((r1 - r0, K), dtype=np.float32, out=x[r0:r1])
+
+    with cf.ThreadPoolExecutor(max_workers=min(32, os.cpu_count() or 1)) as ex:
+        list(ex.map(fill, range(nb)))
+    return x
 
 
 def bf16_bits(x: np.ndarray) -> np.ndarray:
-    """Round fp32 to bf16 (nearest even) and return the raw uint16 patterns."""
-    import torch
+    """Round fp32 to bf16 (nearest even) and return the raw uint16 patterns.
+    (Inputs are finite: the generators draw no NaN.)"""
+    u = np.ascontiguousarray(x, np.float32).view(np.uint32)
+    out = np.empty(u.shape, dtype=np.uint16)
+    flat_u, flat_o = u.reshape(-1), out.reshape(-1)
+    step = 1 << 24
 
-    t = torch.from_numpy(np.ascontiguousarray(x, np.float32)).to(torch.bfloat16)
-    return t.view(torch.int16).numpy().view(np.uint16)
+    def conv(i):
+        v = flat_u[i:i + step]
+        flat_o[i:i + step] = ((v + (np.uint32(0x7FFF) + ((v >> 16) & 1))) >> 16).astype(np.uint16)
+
+    with cf.ThreadPoolExecutor(max_workers=min(32, os.cpu_count() or 1)) as ex:
+        list(ex.map(conv, range(0, flat_u.size, step)))
+    return out
 
 
 def bf16_bits_to_f32(b: np.ndarray) -> np.ndarray:
@@ -63,7 +93,7 @@ def outlier_pattern(seed: int, K: int, frac: float = 0.0, count: int | None = No
 def activations(seed: int, name: str, T: int, K: int, out: Outliers,
                 relu: bool = False) -> np.ndarray:
     """[T, K] fp32 activations with persistent outlier channels."""
-    x = rng_for(seed, name).standard_normal((T, K), dtype=np.float32)
+    x = _normal_rows(seed, name, T, K)
     if out.channels.size:
         x[:, out.channels] *= out.factors[None, :]
     if relu:
@@ -72,7 +102,7 @@ def activations(seed: int, name: str, T: int, K: int, out: Outliers,
 
 
 def weights(seed: int, name: str, N: int, K: int, sigma: float) -> np.ndarray:
-    w = rng_for(seed, name).standard_normal((N, K), dtype=np.float32)
+    w = _normal_rows(seed, name, N, K)
     w *= np.float32(sigma)
     return w
 
@@ -103,6 +133,7 @@ class Linear:
     outlier_count: int | None = None
     relu_input: bool = False
     seed: int = 1000
+    shared: str | None = None  # linears with the same key share W, LN and calibration data
 
 
 @dataclass
@@ -149,7 +180,7 @@ def workloads() -> dict:
         "175B-shaped decode fc1 12288->49152, M in {1,8,32,128}, bf16, 0.3% "
         "outlier channels, INT8 weights streamed from HBM, per-token",
         [Linear(f"fc1_m{m}", 12288, 49152, m, 4096, False, 0.5, True, "bf16", 0.02,
-                outlier_frac=0.003, seed=1003) for m in (1, 8, 32, 128)])
+                outlier_frac=0.003, seed=1003, shared="fc1") for m in (1, 8, 32, 128)])
     w["large_prefill_k8192"] = Workload(
         "large_prefill_k8192",
         "large prefill: absmax over 65536x8192 bf16 calibration tokens, then "
@@ -181,13 +212,14 @@ def make_linear_inputs(lin: Linear, T: int | None = None, T_cal: int | None = No
     out = outlier_pattern(lin.seed, lin.K, lin.outlier_frac, lin.outlier_count,
                           tag=f"k{lin.K}")
     d = {"outliers": out}
-    d["x_cal"] = _store(activations(lin.seed, f"{lin.name}/x_cal", T_cal, lin.K, out,
+    key = lin.shared or lin.name
+    d["x_cal"] = _store(activations(lin.seed, f"{key}/x_cal", T_cal, lin.K, out,
                                     relu=lin.relu_input), lin.dtype)
     d["x"] = _store(activations(lin.seed, f"{lin.name}/x", T, lin.K, out,
                                 relu=lin.relu_input), lin.dtype)
-    d["w"] = _store(weights(lin.seed, f"{lin.name}/w", N, lin.K, lin.w_sigma), lin.dtype)
+    d["w"] = _store(weights(lin.seed, f"{key}/w", N, lin.K, lin.w_sigma), lin.dtype)
     if lin.ln:
-        d["gamma"], d["beta"] = ln_params(lin.seed, f"{lin.name}/ln", lin.K)
+        d["gamma"], d["beta"] = ln_params(lin.seed, f"{key}/ln", lin.K)
     else:
         d["gamma"] = d["beta"] = None
     return d

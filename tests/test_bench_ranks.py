@@ -1,0 +1,62 @@
+"""The multi-rank bits of bench.py on CPU: two gloo ranks agree on the
+slowest rank's time, the whole-job throughput counts every rank's work, and
+the reference arm prints only on rank 0."""
+import os
+import subprocess
+import sys
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _worker(rank, world, port, q):
+    import torch.distributed as dist
+
+    sys.path.insert(0, ROOT)
+    import bench
+
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    local_ms = [12.5, 40.0][rank]
+    mx = bench.max_over_ranks(local_ms, world, "cpu")
+    tops = bench.throughput_tops(2.0e9, 10, world, mx)
+    dist.barrier()
+    dist.destroy_process_group()
+    q.put((rank, mx, tops))
+
+
+def test_two_gloo_ranks_take_the_max():
+    import torch.multiprocessing as mp
+
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = 29600 + os.getpid() % 1000
+    ps = [ctx.Process(target=_worker, args=(r, 2, port, q)) for r in range(2)]
+    for p in ps:
+        p.start()
+    out = sorted(q.get(timeout=120) for _ in ps)
+    for p in ps:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    for rank, mx, tops in out:
+        assert mx == 40.0
+        # 2 ranks x 10 steps x 2e9 ops in 40 ms
+        assert abs(tops - 2 * 10 * 2.0e9 / 0.040 / 1e12) < 1e-12
+
+
+def test_single_rank_is_identity():
+    sys.path.insert(0, ROOT)
+    import bench
+
+    assert bench.max_over_ranks(3.5, 1, "cpu") == 3.5
+
+
+def test_reference_arm_prints_only_on_rank_zero():
+    env = dict(os.environ, RANK="1", WORLD_SIZE="2", LOCAL_RANK="1")
+    r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference",
+                        "--gpus", "2", "--steps", "1", "--warmup", "1"],
+                       env=env, capture_output=True, text=True, timeout=600)
+    assert r.returncode == 0
+    assert r.stdout.strip() == ""

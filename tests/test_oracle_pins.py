@@ -261,7 +261,7 @@ def test_gemm_rows_and_bf16(orc):
     yr, accr = orc.gemm_w8a8(xq, wq, act, ws, rows=rows)
     assert np.array_equal(accr, acc[rows]) and np.array_equal(yr, yf[rows])
     yb, _ = orc.gemm_w8a8(xq, wq, act, ws, out_bf16=True)
-    assert np.array_equal(yb, synth.bf16_bits(yf))
+    assert np.array_equal(yb, _torch_bf16_bits(yf))
     ref = xq.astype(np.int64) @ wq.astype(np.int64).T
     assert np.array_equal(acc, ref)
 
@@ -325,13 +325,25 @@ def test_static_quant_saturates(orc):
     assert ncl == 8
 
 
+def _torch_bf16_bits(v):
+    import torch
+
+    t = torch.from_numpy(np.ascontiguousarray(v, np.float32)).to(torch.bfloat16)
+    return t.view(torch.int16).numpy().view(np.uint16)
+
+
 def test_bf16_rounding_matches_library(orc):
-    """fp32 -> bf16 RNE against torch's conversion, including exact ties."""
+    """fp32 -> bf16 RNE against torch's conversion, including exact ties and
+    NaN (the oracle's and the input generator's casts both)."""
     r = np.random.default_rng(9)
     v = r.standard_normal(3000).astype(np.float32) * 10
     ties = (np.arange(64, dtype=np.uint32) << 16 | 0x8000).view(np.float32)
     v = np.concatenate([v, ties, np.array([0.0, -0.0, 1e-40, 3.4e38], np.float32)])
-    assert np.array_equal(orc.f32_to_bf16_bits(v), synth.bf16_bits(v))
+    want = _torch_bf16_bits(v)
+    assert np.array_equal(orc.f32_to_bf16_bits(v), want)
+    assert np.array_equal(synth.bf16_bits(v), want)
+    nan = orc.f32_to_bf16_bits(np.array([np.nan], np.float32))
+    assert (nan[0] & 0x7F80) == 0x7F80 and (nan[0] & 0x7F) != 0
 
 
 # ------------------------------------------------------------------ P-8 LN

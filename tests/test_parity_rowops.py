@@ -193,3 +193,62 @@ def test_runs_are_deterministic(sq):
         outs.append((host(amax), host(xq), host(act)))
     for a, b_ in zip(outs[0], outs[1]):
         assert_bits_equal(a, b_, "rerun")
+
+
+# Enough rows that every CTA of the row pipeline cycles its shared-memory
+# ring several times (rows per CTA > ring slots), for each ring geometry:
+# 16 slots / 8 slices, 8 / 8, 4 / 4 and 2 slots shared by two 8-warp slices.
+RING_CASES = [
+    (5000, 4096, "ln", True), (2500, 5120, "ln", True), (2500, 8192, "inv_s", False),
+    (1300, 12288, "inv_s", True), (700, 20480, "plain", True), (700, 20480, "inv_s", False),
+]
+
+
+@pytest.mark.parametrize("T,K,mode,per_token", RING_CASES)
+def test_quant_act_ring_reuse(sq, orc, T, K, mode, per_token):
+    x = _x(31, T, K, "bf16", relu=(mode == "plain"))
+    r = np.random.default_rng(T * K)
+    g = b = inv = None
+    if mode == "ln":
+        g, b = _ln(31, K)
+    elif mode == "inv_s":
+        inv = r.uniform(0.02, 2.0, K).astype(np.float32)
+    dstatic = np.float32(0.05)
+    xq_want, act_want, ncl_want = orc.quant_act(
+        x, g, b, 1e-5, inv, per_token=per_token, static_delta=dstatic)
+    xq = torch.empty((T, K), dtype=torch.int8, device="cuda")
+    act = (torch.empty(T, dtype=torch.float32, device="cuda") if per_token
+           else torch.tensor([dstatic], dtype=torch.float32, device="cuda"))
+    ncl = torch.zeros(1, dtype=torch.int64, device="cuda")
+    sq.sq_ln_smooth_quant_act(dev(x), xq, act, dev(g), dev(b), 1e-5, dev(inv),
+                              per_token=per_token, n_clipped=ncl)
+    sq.sq_sync_status()
+    if per_token:
+        assert_bits_equal(host(act), act_want, "act_scale")
+    assert_bits_equal(host(xq), xq_want, "xq")
+    assert int(host(ncl)[0]) == ncl_want
+
+
+@pytest.mark.parametrize("T,K", [(3000, 4096), (3000, 5120), (2000, 1024)])
+def test_calib_absmax_layernorm_ring_reuse(sq, orc, T, K):
+    x = _x(33, T, K, "bf16")
+    g, b = _ln(33, K)
+    want = orc.calib_absmax(x, g, b, 1e-5)
+    amax = torch.zeros(K, dtype=torch.float32, device="cuda")
+    sq.sq_calib_absmax(dev(x), amax, dev(g), dev(b), 1e-5)
+    sq.sq_sync_status()
+    assert_bits_equal(host(amax), want, "amax(LN)")
+
+
+@pytest.mark.parametrize("N,K", [(700, 20480), (1300, 12288), (5000, 4096)])
+def test_fuse_weights_ring_reuse(sq, orc, N, K):
+    r = np.random.default_rng(N + K)
+    w = synth.bf16_bits((r.standard_normal((N, K)) * 0.02).astype(np.float32))
+    s = r.uniform(0.05, 40.0, K).astype(np.float32)
+    wq_want, ws_want = orc.fuse_weights_q8(w, s)
+    wq = torch.empty((N, K), dtype=torch.int8, device="cuda")
+    ws = torch.empty(N, dtype=torch.float32, device="cuda")
+    sq.sq_fuse_weights_q8(dev(w), dev(s), wq, ws)
+    sq.sq_sync_status()
+    assert_bits_equal(host(ws), ws_want, "w_scale")
+    assert_bits_equal(host(wq), wq_want, "wq")

@@ -137,6 +137,12 @@ __device__ __forceinline__ void store_codes(int8_t* dst, const uint32_t (&b)[8])
   *reinterpret_cast<uint2*>(dst) = pk;
 }
 
+// Ring ownership: slice q consumes the CTA's rows i = q, q + NS, ... and row
+// i sits in slot i mod S.  The host makes S a multiple of NS, so each slot
+// is consumed by exactly one slice, in order: a slice waits on a slot only
+// for the phase after the one it released itself, never two phases ahead
+// (mbarrier parity cannot tell those apart).
+//
 // Slices of W warps (ST = 32*W threads).  A slice emulates the 128 canonical
 // LayerNorm slots: thread (v, l) -- warp v of the slice, lane l -- walks the
 // chunks c = 32*v + l + ST*i, i = 0, 1, ...; chunk i belongs to slot
@@ -147,7 +153,8 @@ template <typename T, int W, int CM, bool LN, int MODE>
 __global__ void __launch_bounds__(kThreads, 1) rowpipe_kernel(const Pipe P) {
   constexpr int ST = 32 * W;            // threads per slice
   constexpr int NS = kConsumers / ST;   // slices per CTA
-  constexpr int G = 4 / W;              // slot groups per thread
+  constexpr int G = W <= 4 ? 4 / W : 1;  // slot groups per thread (LayerNorm modes: W <= 4)
+  static_assert(!LN || W == 2 || W == 4, "the LayerNorm order needs 2- or 4-warp slices");
   extern __shared__ __align__(128) uint8_t smem[];
   __shared__ float red[NS][2][3][W];
   __shared__ int abort_s;
@@ -473,21 +480,34 @@ cudaError_t launch_t(const Pipe& P, size_t smem, int grid, cudaStream_t st) {
   return cudaGetLastError();
 }
 
-// Quantizing modes: 64-thread slices (8 rows in flight per SM); the row is
-// held packed in registers when it spans at most 16 chunks per thread
-// (bf16: 64 registers) or 8 (fp32), else each pass re-reads shared memory.
-template <typename T, bool LN, int MODE>
-cudaError_t dispatch_quant(const Pipe& P, size_t smem, int grid, cudaStream_t st) {
+// Quantizing modes.  Slice width W (warps) is chosen by the host from the
+// ring depth: 2 warps (8 slices, 8 rows in process per SM) when 8 or more
+// slots fit, else 4, else -- only without a LayerNorm, whose fixed reduction
+// order needs W <= 4 -- 8 or 16.  The row is held packed in registers when
+// it spans at most 16 chunks per thread (bf16: 64 registers) or 8 (fp32);
+// else each pass re-reads shared memory.
+template <typename T, int W, bool LN, int MODE>
+cudaError_t dispatch_quant_w(const Pipe& P, size_t smem, int grid, cudaStream_t st) {
   constexpr bool kBf16 = sizeof(T) == 2;
-  const int64_t per = (P.a.K / 8 + 63) / 64;
-  if (per <= 2) return launch_t<T, 2, 2, LN, MODE>(P, smem, grid, st);
-  if (per <= 4) return launch_t<T, 2, 4, LN, MODE>(P, smem, grid, st);
-  if (per <= 8) return launch_t<T, 2, 8, LN, MODE>(P, smem, grid, st);
+  const int64_t per = (P.a.K / 8 + 32 * W - 1) / (32 * W);
+  if (per <= 2) return launch_t<T, W, 2, LN, MODE>(P, smem, grid, st);
+  if (per <= 4) return launch_t<T, W, 4, LN, MODE>(P, smem, grid, st);
+  if (per <= 8) return launch_t<T, W, 8, LN, MODE>(P, smem, grid, st);
   if constexpr (kBf16) {
-    if (per <= 12) return launch_t<T, 2, 12, LN, MODE>(P, smem, grid, st);
-    if (per <= 16) return launch_t<T, 2, 16, LN, MODE>(P, smem, grid, st);
+    if (per <= 16) return launch_t<T, W, 16, LN, MODE>(P, smem, grid, st);
   }
-  return launch_t<T, 2, 0, LN, MODE>(P, smem, grid, st);
+  return launch_t<T, W, 0, LN, MODE>(P, smem, grid, st);
+}
+
+template <typename T, bool LN, int MODE>
+cudaError_t dispatch_quant(const Pipe& P, int w, size_t smem, int grid, cudaStream_t st) {
+  if (w == 2) return dispatch_quant_w<T, 2, LN, MODE>(P, smem, grid, st);
+  if (w == 4) return dispatch_quant_w<T, 4, LN, MODE>(P, smem, grid, st);
+  if constexpr (!LN) {
+    if (w == 8) return dispatch_quant_w<T, 8, LN, MODE>(P, smem, grid, st);
+    if (w == 16) return dispatch_quant_w<T, 16, LN, MODE>(P, smem, grid, st);
+  }
+  return cudaErrorInvalidValue;
 }
 
 // Column-peak mode: 128-thread slices; the running peak of each owned
@@ -508,36 +528,58 @@ cudaError_t dispatch_colmax(const Pipe& P, size_t smem, int grid, cudaStream_t s
 }
 
 template <typename T>
-cudaError_t dispatch_mode(const Pipe& P, RowMode mode, size_t smem, int grid, cudaStream_t st) {
+cudaError_t dispatch_mode(const Pipe& P, RowMode mode, int w, size_t smem, int grid,
+                          cudaStream_t st) {
   const bool ln = P.a.g != nullptr;
   switch (mode) {
     case ROW_DYNAMIC:
-      return ln ? dispatch_quant<T, true, ROW_DYNAMIC>(P, smem, grid, st)
-                : dispatch_quant<T, false, ROW_DYNAMIC>(P, smem, grid, st);
+      return ln ? dispatch_quant<T, true, ROW_DYNAMIC>(P, w, smem, grid, st)
+                : dispatch_quant<T, false, ROW_DYNAMIC>(P, w, smem, grid, st);
     case ROW_STATIC:
-      return ln ? dispatch_quant<T, true, ROW_STATIC>(P, smem, grid, st)
-                : dispatch_quant<T, false, ROW_STATIC>(P, smem, grid, st);
+      return ln ? dispatch_quant<T, true, ROW_STATIC>(P, w, smem, grid, st)
+                : dispatch_quant<T, false, ROW_STATIC>(P, w, smem, grid, st);
     case ROW_COLMAX:
       return dispatch_colmax<T>(P, smem, grid, st);
   }
   return cudaErrorInvalidValue;
 }
 
+// Ring depth and slice width: returns false when no valid pairing fits.
+// `slots` is a multiple of the slice count 16/w.
+bool plan(int64_t K, sq_dtype xt, RowMode mode, bool ln, int* slots, int* w, size_t* smem) {
+  const size_t rb = (size_t)K * (xt == SQ_BF16 ? 2 : 4);
+  const size_t fixed = fixed_smem(K, ln, mode);
+  if (fixed + 2 * rb > kSmemBudget) return false;
+  int s = (int)((kSmemBudget - fixed) / rb);
+  if (s > kMaxSlots) s = kMaxSlots;
+  int ww;
+  if (mode == ROW_COLMAX) ww = 4;
+  else if (s >= 8) ww = 2;
+  else if (s >= 4) ww = 4;
+  else if (!ln) ww = 8;  // two slices of 8 warps share the (2 or 3) slots
+  else return false;
+  const int ns = kConsumers / (32 * ww);
+  if (s < ns || s < 2) return false;
+  s = (s / ns) * ns;
+  *slots = s;
+  *w = ww;
+  *smem = (size_t)s * rb + fixed;
+  return true;
+}
+
 }  // namespace
 
 bool rowpipe_fits(int64_t K, sq_dtype xt, RowMode mode, bool ln) {
-  const size_t rb = (size_t)K * (xt == SQ_BF16 ? 2 : 4);
-  const size_t fixed = fixed_smem(K, ln, mode);
-  return fixed + 2 * rb <= kSmemBudget;
+  int slots, w;
+  size_t smem;
+  return plan(K, xt, mode, ln, &slots, &w, &smem);
 }
 
 cudaError_t launch_rowpipe(const RowArgs& a, sq_dtype xt, RowMode mode, cudaStream_t st) {
   const size_t rb = (size_t)a.K * (xt == SQ_BF16 ? 2 : 4);
-  const bool ln = a.g != nullptr;
-  const size_t fixed = fixed_smem(a.K, ln, mode);
-  int slots = (int)((kSmemBudget - fixed) / rb);
-  if (slots > kMaxSlots) slots = kMaxSlots;
-  if (slots < 2) return cudaErrorInvalidValue;
+  int slots = 0, w = 0;
+  size_t smem = 0;
+  if (!plan(a.K, xt, mode, a.g != nullptr, &slots, &w, &smem)) return cudaErrorInvalidValue;
   unsigned int* sw = status_word();
   if (!sw) return cudaErrorInvalidDevice;
   int grid = sm_count();
@@ -550,9 +592,8 @@ cudaError_t launch_rowpipe(const RowArgs& a, sq_dtype xt, RowMode mode, cudaStre
   P.slots = slots;
   P.count = a.n_clipped != nullptr;
   P.status = sw;
-  const size_t smem = (size_t)slots * rb + fixed;
-  return xt == SQ_BF16 ? dispatch_mode<uint16_t>(P, mode, smem, grid, st)
-                       : dispatch_mode<float>(P, mode, smem, grid, st);
+  return xt == SQ_BF16 ? dispatch_mode<uint16_t>(P, mode, w, smem, grid, st)
+                       : dispatch_mode<float>(P, mode, w, smem, grid, st);
 }
 
 }  // namespace sq
