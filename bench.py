@@ -66,6 +66,8 @@ def parse():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--e2e-steps", type=int, default=20)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-small-m", action="store_true",
+                    help="skip the decode-shaped (small-M) GEMM measurement")
     return ap.parse_args()
 
 
@@ -311,6 +313,7 @@ def run_ours(args):
 
     # ---- e2e through the public API with pinned host buffers
     e2e = run_e2e(sq, torch, layer, lin, d, dev, args.e2e_steps, world, barrier)
+    small_m = None if args.no_small_m else run_small_m(sq, torch, dev, flush)
 
     peaks, peak_kind = load_peaks()
     bf16_peak = peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"])
@@ -354,6 +357,7 @@ def run_ours(args):
                          "(nominal int8:bf16 ratio); 'TFLOP/s' here counts int8 ops",
         },
         "kernels": kernels,
+        "small_m_decode": small_m,
         "e2e": e2e,
         "gpu_launches": layer.kernels_per_step * K,
         "clocks": clocks.summary(),
@@ -365,6 +369,51 @@ def run_ours(args):
         dist.destroy_process_group()
     if rank == 0:
         print(json.dumps(line), flush=True)
+
+
+def run_small_m(sq, torch, dev, flush, reps=20):
+    """The metric's small-M half: the INT8 GEMM of the 175B-shaped decode fc1
+    (K=12288 -> N=49152) at M = 1, 8, 32, 128 tokens, per-token scales, bf16
+    out, on seeded random INT8 operands (604 MB of weights streamed from HBM
+    each call).  One CUDA-graph replay per call, L2 flushed before each,
+    device events around it; GB/s = algorithmic bytes / time."""
+    lin = next(l for l in synth.workloads()["175b_fc1_decode"].linears)
+    N, K = lin.N, lin.K
+    g = torch.Generator(device=dev).manual_seed(1003)
+    wq = torch.randint(-127, 128, (N, K), dtype=torch.int8, device=dev, generator=g)
+    ws = torch.rand(N, device=dev, generator=g) * 1e-3 + 1e-5
+    hbm = load_peaks()[0].get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"])
+    out = {"workload": "175b_fc1_decode: fc1 12288->49152, per-token, bf16 out",
+           "kernel": "gemm_w8a8 weight-streaming path (tcgen05 kind::i8, stream-K)",
+           "hbm_peak_gbs": hbm}
+    for M in (1, 8, 32, 128):
+        xq = torch.randint(-127, 128, (M, K), dtype=torch.int8, device=dev, generator=g)
+        act = torch.rand(M, device=dev, generator=g) * 1e-2 + 1e-4
+        y = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+        wsp = sq.Workspace(dev)
+        for _ in range(3):
+            sq.sq_gemm_w8a8(xq, wq, act, ws, y, workspace=wsp)
+        e0 = torch.cuda.Event(enable_timing=True, external=True)
+        e1 = torch.cuda.Event(enable_timing=True, external=True)
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph):
+            e0.record()
+            sq.sq_gemm_w8a8(xq, wq, act, ws, y, workspace=wsp)
+            e1.record()
+        times = []
+        for i in range(reps):
+            flush.fill_(i)
+            graph.replay()
+            torch.cuda.synchronize()
+            times.append(e0.elapsed_time(e1))
+        sq.sq_sync_status()
+        ms = statistics.mean(times)
+        nbytes = M * K + N * K + M * N * 2 + 4 * N + 4 * M
+        gbs = nbytes / (ms * 1e-3) / 1e9
+        out[f"M{M}"] = {"us": round(ms * 1e3, 2), "gbs": round(gbs, 1),
+                        "hbm_frac": round(gbs / hbm, 3), "bytes": int(nbytes)}
+        del graph
+    return out
 
 
 def run_e2e(sq, torch, layer, lin, d, dev, steps, world, barrier):
