@@ -45,6 +45,11 @@ FLUSH_BYTES = 256 << 20
 # (4.5 POPS : 2.25 PFLOP/s = 2).
 INT8_PER_BF16 = 2.0
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+# DRAM bytes (read + write) of one launch of the dominant kernel, from the ncu
+# capture summarised in profiles/ (null when the kernel has changed since)
+GEMM_DRAM_TRAFFIC = {
+    "opt6.7b_qkv_t2048": (67.81e6, "profiles/gemm_w8a8_tc_opt6.7b_qkv_t2048.md"),
+}
 
 
 def load_peaks():
@@ -352,7 +357,8 @@ def run_ours(args):
             "peak": round(int8_peak, 1),
             "unit": "TFLOP/s",
             "frac": round(gemm_tops / int8_peak, 4),
-            "traffic": None,
+            "traffic": GEMM_DRAM_TRAFFIC.get(wl.name, (None, None))[0],
+            "traffic_source": GEMM_DRAM_TRAFFIC.get(wl.name, (None, None))[1],
             "peak_note": f"int8 dense = {peak_kind} bf16 burst {bf16_peak} TFLOP/s x 2 "
                          "(nominal int8:bf16 ratio); 'TFLOP/s' here counts int8 ops",
         },
