@@ -17,6 +17,10 @@ LIB = os.path.join(HERE, "libsq_b200.so")
 INCLUDE = os.path.join(os.path.dirname(HERE), "include")
 
 SOURCES = ["api.cpp", "status.cu", "rowops.cu", "rowpipe.cu", "gemm.cu"]
+# The row pipeline's packed fp32 multiplies and adds must stay separately
+# rounded (the INT8 codes are bit-exact against the oracle); its one intended
+# fused multiply-add is an explicit intrinsic, which this flag leaves alone.
+EXTRA_FLAGS = {"rowpipe.cu": ["-fmad=false"]}
 HEADERS = ["sq_internal.h", "sq_device.cuh", "tc_ptx.cuh"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 NVCC_FLAGS = ["-O3", "-std=c++17", "-lineinfo", "-Xcompiler", "-fPIC",
@@ -37,7 +41,8 @@ def _stale(target: str, deps: list[str]) -> bool:
 
 def build(force: bool = False, verbose: bool = False, ptxas_verbose: bool = False) -> str:
     os.makedirs(OBJ, exist_ok=True)
-    hdrs = [os.path.join(CSRC, h) for h in HEADERS] + [os.path.join(INCLUDE, "sq.h")]
+    hdrs = [os.path.join(CSRC, h) for h in HEADERS] + [os.path.join(INCLUDE, "sq.h"),
+                                                        os.path.abspath(__file__)]
     jobs = []
     objs = []
     for src in SOURCES:
@@ -45,7 +50,7 @@ def build(force: bool = False, verbose: bool = False, ptxas_verbose: bool = Fals
         o = os.path.join(OBJ, src + ".o")
         objs.append(o)
         if force or _stale(o, [s] + hdrs):
-            cmd = [nvcc(), *ARCH, *NVCC_FLAGS, "-c", s, "-o", o]
+            cmd = [nvcc(), *ARCH, *NVCC_FLAGS, *EXTRA_FLAGS.get(src, []), "-c", s, "-o", o]
             if ptxas_verbose and src.endswith(".cu"):
                 cmd += ["-Xptxas", "-v"]
             jobs.append(cmd)

@@ -84,8 +84,11 @@ colmax_kernel(const T* __restrict__ x, int64_t T_, int64_t K, int64_t rows_per_s
   if (k < K) atomicMax(out + k, __float_as_uint(v));
 }
 
-cudaError_t launch_colmax(const void* x, sq_dtype xt, int64_t T, int64_t K,
-                          float* out, cudaStream_t st) {
+// Column strips stream the rows with plain 16-byte loads and no
+// synchronisation at all; measured faster here than staging whole rows
+// through the shared-memory ring (which pays a handshake per row).
+cudaError_t launch_colmax(const void* x, sq_dtype xt, int64_t T, int64_t K, float* out,
+                          cudaStream_t st) {
   const int64_t strips = (K + 255) / 256;
   static std::once_flag once[2][64];
   static int occ[2][64];

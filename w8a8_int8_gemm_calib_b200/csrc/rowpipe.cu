@@ -91,27 +91,77 @@ template <typename T> struct RawC;
 template <> struct RawC<uint16_t> { uint4 a; };
 template <> struct RawC<float> { uint4 a, b; };
 
-__device__ __forceinline__ void lds_raw(const uint8_t* row, int64_t c, RawC<uint16_t>& r) {
+__device__ __forceinline__ void lds_raw(const uint8_t* row, int c, RawC<uint16_t>& r) {
   r.a = *reinterpret_cast<const uint4*>(row + c * 16);
 }
-__device__ __forceinline__ void lds_raw(const uint8_t* row, int64_t c, RawC<float>& r) {
+__device__ __forceinline__ void lds_raw(const uint8_t* row, int c, RawC<float>& r) {
   r.a = *reinterpret_cast<const uint4*>(row + c * 32);
   r.b = *reinterpret_cast<const uint4*>(row + c * 32 + 16);
 }
-__device__ __forceinline__ void unpack8(const RawC<uint16_t>& r, float (&v)[8]) {
-  v[0] = bf16lo(r.a.x); v[1] = bf16hi(r.a.x); v[2] = bf16lo(r.a.y); v[3] = bf16hi(r.a.y);
-  v[4] = bf16lo(r.a.z); v[5] = bf16hi(r.a.z); v[6] = bf16lo(r.a.w); v[7] = bf16hi(r.a.w);
+// a chunk as four (even, odd) element pairs
+__device__ __forceinline__ void unpack8(const RawC<uint16_t>& r, float2 (&v)[4]) {
+  v[0] = make_float2(bf16lo(r.a.x), bf16hi(r.a.x));
+  v[1] = make_float2(bf16lo(r.a.y), bf16hi(r.a.y));
+  v[2] = make_float2(bf16lo(r.a.z), bf16hi(r.a.z));
+  v[3] = make_float2(bf16lo(r.a.w), bf16hi(r.a.w));
 }
-__device__ __forceinline__ void unpack8(const RawC<float>& r, float (&v)[8]) {
-  v[0] = __uint_as_float(r.a.x); v[1] = __uint_as_float(r.a.y);
-  v[2] = __uint_as_float(r.a.z); v[3] = __uint_as_float(r.a.w);
-  v[4] = __uint_as_float(r.b.x); v[5] = __uint_as_float(r.b.y);
-  v[6] = __uint_as_float(r.b.z); v[7] = __uint_as_float(r.b.w);
+__device__ __forceinline__ void unpack8(const RawC<float>& r, float2 (&v)[4]) {
+  v[0] = make_float2(__uint_as_float(r.a.x), __uint_as_float(r.a.y));
+  v[1] = make_float2(__uint_as_float(r.a.z), __uint_as_float(r.a.w));
+  v[2] = make_float2(__uint_as_float(r.b.x), __uint_as_float(r.b.y));
+  v[3] = make_float2(__uint_as_float(r.b.z), __uint_as_float(r.b.w));
 }
-__device__ __forceinline__ void lds8(const float* p, float (&v)[8]) {
-  const float4 a = *reinterpret_cast<const float4*>(p);
-  const float4 b = *reinterpret_cast<const float4*>(p + 4);
-  v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w; v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
+
+// Per-column parameters live in shared memory in a split layout: elements
+// 0-3 of chunk c at [4c, 4c+4), elements 4-7 at [K/2 + 4c, K/2 + 4c + 4).
+// Lanes that read consecutive chunks then read consecutive 16-byte words
+// (a 128-bit load per lane without bank conflicts).
+__device__ __forceinline__ int param_index(int k, int half) {
+  const int c = k >> 3, e = k & 7;
+  return e < 4 ? c * 4 + e : half + c * 4 + (e - 4);
+}
+__device__ __forceinline__ void lds8(const float* p, int c, int half, float2 (&v)[4]) {
+  const float4 a = *reinterpret_cast<const float4*>(p + c * 4);
+  const float4 b = *reinterpret_cast<const float4*>(p + half + c * 4);
+  v[0] = make_float2(a.x, a.y); v[1] = make_float2(a.z, a.w);
+  v[2] = make_float2(b.x, b.y); v[3] = make_float2(b.z, b.w);
+}
+
+// Packed (even, odd) fp32 add and multiply, each lane one IEEE
+// round-to-nearest operation.  They are used only where no multiply feeds an
+// add: the code generator was seen to fuse a packed multiply and a following
+// packed add into one fused multiply-add (one rounding instead of two) even
+// with the explicit .rn modifier and -fmad=false.  Every add that follows a
+// multiply is the scalar __fadd_rn, which is never fused.
+__device__ __forceinline__ float2 add2(float2 a, float2 b) {
+  float2 r;
+  asm("{\n\t.reg .b64 pa, pb, pd;\n\t"
+      "mov.b64 pa, {%2, %3};\n\t"
+      "mov.b64 pb, {%4, %5};\n\t"
+      "add.rn.f32x2 pd, pa, pb;\n\t"
+      "mov.b64 {%0, %1}, pd;\n\t}"
+      : "=f"(r.x), "=f"(r.y)
+      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+  return r;
+}
+__device__ __forceinline__ float2 mul2(float2 a, float2 b) {
+  float2 r;
+  asm("{\n\t.reg .b64 pa, pb, pd;\n\t"
+      "mov.b64 pa, {%2, %3};\n\t"
+      "mov.b64 pb, {%4, %5};\n\t"
+      "mul.rn.f32x2 pd, pa, pb;\n\t"
+      "mov.b64 {%0, %1}, pd;\n\t}"
+      : "=f"(r.x), "=f"(r.y)
+      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+  return r;
+}
+
+// max(|m|, |y|) with NaN propagated (the sign bit of the result is not
+// meaningful: callers take the magnitude at the end)
+__device__ __forceinline__ float maxabs_nan(float m, float y) {
+  float r;
+  asm("max.NaN.xorsign.abs.f32 %0, %1, %2;" : "=f"(r) : "f"(m), "f"(y));
+  return r;
 }
 
 // Q(y; Delta) given inv = 1/Delta, as the fp32 whose low byte is the code:
@@ -123,17 +173,16 @@ __device__ __forceinline__ uint32_t qbits(float y, float inv, bool count, unsign
   r = fminf(fmaxf(r, -127.0f), 127.0f);
   return __float_as_uint(__fadd_rn(r, kRoundMagic));
 }
-// Per-token form for rows whose elements are all finite: |y| <= m and
-// inv = 1/fl(max(m,1e-7)/127) give |y*inv| <= 127*(1+2^-23) < 127.5, so no
-// element can saturate and no clamp is needed.
-__device__ __forceinline__ uint32_t qbits_fast(float y, float inv) {
-  return __float_as_uint(__fadd_rn(__fmul_rn(y, inv), kRoundMagic));
-}
 
+__device__ __forceinline__ uint32_t pack4u(uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
+  const uint32_t lo = __byte_perm(a, b, 0x0040);
+  const uint32_t hi = __byte_perm(c, d, 0x0040);
+  return __byte_perm(lo, hi, 0x5410);
+}
 __device__ __forceinline__ void store_codes(int8_t* dst, const uint32_t (&b)[8]) {
   uint2 pk;
-  pk.x = pack4((int)b[0], (int)b[1], (int)b[2], (int)b[3]);
-  pk.y = pack4((int)b[4], (int)b[5], (int)b[6], (int)b[7]);
+  pk.x = pack4u(b[0], b[1], b[2], b[3]);
+  pk.y = pack4u(b[4], b[5], b[6], b[7]);
   *reinterpret_cast<uint2*>(dst) = pk;
 }
 
@@ -149,12 +198,19 @@ __device__ __forceinline__ void store_codes(int8_t* dst, const uint32_t (&b)[8])
 // 32*(v + W*(i mod G)) + l with G = 4/W slot groups per thread, so each slot
 // still accumulates its own chunks in increasing c.  The slot groups are
 // then combined exactly as (r0 + r2) + (r1 + r3).
+//
+// Element-wise arithmetic runs on (even, odd) pairs with the packed fp32
+// instructions (add2, mul2) where no multiply feeds an add: each lane is the
+// same IEEE round-to-nearest operation as its scalar form; x - mu is
+// computed as x + (-mu), which IEEE defines identically.  The running sums of the
+// LayerNorm stay scalar (their order is fixed).
 template <typename T, int W, int CM, bool LN, int MODE>
 __global__ void __launch_bounds__(kThreads, 1) rowpipe_kernel(const Pipe P) {
   constexpr int ST = 32 * W;            // threads per slice
   constexpr int NS = kConsumers / ST;   // slices per CTA
   constexpr int G = W <= 4 ? 4 / W : 1;  // slot groups per thread (LayerNorm modes: W <= 4)
   static_assert(!LN || W == 2 || W == 4, "the LayerNorm order needs 2- or 4-warp slices");
+  static_assert(MODE != ROW_COLMAX || LN, "raw column peaks use the column-strip kernel");
   extern __shared__ __align__(128) uint8_t smem[];
   __shared__ float red[NS][2][3][W];
   __shared__ int abort_s;
@@ -174,17 +230,7 @@ __global__ void __launch_bounds__(kThreads, 1) rowpipe_kernel(const Pipe P) {
 
   const int tid = threadIdx.x;
   const bool has_mul = !LN && a.mul != nullptr;
-  if (tid < kConsumers) {
-    for (int64_t k = tid; k < K; k += kConsumers) {
-      if (LN) {
-        pg[k] = a.g[k];
-        pb[k] = a.b ? a.b[k] : 0.0f;
-      } else if (has_mul) {
-        pg[k] = a.mul[k];
-      }
-      if (MODE == ROW_COLMAX) colmax_s[k] = 0u;
-    }
-  }
+  const int khalf = (int)(K >> 1);
   if (tid == 0) {
     for (int s = 0; s < S; ++s) {
       tc::mbar_init(full_bar(s), 1);
@@ -204,6 +250,7 @@ __global__ void __launch_bounds__(kThreads, 1) rowpipe_kernel(const Pipe P) {
 
   if (tid >= kConsumers) {
     // ------------------------------------------------------------ producer
+    // (starts streaming rows while the consumers stage the parameters)
     if (tid == kConsumers) {
       uint32_t issued = 0, issued_par = 0;
       bool ok = true;
@@ -234,6 +281,18 @@ __global__ void __launch_bounds__(kThreads, 1) rowpipe_kernel(const Pipe P) {
     }
   } else {
     // ------------------------------------------------------------ consumers
+    for (int k = tid; k < (int)K; k += kConsumers) {
+      const int pk = param_index(k, khalf);
+      if (LN) {
+        pg[pk] = a.g[k];
+        pb[pk] = a.b ? a.b[k] : 0.0f;
+      } else if (has_mul) {
+        pg[pk] = a.mul[k];
+      }
+      if (MODE == ROW_COLMAX) colmax_s[k] = 0u;
+    }
+    asm volatile("bar.sync 9, %0;" ::"r"(kConsumers) : "memory");  // consumers only
+
     const int q = tid / ST, j = tid % ST;
     const int v = j >> 5, lane = j & 31;
     const float kf = (float)K;
@@ -244,13 +303,14 @@ __global__ void __launch_bounds__(kThreads, 1) rowpipe_kernel(const Pipe P) {
     const float static_inv = MODE == ROW_STATIC ? __fdiv_rn(1.0f, __ldg(a.scale)) : 0.0f;
     const bool count = P.count != 0;
     int parity = 0;
-    auto chunk_of = [&](int i) -> int64_t { return 32 * v + lane + (int64_t)ST * i; };
+    const int nch = (int)nchunk;  // < 2^14 here: rows fit in shared memory
+    auto chunk_of = [&](int i) -> int { return 32 * v + lane + ST * i; };
     auto sync = [&]() { slice_sync_t<ST>(q); };
 
     for (int64_t i = q; i < R; i += NS) {
       const int s = (int)(i % S);
       const int64_t u = i / S;
-      bool ok = tc::mbar_wait(full_bar(s), (uint32_t)(u & 1), abort_flag, kWaitNs, P.status);
+      const bool ok = tc::mbar_wait(full_bar(s), (uint32_t)(u & 1), abort_flag, kWaitNs, P.status);
       if (!slice_and_t<ST>(q, ok)) break;
       const uint8_t* rowp = ring + (size_t)s * RB;
       const int64_t row = r0 + i;
@@ -259,26 +319,26 @@ __global__ void __launch_bounds__(kThreads, 1) rowpipe_kernel(const Pipe P) {
       if constexpr (CM > 0) {
 #pragma unroll
         for (int m = 0; m < CM; ++m)
-          if (chunk_of(m) < nchunk) lds_raw(rowp, chunk_of(m), xr[m]);
+          if (chunk_of(m) < nch) lds_raw(rowp, chunk_of(m), xr[m]);
       }
-      // f(m, c, x[8]) over the thread's chunks in increasing c
+      // f(m, c, x[4]) over the thread's chunks in increasing c
       auto for_chunks = [&](auto&& f) {
         if constexpr (CM > 0) {
 #pragma unroll
           for (int m = 0; m < CM; ++m) {
-            const int64_t c = chunk_of(m);
-            if (c < nchunk) {
-              float x[8];
+            const int c = chunk_of(m);
+            if (c < nch) {
+              float2 x[4];
               unpack8(xr[m], x);
               f(m, c, x);
             }
           }
         } else {
           int m = 0;
-          for (int64_t c = chunk_of(0); c < nchunk; c += ST, ++m) {
+          for (int c = chunk_of(0); c < nch; c += ST, ++m) {
             RawC<T> r;
             lds_raw(rowp, c, r);
-            float x[8];
+            float2 x[4];
             unpack8(r, x);
             f(m, c, x);
           }
@@ -298,98 +358,111 @@ __global__ void __launch_bounds__(kThreads, 1) rowpipe_kernel(const Pipe P) {
         else return __fadd_rn(r[0], r[1]);
       };
 
-      float mu = 0.0f, rstd = 0.0f;
+      float2 negmu2 = make_float2(0.0f, 0.0f), rstd2 = make_float2(0.0f, 0.0f);
       if constexpr (LN) {
         float p[G];
 #pragma unroll
         for (int g = 0; g < G; ++g) p[g] = 0.0f;
-        for_chunks([&](int m, int64_t, const float (&x)[8]) {
+        for_chunks([&](int m, int, const float2 (&x)[4]) {
 #pragma unroll
-          for (int e = 0; e < 8; ++e) p[m % G] = __fadd_rn(p[m % G], x[e]);
-        });
-        mu = __fdiv_rn(slot_sum(p, 0), kf);
-#pragma unroll
-        for (int g = 0; g < G; ++g) p[g] = 0.0f;
-        for_chunks([&](int m, int64_t, const float (&x)[8]) {
-#pragma unroll
-          for (int e = 0; e < 8; ++e) {
-            const float d = __fsub_rn(x[e], mu);
-            p[m % G] = __fmaf_rn(d, d, p[m % G]);
+          for (int e = 0; e < 4; ++e) {
+            p[m % G] = __fadd_rn(p[m % G], x[e].x);
+            p[m % G] = __fadd_rn(p[m % G], x[e].y);
           }
         });
-        rstd = __fdiv_rn(1.0f, __fsqrt_rn(__fadd_rn(__fdiv_rn(slot_sum(p, 1), kf), a.eps)));
-      }
-      auto ychunk = [&](int64_t c, const float (&x)[8], float (&y)[8]) {
-        if constexpr (LN) {
-          float g8[8], b8[8];
-          lds8(pg + c * 8, g8);
-          lds8(pb + c * 8, b8);
+        const float mu = __fdiv_rn(slot_sum(p, 0), kf);
+        negmu2 = make_float2(-mu, -mu);
 #pragma unroll
-          for (int e = 0; e < 8; ++e)
-            y[e] = __fadd_rn(__fmul_rn(__fmul_rn(__fsub_rn(x[e], mu), rstd), g8[e]), b8[e]);
+        for (int g = 0; g < G; ++g) p[g] = 0.0f;
+        for_chunks([&](int m, int, const float2 (&x)[4]) {
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const float2 d = add2(x[e], negmu2);
+            p[m % G] = __fmaf_rn(d.x, d.x, p[m % G]);
+            p[m % G] = __fmaf_rn(d.y, d.y, p[m % G]);
+          }
+        });
+        const float rstd = __fdiv_rn(1.0f, __fsqrt_rn(__fadd_rn(__fdiv_rn(slot_sum(p, 1), kf), a.eps)));
+        rstd2 = make_float2(rstd, rstd);
+      }
+      // y of one chunk: ((x - mu) * rstd) * g + b, or x * m, or x
+      auto ychunk = [&](int c, const float2 (&x)[4], float2 (&y)[4]) {
+        if constexpr (LN) {
+          float2 g8[4], b8[4];
+          lds8(pg, c, khalf, g8);
+          lds8(pb, c, khalf, b8);
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const float2 t = mul2(mul2(add2(x[e], negmu2), rstd2), g8[e]);
+            y[e] = make_float2(__fadd_rn(t.x, b8[e].x), __fadd_rn(t.y, b8[e].y));
+          }
         } else {
           if (has_mul) {
-            float m8[8];
-            lds8(pg + c * 8, m8);
+            float2 m8[4];
+            lds8(pg, c, khalf, m8);
 #pragma unroll
-            for (int e = 0; e < 8; ++e) y[e] = __fmul_rn(x[e], m8[e]);
+            for (int e = 0; e < 4; ++e) y[e] = mul2(x[e], m8[e]);
           } else {
 #pragma unroll
-            for (int e = 0; e < 8; ++e) y[e] = x[e];
+            for (int e = 0; e < 4; ++e) y[e] = x[e];
           }
         }
       };
 
       if constexpr (MODE == ROW_COLMAX) {
-        for_chunks([&](int m, int64_t c, const float (&x)[8]) {
-          float y[8];
+        for_chunks([&](int m, int c, const float2 (&x)[4]) {
+          float2 y[4];
           ychunk(c, x, y);
 #pragma unroll
-          for (int e = 0; e < 8; ++e) {
+          for (int e = 0; e < 4; ++e) {
             if constexpr (CM > 0) {
-              cmax[m * 8 + e] = fmaxf(cmax[m * 8 + e], fabsf(y[e]));
+              cmax[m * 8 + 2 * e] = fmaxf(cmax[m * 8 + 2 * e], fabsf(y[e].x));
+              cmax[m * 8 + 2 * e + 1] = fmaxf(cmax[m * 8 + 2 * e + 1], fabsf(y[e].y));
             } else {
-              atomicMax(&colmax_s[c * 8 + e], __float_as_uint(fabsf(y[e])));
+              atomicMax(&colmax_s[c * 8 + 2 * e], __float_as_uint(fabsf(y[e].x)));
+              atomicMax(&colmax_s[c * 8 + 2 * e + 1], __float_as_uint(fabsf(y[e].y)));
             }
           }
         });
       } else if constexpr (MODE == ROW_STATIC) {
         int8_t* qr = a.q + row * K;
-        for_chunks([&](int, int64_t c, const float (&x)[8]) {
-          float y[8];
+        for_chunks([&](int, int c, const float2 (&x)[4]) {
+          float2 y[4];
           ychunk(c, x, y);
           uint32_t b[8];
 #pragma unroll
-          for (int e = 0; e < 8; ++e) b[e] = qbits(y[e], static_inv, count, clipped);
+          for (int e = 0; e < 4; ++e) {
+            b[2 * e] = qbits(y[e].x, static_inv, count, clipped);
+            b[2 * e + 1] = qbits(y[e].y, static_inv, count, clipped);
+          }
           store_codes(qr + c * 8, b);
         });
       } else {
-        // peak of |y| as the maximum of the fp32 bit patterns: exact for
-        // finite values, and any inf/NaN element shows up as a pattern at or
-        // above that of +inf
-        uint32_t mb = 0;
-        for_chunks([&](int, int64_t c, const float (&x)[8]) {
-          float y[8];
+        // peak magnitude with NaN propagated: a finite result means every
+        // element is finite (and then it equals the NaN-ignoring peak)
+        float mn = 0.0f;
+        for_chunks([&](int, int c, const float2 (&x)[4]) {
+          float2 y[4];
           ychunk(c, x, y);
 #pragma unroll
-          for (int e = 0; e < 8; ++e) mb = max(mb, __float_as_uint(fabsf(y[e])));
+          for (int e = 0; e < 4; ++e) mn = maxabs_nan(maxabs_nan(mn, y[e].x), y[e].y);
         });
 #pragma unroll
-        for (int o = 16; o >= 1; o >>= 1) mb = max(mb, __shfl_xor_sync(0xffffffffu, mb, o));
-        if (lane == 0) red[q][parity][2][v] = __uint_as_float(mb);
+        for (int o = 16; o >= 1; o >>= 1) mn = maxabs_nan(mn, __shfl_xor_sync(0xffffffffu, mn, o));
+        if (lane == 0) red[q][parity][2][v] = mn;
         sync();
 #pragma unroll
-        for (int t = 0; t < W; ++t) mb = max(mb, __float_as_uint(red[q][parity][2][t]));
-        const bool clean = mb < 0x7f800000u;
-        float mx = __uint_as_float(mb);
+        for (int t = 0; t < W; ++t) mn = maxabs_nan(mn, red[q][parity][2][t]);
+        float mx = fabsf(mn);
+        const bool clean = mx < INFINITY;  // false for inf and NaN
         if (!clean) {
-          // non-finite elements: the peak over the non-NaN values, as fmaxf
+          // non-finite elements: the peak over the non-NaN values (fmaxf)
           float m2 = 0.0f;
-          for_chunks([&](int, int64_t c, const float (&x)[8]) {
-            float y[8];
+          for_chunks([&](int, int c, const float2 (&x)[4]) {
+            float2 y[4];
             ychunk(c, x, y);
 #pragma unroll
-            for (int e = 0; e < 8; ++e) m2 = fmaxf(m2, fabsf(y[e]));
+            for (int e = 0; e < 4; ++e) m2 = fmaxf(fmaxf(m2, fabsf(y[e].x)), fabsf(y[e].y));
           });
           m2 = bmax(m2);
           sync();  // everyone has read red[..][2] above
@@ -404,21 +477,31 @@ __global__ void __launch_bounds__(kThreads, 1) rowpipe_kernel(const Pipe P) {
         if (j == 0) a.scale[row] = delta;
         int8_t* qr = a.q + row * K;
         if (clean) {
-          for_chunks([&](int, int64_t c, const float (&x)[8]) {
-            float y[8];
+          // |y * inv| <= 127*(1 + 2^-23) < 127.5 for every element of a
+          // finite row: round (1.5 * 2^23 addition) without clamping
+          const float2 inv2 = make_float2(inv, inv);
+          for_chunks([&](int, int c, const float2 (&x)[4]) {
+            float2 y[4];
             ychunk(c, x, y);
             uint32_t b[8];
 #pragma unroll
-            for (int e = 0; e < 8; ++e) b[e] = qbits_fast(y[e], inv);
+            for (int e = 0; e < 4; ++e) {
+              const float2 r = mul2(y[e], inv2);
+              b[2 * e] = __float_as_uint(__fadd_rn(r.x, kRoundMagic));
+              b[2 * e + 1] = __float_as_uint(__fadd_rn(r.y, kRoundMagic));
+            }
             store_codes(qr + c * 8, b);
           });
         } else {
-          for_chunks([&](int, int64_t c, const float (&x)[8]) {
-            float y[8];
+          for_chunks([&](int, int c, const float2 (&x)[4]) {
+            float2 y[4];
             ychunk(c, x, y);
             uint32_t b[8];
 #pragma unroll
-            for (int e = 0; e < 8; ++e) b[e] = qbits(y[e], inv, count, clipped);
+            for (int e = 0; e < 4; ++e) {
+              b[2 * e] = qbits(y[e].x, inv, count, clipped);
+              b[2 * e + 1] = qbits(y[e].y, inv, count, clipped);
+            }
             store_codes(qr + c * 8, b);
           });
         }
@@ -430,8 +513,8 @@ __global__ void __launch_bounds__(kThreads, 1) rowpipe_kernel(const Pipe P) {
     if constexpr (MODE == ROW_COLMAX && CM > 0) {
 #pragma unroll
       for (int m = 0; m < CM; ++m) {
-        const int64_t c = chunk_of(m);
-        if (c < nchunk) {
+        const int c = chunk_of(m);
+        if (c < nch && R > 0) {
 #pragma unroll
           for (int e = 0; e < 8; ++e)
             atomicMax(&colmax_s[c * 8 + e], __float_as_uint(cmax[m * 8 + e]));
@@ -539,7 +622,7 @@ cudaError_t dispatch_mode(const Pipe& P, RowMode mode, int w, size_t smem, int g
       return ln ? dispatch_quant<T, true, ROW_STATIC>(P, w, smem, grid, st)
                 : dispatch_quant<T, false, ROW_STATIC>(P, w, smem, grid, st);
     case ROW_COLMAX:
-      return dispatch_colmax<T>(P, smem, grid, st);
+      return ln ? dispatch_colmax<T>(P, smem, grid, st) : cudaErrorInvalidValue;
   }
   return cudaErrorInvalidValue;
 }
@@ -552,6 +635,7 @@ bool plan(int64_t K, sq_dtype xt, RowMode mode, bool ln, int* slots, int* w, siz
   if (fixed + 2 * rb > kSmemBudget) return false;
   int s = (int)((kSmemBudget - fixed) / rb);
   if (s > kMaxSlots) s = kMaxSlots;
+  if (mode == ROW_COLMAX && !ln) return false;  // raw peaks: column strips (rowops.cu)
   int ww;
   if (mode == ROW_COLMAX) ww = 4;
   else if (s >= 8) ww = 2;
