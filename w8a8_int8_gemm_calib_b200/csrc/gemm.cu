@@ -23,6 +23,7 @@
 #include <stdint.h>
 
 #include <mutex>
+#include <string.h>
 
 #include "sq_device.cuh"
 #include "sq_internal.h"
@@ -45,11 +46,16 @@ constexpr uint32_t TMEM_COLS = 2 * BN;
 constexpr int GROUP_M = 16;  // tile raster: 16 row blocks share each column sweep
 constexpr uint64_t kWaitNs = 4000000000ull;   // 4 s: far above any pipeline step
 constexpr uint64_t kDrainNs = 1000000000ull;  // waits for copies already in flight
-constexpr size_t SMEM_BYTES = 1024 + (size_t)STAGES * STAGE_BYTES + 256;
+// Output staging for the TMA-store epilogue: per epilogue warp, two buffers
+// of 32 rows x 64 bytes (32 bf16 or 16 fp32 columns), 64-byte swizzled.
+constexpr int EPI_BUF = 32 * 64;
+constexpr int EPI_BYTES = 4 * 2 * EPI_BUF;
+constexpr size_t SMEM_BYTES = 1024 + (size_t)STAGES * STAGE_BYTES + EPI_BYTES + 256;
 
 struct Params {
   int M, N, K;
   int m_tiles, n_tiles, num_tiles, nk;
+  int tma_store;  // outputs leave through shared memory and TMA stores
   const float* act_scale;
   int per_token;
   const float* w_scale;
@@ -138,12 +144,13 @@ __device__ __forceinline__ void store_chunk(const Params& p, int row, int col0,
 template <bool BF16>
 __global__ void __launch_bounds__(THREADS, 1)
 gemm_w8a8_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                    const Params p) {
+                    const __grid_constant__ CUtensorMap tmY, const Params p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
   uint8_t* sA = smem;
   uint8_t* sB = smem + STAGES * A_BYTES;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + STAGES * STAGE_BYTES);
+  uint8_t* sEpi = smem + STAGES * STAGE_BYTES;  // 1024-aligned
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sEpi + EPI_BYTES);
   // bars: full[STAGES], empty[STAGES], tfull[2], tempty[2], drain
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * STAGES + 5);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
@@ -251,13 +258,16 @@ gemm_w8a8_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
   } else {
     // ------------------------------------------------------------ epilogue
     const int quarter = warp & 3;  // this warp may read TMEM lanes 32*quarter..+31
+    uint8_t* ebuf = sEpi + (warp - 2) * 2 * EPI_BUF;
+    uint32_t nstore = 0;  // TMA stores issued by this warp (selects the buffer)
     uint32_t abuf = 0, aphase = 0;
     for (int tile = blockIdx.x; tile < p.num_tiles; tile += gridDim.x) {
       int mb, nb;
       tile_coords(tile, p.m_tiles, p.n_tiles, mb, nb);
       if (!tc::mbar_wait(tfull_bar(abuf), aphase, abort_flag, kWaitNs, p.status)) break;
       tc::tc_fence_after();
-      const int row = mb * BM + quarter * 32 + lane;
+      const int row0 = mb * BM + quarter * 32;
+      const int row = row0 + lane;
       const bool row_ok = row < p.M;
       const float as = p.per_token ? (row_ok ? __ldg(p.act_scale + row) : 0.0f) : __ldg(p.act_scale);
       const uint32_t taddr = tmem_base + abuf * BN + ((uint32_t)(quarter * 32) << 16);
@@ -267,7 +277,67 @@ gemm_w8a8_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
         tc::tmem_ld32(taddr + c * 32, r);
         tc::tmem_ld_wait();
         const int col0 = nb * BN + c * 32;
-        if (row_ok && col0 < p.N) store_chunk<BF16>(p, row, col0, r, as);
+        if (!p.tma_store) {
+          if (row_ok && col0 < p.N) store_chunk<BF16>(p, row, col0, r, as);
+          continue;
+        }
+        // dequantize this lane's 32 outputs (row `row`, columns col0..+31)
+        float ws[32];
+        if (col0 + 32 <= p.N) {
+          const float4* w4 = reinterpret_cast<const float4*>(p.w_scale + col0);
+#pragma unroll
+          for (int i = 0; i < 8; ++i) {
+            const float4 v = __ldg(w4 + i);
+            ws[4 * i] = v.x; ws[4 * i + 1] = v.y; ws[4 * i + 2] = v.z; ws[4 * i + 3] = v.w;
+          }
+        } else {
+#pragma unroll
+          for (int i = 0; i < 32; ++i) ws[i] = col0 + i < p.N ? __ldg(p.w_scale + col0 + i) : 0.0f;
+        }
+        uint32_t wv[BF16 ? 16 : 32];
+#pragma unroll
+        for (int i = 0; i < 32; i += 2) {
+          const float y0 = __fmul_rn(__int2float_rn((int)r[i]), __fmul_rn(as, ws[i]));
+          const float y1 = __fmul_rn(__int2float_rn((int)r[i + 1]), __fmul_rn(as, ws[i + 1]));
+          if (BF16) {
+            __nv_bfloat162 t = __floats2bfloat162_rn(y0, y1);
+            wv[i / 2] = *reinterpret_cast<uint32_t*>(&t);
+          } else {
+            wv[i] = __float_as_uint(y0);
+            wv[i + 1] = __float_as_uint(y1);
+          }
+        }
+        if (p.acc && row_ok && col0 < p.N) {
+          int32_t* a = p.acc + (size_t)row * p.N + col0;
+#pragma unroll
+          for (int i = 0; i < 32; ++i)
+            if (col0 + i < p.N) a[i] = (int)r[i];
+        }
+        // 64-byte rows: one box for bf16 (32 columns), two for fp32 (16 each)
+        const bool any = row0 < p.M && col0 < p.N;  // warp-uniform
+#pragma unroll
+        for (int h = 0; h < (BF16 ? 1 : 2); ++h) {
+          uint8_t* buf = ebuf + (nstore & 1) * EPI_BUF;
+          if (lane == 0) tc::bulk_wait_read<1>();  // the store that last read `buf` is done
+          __syncwarp();
+          // row `lane`, 16-byte chunk k at chunk k ^ ((lane >> 1) & 3): the
+          // 64-byte swizzle the tensor map undoes (conflict-free writes)
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            const int pk = k ^ ((lane >> 1) & 3);
+            *reinterpret_cast<uint4*>(buf + lane * 64 + pk * 16) =
+                make_uint4(wv[h * 16 + 4 * k], wv[h * 16 + 4 * k + 1], wv[h * 16 + 4 * k + 2],
+                           wv[h * 16 + 4 * k + 3]);
+          }
+          tc::fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) {
+            const int cx = col0 + h * 16;
+            if (any && cx < p.N) tc::tma_store_2d(&tmY, tc::smem_u32(buf), cx, row0);
+            tc::bulk_commit();
+          }
+          ++nstore;
+        }
       }
       tc::tc_fence_before();
       __syncwarp();
@@ -275,6 +345,8 @@ gemm_w8a8_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
       abuf ^= 1u;
       if (abuf == 0) aphase ^= 1u;
     }
+    if (lane == 0) tc::bulk_wait_all();  // staged outputs written before the CTA exits
+    __syncwarp();
   }
 
   tc::tc_fence_before();
@@ -605,9 +677,26 @@ bool make_tmap(CUtensorMap* m, const void* base, uint64_t inner, uint64_t rows, 
   return r == CUDA_SUCCESS;
 }
 
+// Output tensor map for the TMA-store epilogue: [rows, cols] of bf16/fp32,
+// box 64 bytes x 32 rows, 64-byte swizzle.
+bool make_tmap_out(CUtensorMap* m, void* base, uint64_t cols, uint64_t rows, bool bf16) {
+  auto enc = encode_fn();
+  if (!enc) return false;
+  const uint64_t esz = bf16 ? 2 : 4;
+  cuuint64_t dims[2] = {cols, rows};
+  cuuint64_t strides[1] = {cols * esz};
+  cuuint32_t box[2] = {(cuuint32_t)(64 / esz), 32};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = enc(m, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2,
+                   base, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                   CU_TENSOR_MAP_SWIZZLE_64B, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
 template <bool BF16>
-cudaError_t launch_tc(const CUtensorMap& ta, const CUtensorMap& tb, const Params& p, int grid,
-                      cudaStream_t st) {
+cudaError_t launch_tc(const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& ty,
+                      const Params& p, int grid, cudaStream_t st) {
   static std::once_flag once[64];
   static cudaError_t attr_err[64];
   int dev = 0;
@@ -619,7 +708,7 @@ cudaError_t launch_tc(const CUtensorMap& ta, const CUtensorMap& tb, const Params
                                          (int)SMEM_BYTES);
   });
   if (attr_err[dev] != cudaSuccess) return attr_err[dev];
-  gemm_w8a8_tc_kernel<BF16><<<grid, THREADS, SMEM_BYTES, st>>>(ta, tb, p);
+  gemm_w8a8_tc_kernel<BF16><<<grid, THREADS, SMEM_BYTES, st>>>(ta, tb, ty, p);
   return cudaGetLastError();
 }
 
@@ -767,10 +856,16 @@ sq_status launch_gemm(const GemmArgs& a, cudaStream_t st) {
   p.y = a.y;
   p.acc = a.acc_out;
   p.status = sw;
+  // TMA stores need 16-byte row pitches; other widths store directly
+  CUtensorMap ty;
+  memset(&ty, 0, sizeof ty);
+  const bool bf16 = a.yt == SQ_BF16;
+  p.tma_store = (a.N % (bf16 ? 8 : 4)) == 0 &&
+                make_tmap_out(&ty, a.y, (uint64_t)a.N, (uint64_t)a.M, bf16);
   int grid = sm_count();
   if (grid > p.num_tiles) grid = p.num_tiles;
-  cudaError_t e = a.yt == SQ_BF16 ? launch_tc<true>(ta, tb, p, grid, st)
-                                  : launch_tc<false>(ta, tb, p, grid, st);
+  cudaError_t e = bf16 ? launch_tc<true>(ta, tb, ty, p, grid, st)
+                       : launch_tc<false>(ta, tb, ty, p, grid, st);
   if (e != cudaSuccess) return fail(SQ_ERR_CUDA, "sq_gemm_w8a8: %s", cudaGetErrorString(e));
   return SQ_OK;
 }
