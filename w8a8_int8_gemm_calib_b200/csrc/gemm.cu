@@ -52,6 +52,18 @@ constexpr int EPI_BUF = 32 * 64;
 constexpr int EPI_BYTES = 4 * 2 * EPI_BUF;
 constexpr size_t SMEM_BYTES = 1024 + (size_t)STAGES * STAGE_BYTES + EPI_BYTES + 256;
 
+// Large-M tile shapes: 128 x TBN outputs per tile, TBN in {256, 192}; the
+// host picks the one that fills the last wave of SMs best.
+template <int TBN>
+struct TcCfg {
+  static constexpr int B_BYTES = TBN * BK;
+  static constexpr int STAGE = A_BYTES + B_BYTES;
+  static constexpr int STAGES = TBN == 256 ? 4 : 5;
+  static constexpr uint32_t TMEM_COLS = 2 * TBN <= 256 ? 256 : 512;  // power of two
+  static constexpr size_t SMEM = 1024 + (size_t)STAGES * STAGE + EPI_BYTES + 256;
+  static_assert(SMEM <= 227 * 1024, "shared memory");
+};
+
 struct Params {
   int M, N, K;
   int m_tiles, n_tiles, num_tiles, nk;
@@ -141,10 +153,16 @@ __device__ __forceinline__ void store_chunk(const Params& p, int row, int col0,
   }
 }
 
-template <bool BF16>
+template <bool BF16, int TBN>
 __global__ void __launch_bounds__(THREADS, 1)
 gemm_w8a8_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                     const __grid_constant__ CUtensorMap tmY, const Params p) {
+  using C = TcCfg<TBN>;
+  constexpr int STAGES = C::STAGES;
+  constexpr int B_BYTES = C::B_BYTES;
+  constexpr int STAGE_BYTES = C::STAGE;
+  constexpr uint32_t TMEM_COLS = C::TMEM_COLS;
+  constexpr int BN = TBN;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
   uint8_t* sA = smem;
@@ -694,7 +712,7 @@ bool make_tmap_out(CUtensorMap* m, void* base, uint64_t cols, uint64_t rows, boo
   return r == CUDA_SUCCESS;
 }
 
-template <bool BF16>
+template <bool BF16, int TBN>
 cudaError_t launch_tc(const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& ty,
                       const Params& p, int grid, cudaStream_t st) {
   static std::once_flag once[64];
@@ -703,13 +721,29 @@ cudaError_t launch_tc(const CUtensorMap& ta, const CUtensorMap& tb, const CUtens
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess || dev < 0 || dev >= 64) return e != cudaSuccess ? e : cudaErrorInvalidDevice;
   std::call_once(once[dev], [&] {
-    attr_err[dev] = cudaFuncSetAttribute(gemm_w8a8_tc_kernel<BF16>,
+    attr_err[dev] = cudaFuncSetAttribute(gemm_w8a8_tc_kernel<BF16, TBN>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)SMEM_BYTES);
+                                         (int)TcCfg<TBN>::SMEM);
   });
   if (attr_err[dev] != cudaSuccess) return attr_err[dev];
-  gemm_w8a8_tc_kernel<BF16><<<grid, THREADS, SMEM_BYTES, st>>>(ta, tb, ty, p);
+  gemm_w8a8_tc_kernel<BF16, TBN><<<grid, THREADS, TcCfg<TBN>::SMEM, st>>>(ta, tb, ty, p);
   return cudaGetLastError();
+}
+
+// Tile width for the large-M kernel: the per-tile time grows with the width,
+// and a partly filled last wave costs a whole tile time, so take the width
+// with the smaller (waves x width) -- plus a fixed per-tile cost.
+int pick_tile_n(int64_t M, int64_t N, int sms) {
+  const int64_t mt = (M + BM - 1) / BM;
+  int best = 256;
+  int64_t best_cost = -1;
+  for (int tbn : {256, 192}) {
+    const int64_t tiles = mt * ((N + tbn - 1) / tbn);
+    const int64_t waves = (tiles + sms - 1) / sms;
+    const int64_t cost = waves * (tbn + 16);
+    if (best_cost < 0 || cost < best_cost) { best = tbn; best_cost = cost; }
+  }
+  return best;
 }
 
 
@@ -840,14 +874,15 @@ sq_status launch_gemm(const GemmArgs& a, cudaStream_t st) {
     if (e != cudaSuccess) return fail(SQ_ERR_CUDA, "sq_gemm_w8a8: %s", cudaGetErrorString(e));
     return SQ_OK;
   }
+  const int tbn = pick_tile_n(a.M, a.N, sm_count());
   CUtensorMap ta, tb;
   if (!make_tmap(&ta, a.xq, (uint64_t)a.K, (uint64_t)a.M, BM) ||
-      !make_tmap(&tb, a.wq, (uint64_t)a.K, (uint64_t)a.N, BN))
+      !make_tmap(&tb, a.wq, (uint64_t)a.K, (uint64_t)a.N, (uint32_t)tbn))
     return fail(SQ_ERR_CUDA, "sq_gemm_w8a8: cuTensorMapEncodeTiled failed");
   Params p{};
   p.M = (int)a.M; p.N = (int)a.N; p.K = (int)a.K;
   p.m_tiles = (int)((a.M + BM - 1) / BM);
-  p.n_tiles = (int)((a.N + BN - 1) / BN);
+  p.n_tiles = (int)((a.N + tbn - 1) / tbn);
   p.num_tiles = p.m_tiles * p.n_tiles;
   p.nk = (int)((a.K + BK - 1) / BK);
   p.act_scale = a.act_scale;
@@ -864,8 +899,10 @@ sq_status launch_gemm(const GemmArgs& a, cudaStream_t st) {
                 make_tmap_out(&ty, a.y, (uint64_t)a.N, (uint64_t)a.M, bf16);
   int grid = sm_count();
   if (grid > p.num_tiles) grid = p.num_tiles;
-  cudaError_t e = bf16 ? launch_tc<true>(ta, tb, ty, p, grid, st)
-                       : launch_tc<false>(ta, tb, ty, p, grid, st);
+  cudaError_t e = tbn == 256 ? (bf16 ? launch_tc<true, 256>(ta, tb, ty, p, grid, st)
+                                     : launch_tc<false, 256>(ta, tb, ty, p, grid, st))
+                              : (bf16 ? launch_tc<true, 192>(ta, tb, ty, p, grid, st)
+                                      : launch_tc<false, 192>(ta, tb, ty, p, grid, st));
   if (e != cudaSuccess) return fail(SQ_ERR_CUDA, "sq_gemm_w8a8: %s", cudaGetErrorString(e));
   return SQ_OK;
 }
