@@ -25,6 +25,7 @@
 #include <mutex>
 #include <string.h>
 
+#include "launch.cuh"
 #include "sq_device.cuh"
 #include "sq_internal.h"
 #include "tc_ptx.cuh"
@@ -173,6 +174,7 @@ gemm_w8a8_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * STAGES + 5);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
+  pdl_launch_dependents();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   auto full_bar = [&](int s) { return tc::smem_u32(bars + s); };
   auto empty_bar = [&](int s) { return tc::smem_u32(bars + STAGES + s); };
@@ -203,6 +205,7 @@ gemm_w8a8_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
   __syncthreads();
   tc::tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
+  pdl_wait();  // the prologue above touches no global memory
 
   if (warp == 0) {
     // ------------------------------------------------------------ TMA producer
@@ -481,6 +484,7 @@ gemm_w8a8_smallm_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_co
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   volatile int* last_flag = reinterpret_cast<volatile int*>(tmem_slot + 2);
 
+  pdl_launch_dependents();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   auto full_bar = [&](int s) { return tc::smem_u32(bars + s); };
   auto empty_bar = [&](int s) { return tc::smem_u32(bars + S + s); };
@@ -511,6 +515,7 @@ gemm_w8a8_smallm_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_co
   __syncthreads();
   tc::tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
+  pdl_wait();  // the prologue above touches no global memory
   const int64_t ub = unit_begin(blockIdx.x, p), ue = unit_begin(blockIdx.x + 1, p);
 
   if (warp == 0) {
@@ -726,8 +731,8 @@ cudaError_t launch_tc(const CUtensorMap& ta, const CUtensorMap& tb, const CUtens
                                          (int)TcCfg<TBN>::SMEM);
   });
   if (attr_err[dev] != cudaSuccess) return attr_err[dev];
-  gemm_w8a8_tc_kernel<BF16, TBN><<<grid, THREADS, TcCfg<TBN>::SMEM, st>>>(ta, tb, ty, p);
-  return cudaGetLastError();
+  return launch_pdl(gemm_w8a8_tc_kernel<BF16, TBN>, dim3(grid), dim3(THREADS), TcCfg<TBN>::SMEM, st,
+                    ta, tb, ty, p);
 }
 
 // Tile width for the large-M kernel: the per-tile time grows with the width,
@@ -782,8 +787,8 @@ cudaError_t launch_small_t(const CUtensorMap& tw, const CUtensorMap& tx, const S
                                          (int)SmallCfg<NPAD>::SMEM);
   });
   if (attr_err[dev] != cudaSuccess) return attr_err[dev];
-  gemm_w8a8_smallm_kernel<NPAD, BF16><<<p.grid, THREADS, SmallCfg<NPAD>::SMEM, st>>>(tw, tx, p);
-  return cudaGetLastError();
+  return launch_pdl(gemm_w8a8_smallm_kernel<NPAD, BF16>, dim3(p.grid), dim3(THREADS),
+                    SmallCfg<NPAD>::SMEM, st, tw, tx, p);
 }
 
 template <bool BF16>

@@ -1,0 +1,29 @@
+// launch.cuh -- kernel launch with programmatic stream serialization (see
+// pdl_wait / pdl_launch_dependents in sq_device.cuh): the kernel may begin
+// launching before the previous kernel of the stream has finished; it
+// orders itself after that kernel with pdl_wait() on the device.  Inside
+// a captured CUDA graph the attribute becomes a programmatic dependency
+// edge between the two kernel nodes.
+#pragma once
+
+#include <cuda_runtime.h>
+
+namespace sq {
+
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                       cudaStream_t st, Args... args) {
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, args...);
+}
+
+}  // namespace sq

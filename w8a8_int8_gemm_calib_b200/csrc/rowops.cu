@@ -19,6 +19,7 @@
 
 #include <mutex>
 
+#include "launch.cuh"
 #include "sq_device.cuh"
 #include "sq_internal.h"
 
@@ -38,6 +39,8 @@ __global__ void __launch_bounds__(kColWarps * 32)
 colmax_kernel(const T* __restrict__ x, int64_t T_, int64_t K, int64_t rows_per_slab,
               unsigned int* __restrict__ out) {
   __shared__ float part[kColWarps][256];
+  pdl_launch_dependents();
+  pdl_wait();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int64_t nchunk = K >> 3;
   const int64_t chunk = (int64_t)blockIdx.x * 32 + lane;
@@ -116,12 +119,10 @@ cudaError_t launch_colmax(const void* x, sq_dtype xt, int64_t T, int64_t K, floa
   slabs = (T + rows - 1) / rows;
   dim3 grid((unsigned)strips, (unsigned)slabs);
   if (xt == SQ_BF16)
-    colmax_kernel<uint16_t><<<grid, kColWarps * 32, 0, st>>>(
-        (const uint16_t*)x, T, K, rows, (unsigned int*)out);
-  else
-    colmax_kernel<float><<<grid, kColWarps * 32, 0, st>>>(
-        (const float*)x, T, K, rows, (unsigned int*)out);
-  return cudaGetLastError();
+    return launch_pdl(colmax_kernel<uint16_t>, grid, dim3(kColWarps * 32), 0, st,
+                      (const uint16_t*)x, T, K, rows, (unsigned int*)out);
+  return launch_pdl(colmax_kernel<float>, grid, dim3(kColWarps * 32), 0, st, (const float*)x, T,
+                    K, rows, (unsigned int*)out);
 }
 
 // ============================================================ row kernel
@@ -205,6 +206,8 @@ row_kernel(RowArgs a) {
   // [slice][parity][reduction][warp]
   __shared__ float red[kSlices][2][3][4];
   extern __shared__ unsigned int colmax_s[];  // ROW_COLMAX: per-CTA column peaks [K]
+  pdl_launch_dependents();
+  pdl_wait();
 
   uint32_t dyn_smem;
   asm("mov.u32 %0, %%dynamic_smem_size;" : "=r"(dyn_smem));
@@ -448,8 +451,7 @@ static cudaError_t launch_row_t(const RowArgs& a, cudaStream_t st) {
   int64_t cap = (int64_t)sm_count() * per_sm;
   int64_t grid = want < cap ? want : cap;
   if (grid < 1) grid = 1;
-  kern<<<(unsigned)grid, kSlices * kSliceThreads, smem, st>>>(a);
-  return cudaGetLastError();
+  return launch_pdl(kern, dim3((unsigned)grid), dim3(kSlices * kSliceThreads), smem, st, a);
 }
 
 // Rows too wide for the shared-memory pipeline (rowpipe.cu) take the
@@ -500,6 +502,8 @@ __global__ void __launch_bounds__(kScaleThreads)
 scales_kernel(const float* __restrict__ amax_x, int64_t K, float alpha,
               float* s, float* __restrict__ inv_s, unsigned int* __restrict__ delta_out) {
   __shared__ float wmax[kScaleThreads / 32];
+  pdl_launch_dependents();
+  pdl_wait();
   float lmax = 0.0f;
   const double al = (double)alpha;
   for (int64_t k = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; k < K;
@@ -543,9 +547,8 @@ cudaError_t launch_scales(const float* amax_x, int64_t K, float alpha, float* s,
   }
   int64_t blocks = (K + kScaleThreads - 1) / kScaleThreads;
   if (blocks > 4 * (int64_t)sm_count()) blocks = 4 * (int64_t)sm_count();
-  scales_kernel<<<(unsigned)blocks, kScaleThreads, 0, st>>>(amax_x, K, alpha, s, inv_s,
-                                                           (unsigned int*)delta_out);
-  return cudaGetLastError();
+  return launch_pdl(scales_kernel, dim3((unsigned)blocks), dim3(kScaleThreads), 0, st, amax_x, K,
+                    alpha, s, inv_s, (unsigned int*)delta_out);
 }
 
 // ============================================================ LayerNorm fold
@@ -553,6 +556,8 @@ cudaError_t launch_scales(const float* amax_x, int64_t K, float alpha, float* s,
 __global__ void fold_ln_kernel(const float* __restrict__ gamma, const float* __restrict__ beta,
                                const float* __restrict__ s, int64_t K,
                                float* __restrict__ gamma_out, float* __restrict__ beta_out) {
+  pdl_launch_dependents();
+  pdl_wait();
   for (int64_t k = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; k < K;
        k += (int64_t)gridDim.x * blockDim.x) {
     const float sk = s[k];
@@ -565,8 +570,8 @@ cudaError_t launch_fold_ln(const float* gamma, const float* beta, const float* s
                            float* gamma_out, float* beta_out, cudaStream_t st) {
   int64_t blocks = (K + 255) / 256;
   if (blocks > 1024) blocks = 1024;
-  fold_ln_kernel<<<(unsigned)blocks, 256, 0, st>>>(gamma, beta, s, K, gamma_out, beta_out);
-  return cudaGetLastError();
+  return launch_pdl(fold_ln_kernel, dim3((unsigned)blocks), dim3(256), 0, st, gamma, beta, s, K,
+                    gamma_out, beta_out);
 }
 
 }  // namespace sq

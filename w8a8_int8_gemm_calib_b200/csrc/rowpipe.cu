@@ -12,13 +12,14 @@
 //              quantizer; W * diag(s) with static per-channel INT8)
 //
 // Design.  One CTA per SM: a producer warp streams whole rows (contiguous
-// K-element runs) from HBM into a ring of shared-memory row slots with 1-D
-// bulk copies completing on mbarriers, up to 16 rows ahead; four 128-thread
-// slices consume the rows.  Slot j = 32*w + l of a slice owns the 8-element
-// chunks c = j, j+128, ... of the row, which fixes the LayerNorm reduction
-// order (see rowops.cu; both files implement the same order).  Per-column
-// parameters (gamma, beta, or the column multiplier) are staged in shared
-// memory once per CTA.  Every mbarrier wait is bounded.
+// K-element runs) from HBM into a ring of up to 24 shared-memory row slots
+// with 1-D bulk copies completing on mbarriers; slices of W warps consume the
+// rows.  A thread loads its part of a row into registers as fp32 at once and
+// hands the slot back, then works on the registers in place (x, x - mu, y).
+// The slice emulates the 128 canonical LayerNorm slots, which fixes the
+// reduction order (see rowops.cu; both files implement the same order).
+// Per-column parameters (gamma, beta, or the column multiplier) are staged in
+// shared memory once per CTA.  Every mbarrier wait is bounded.
 //
 // Rounding: r = y * (1/Delta) is clamped to [-127, 127] (NaN -> 0) and
 // 1.5 * 2^23 is added: the fp32 addition rounds r to the nearest integer, ties
@@ -30,6 +31,7 @@
 
 #include <mutex>
 
+#include "launch.cuh"
 #include "sq_device.cuh"
 #include "sq_internal.h"
 #include "tc_ptx.cuh"
@@ -40,12 +42,13 @@ namespace {
 
 constexpr int kConsumers = 512;        // consumer threads per CTA
 constexpr int kThreads = kConsumers + 32;
-constexpr int kMaxSlots = 16;
-constexpr size_t kSmemBudget = 200 * 1024;
+constexpr int kMaxSlots = 24;
+constexpr size_t kSmemBudget = 226 * 1024;  // + static shared memory stays under the 227 KB per-block limit
 constexpr uint32_t kCopyPiece = 32768;
 constexpr uint64_t kWaitNs = 2000000000ull;
 constexpr uint64_t kDrainNs = 1000000000ull;
 constexpr float kRoundMagic = 12582912.0f;  // 1.5 * 2^23
+constexpr int kSrcSmem = 0, kSrcRaw = 1, kSrcF32 = 2;
 
 struct Pipe {
   RowArgs a;
@@ -209,8 +212,13 @@ __global__ void __launch_bounds__(kThreads, 1) rowpipe_kernel(const Pipe P) {
   constexpr int ST = 32 * W;            // threads per slice
   constexpr int NS = kConsumers / ST;   // slices per CTA
   constexpr int G = W <= 4 ? 4 / W : 1;  // slot groups per thread (LayerNorm modes: W <= 4)
-  static_assert(!LN || W == 2 || W == 4, "the LayerNorm order needs 2- or 4-warp slices");
+  static_assert(!LN || W == 1 || W == 2 || W == 4, "the LayerNorm order needs 1-, 2- or 4-warp slices");
   static_assert(MODE != ROW_COLMAX || LN, "raw column peaks use the column-strip kernel");
+  // where the row is kept while a slice works on it: fp32 registers (at most
+  // 64 per thread, with the column peaks when those are kept too), the
+  // storage form in registers, or the shared-memory slot itself
+  constexpr int SRC = CM == 0 ? kSrcSmem
+                      : CM * 8 * (MODE == ROW_COLMAX ? 2 : 1) <= 64 ? kSrcF32 : kSrcRaw;
   extern __shared__ __align__(128) uint8_t smem[];
   __shared__ float red[NS][2][3][W];
   __shared__ int abort_s;
@@ -229,17 +237,19 @@ __global__ void __launch_bounds__(kThreads, 1) rowpipe_kernel(const Pipe P) {
   auto empty_bar = [&](int s) { return tc::smem_u32(bars + kMaxSlots + s); };
 
   const int tid = threadIdx.x;
+  pdl_launch_dependents();
   const bool has_mul = !LN && a.mul != nullptr;
   const int khalf = (int)(K >> 1);
   if (tid == 0) {
     for (int s = 0; s < S; ++s) {
       tc::mbar_init(full_bar(s), 1);
-      tc::mbar_init(empty_bar(s), 1);
+      tc::mbar_init(empty_bar(s), W);  // one arrival per consumer warp of the slice
     }
     abort_s = 0;
     tc::mbar_fence_init();
   }
   __syncthreads();
+  pdl_wait();
   volatile int* abort_flag = &abort_s;
 
   const int64_t r0 = (int64_t)blockIdx.x * P.rows_per_cta;
@@ -281,15 +291,41 @@ __global__ void __launch_bounds__(kThreads, 1) rowpipe_kernel(const Pipe P) {
     }
   } else {
     // ------------------------------------------------------------ consumers
-    for (int k = tid; k < (int)K; k += kConsumers) {
-      const int pk = param_index(k, khalf);
-      if (LN) {
-        pg[pk] = a.g[k];
-        pb[pk] = a.b ? a.b[k] : 0.0f;
-      } else if (has_mul) {
-        pg[pk] = a.mul[k];
+    // per-column parameters into the split layout, with the global loads
+    // batched so that several are in flight per thread
+    {
+      constexpr int U = 8;
+      for (int k0 = tid; k0 < (int)K; k0 += U * kConsumers) {
+        float gv[U], bv[U];
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+          const int k = k0 + u * kConsumers;
+          gv[u] = 0.0f;
+          bv[u] = 0.0f;
+          if (k < (int)K) {
+            if (LN) {
+              gv[u] = __ldg(a.g + k);
+              if (a.b) bv[u] = __ldg(a.b + k);
+            } else if (has_mul) {
+              gv[u] = __ldg(a.mul + k);
+            }
+          }
+        }
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+          const int k = k0 + u * kConsumers;
+          if (k < (int)K) {
+            const int pk = param_index(k, khalf);
+            if (LN) {
+              pg[pk] = gv[u];
+              pb[pk] = bv[u];
+            } else if (has_mul) {
+              pg[pk] = gv[u];
+            }
+            if (MODE == ROW_COLMAX) colmax_s[k] = 0u;
+          }
+        }
       }
-      if (MODE == ROW_COLMAX) colmax_s[k] = 0u;
     }
     asm volatile("bar.sync 9, %0;" ::"r"(kConsumers) : "memory");  // consumers only
 
@@ -305,31 +341,95 @@ __global__ void __launch_bounds__(kThreads, 1) rowpipe_kernel(const Pipe P) {
     int parity = 0;
     const int nch = (int)nchunk;  // < 2^14 here: rows fit in shared memory
     auto chunk_of = [&](int i) -> int { return 32 * v + lane + ST * i; };
-    auto sync = [&]() { slice_sync_t<ST>(q); };
+    auto sync = [&]() {
+      if constexpr (W == 1) __syncwarp();
+      else slice_sync_t<ST>(q);
+    };
 
     for (int64_t i = q; i < R; i += NS) {
       const int s = (int)(i % S);
       const int64_t u = i / S;
       const bool ok = tc::mbar_wait(full_bar(s), (uint32_t)(u & 1), abort_flag, kWaitNs, P.status);
-      if (!slice_and_t<ST>(q, ok)) break;
+      if constexpr (W == 1) {
+        if (!__all_sync(0xffffffffu, ok)) break;
+      } else {
+        if (!slice_and_t<ST>(q, ok)) break;
+      }
       const uint8_t* rowp = ring + (size_t)s * RB;
       const int64_t row = r0 + i;
 
-      RawC<T> xr[CM > 0 ? CM : 1];
-      if constexpr (CM > 0) {
+      // The thread's part of the row in registers: as fp32 pairs (updated in
+      // place by the passes below: x, then x - mu, then y) or in storage form.
+      float2 xf[SRC == kSrcF32 ? CM : 1][4];
+      RawC<T> xr[SRC == kSrcRaw ? CM : 1];
+      if constexpr (SRC != kSrcSmem) {
 #pragma unroll
-        for (int m = 0; m < CM; ++m)
-          if (chunk_of(m) < nch) lds_raw(rowp, chunk_of(m), xr[m]);
+        for (int m = 0; m < CM; ++m) {
+          const int c = chunk_of(m);
+          if (c < nch) {
+            if constexpr (SRC == kSrcF32) {
+              RawC<T> r;
+              lds_raw(rowp, c, r);
+              unpack8(r, xf[m]);
+            } else {
+              lds_raw(rowp, c, xr[m]);
+            }
+          }
+        }
+        // the row now lives in registers: each warp hands the slot back at
+        // once, so the producer refills it while this row is processed
+        __syncwarp();
+        if (lane == 0) tc::mbar_arrive(empty_bar(s));
       }
-      // f(m, c, x[4]) over the thread's chunks in increasing c
-      auto for_chunks = [&](auto&& f) {
-        if constexpr (CM > 0) {
+
+      float2 negmu2 = make_float2(0.0f, 0.0f), rstd2 = make_float2(0.0f, 0.0f);
+      // y of one chunk in place: ((x - mu) * rstd) * g + b from x - mu, or
+      // x * m, or x
+      auto ytrans = [&](int c, float2 (&x)[4]) {
+        if constexpr (LN) {
+          float2 g8[4], b8[4];
+          lds8(pg, c, khalf, g8);
+          lds8(pb, c, khalf, b8);
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const float2 t = mul2(mul2(x[e], rstd2), g8[e]);
+            x[e] = make_float2(__fadd_rn(t.x, b8[e].x), __fadd_rn(t.y, b8[e].y));
+          }
+        } else {
+          if (has_mul) {
+            float2 m8[4];
+            lds8(pg, c, khalf, m8);
+#pragma unroll
+            for (int e = 0; e < 4; ++e) x[e] = mul2(x[e], m8[e]);
+          }
+        }
+      };
+      // f(m, c, x[4]) over the thread's chunks in increasing c, with x at
+      // level `lvl` (0: x, 1: x - mu, 2: y).  The fp32 register copy is
+      // already at the level the previous pass left it at; the other sources
+      // recompute the level from the stored row.
+      auto for_level = [&](int lvl, auto&& f) {
+        auto lift = [&](int c, float2 (&x)[4]) {
+          if (LN && lvl >= 1) {
+#pragma unroll
+            for (int e = 0; e < 4; ++e) x[e] = add2(x[e], negmu2);
+          }
+          if (lvl >= 2) ytrans(c, x);
+        };
+        if constexpr (SRC == kSrcF32) {
+#pragma unroll
+          for (int m = 0; m < CM; ++m) {
+            const int c = chunk_of(m);
+            if (c < nch) f(m, c, xf[m]);
+          }
+        } else if constexpr (SRC == kSrcRaw) {
 #pragma unroll
           for (int m = 0; m < CM; ++m) {
             const int c = chunk_of(m);
             if (c < nch) {
               float2 x[4];
               unpack8(xr[m], x);
+              lift(c, x);
               f(m, c, x);
             }
           }
@@ -340,6 +440,7 @@ __global__ void __launch_bounds__(kThreads, 1) rowpipe_kernel(const Pipe P) {
             lds_raw(rowp, c, r);
             float2 x[4];
             unpack8(r, x);
+            lift(c, x);
             f(m, c, x);
           }
         }
@@ -349,6 +450,9 @@ __global__ void __launch_bounds__(kThreads, 1) rowpipe_kernel(const Pipe P) {
         float t[G];
 #pragma unroll
         for (int g = 0; g < G; ++g) t[g] = bsum(p[g]);
+        if constexpr (W == 1) {  // one lane holds all four slot groups
+          return __fadd_rn(__fadd_rn(t[0], t[2]), __fadd_rn(t[1], t[3]));
+        }
         float mine = t[0];
         if constexpr (G == 2) mine = __fadd_rn(t[0], t[1]);  // r_v + r_(v+2)
         if (lane == 0) red[q][parity][which][v] = mine;
@@ -358,12 +462,11 @@ __global__ void __launch_bounds__(kThreads, 1) rowpipe_kernel(const Pipe P) {
         else return __fadd_rn(r[0], r[1]);
       };
 
-      float2 negmu2 = make_float2(0.0f, 0.0f), rstd2 = make_float2(0.0f, 0.0f);
       if constexpr (LN) {
         float p[G];
 #pragma unroll
         for (int g = 0; g < G; ++g) p[g] = 0.0f;
-        for_chunks([&](int m, int, const float2 (&x)[4]) {
+        for_level(0, [&](int m, int, float2 (&x)[4]) {
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
             p[m % G] = __fadd_rn(p[m % G], x[e].x);
@@ -374,66 +477,42 @@ __global__ void __launch_bounds__(kThreads, 1) rowpipe_kernel(const Pipe P) {
         negmu2 = make_float2(-mu, -mu);
 #pragma unroll
         for (int g = 0; g < G; ++g) p[g] = 0.0f;
-        for_chunks([&](int m, int, const float2 (&x)[4]) {
+        for_level(0, [&](int m, int, float2 (&x)[4]) {
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
-            const float2 d = add2(x[e], negmu2);
-            p[m % G] = __fmaf_rn(d.x, d.x, p[m % G]);
-            p[m % G] = __fmaf_rn(d.y, d.y, p[m % G]);
+            x[e] = add2(x[e], negmu2);  // now x - mu
+            p[m % G] = __fmaf_rn(x[e].x, x[e].x, p[m % G]);
+            p[m % G] = __fmaf_rn(x[e].y, x[e].y, p[m % G]);
           }
         });
         const float rstd = __fdiv_rn(1.0f, __fsqrt_rn(__fadd_rn(__fdiv_rn(slot_sum(p, 1), kf), a.eps)));
         rstd2 = make_float2(rstd, rstd);
       }
-      // y of one chunk: ((x - mu) * rstd) * g + b, or x * m, or x
-      auto ychunk = [&](int c, const float2 (&x)[4], float2 (&y)[4]) {
-        if constexpr (LN) {
-          float2 g8[4], b8[4];
-          lds8(pg, c, khalf, g8);
-          lds8(pb, c, khalf, b8);
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const float2 t = mul2(mul2(add2(x[e], negmu2), rstd2), g8[e]);
-            y[e] = make_float2(__fadd_rn(t.x, b8[e].x), __fadd_rn(t.y, b8[e].y));
-          }
-        } else {
-          if (has_mul) {
-            float2 m8[4];
-            lds8(pg, c, khalf, m8);
-#pragma unroll
-            for (int e = 0; e < 4; ++e) y[e] = mul2(x[e], m8[e]);
-          } else {
-#pragma unroll
-            for (int e = 0; e < 4; ++e) y[e] = x[e];
-          }
-        }
-      };
+      constexpr int kLvlIn = LN ? 1 : 0;  // level the y pass starts from
 
       if constexpr (MODE == ROW_COLMAX) {
-        for_chunks([&](int m, int c, const float2 (&x)[4]) {
-          float2 y[4];
-          ychunk(c, x, y);
+        for_level(kLvlIn, [&](int m, int c, float2 (&x)[4]) {
+          ytrans(c, x);
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
             if constexpr (CM > 0) {
-              cmax[m * 8 + 2 * e] = fmaxf(cmax[m * 8 + 2 * e], fabsf(y[e].x));
-              cmax[m * 8 + 2 * e + 1] = fmaxf(cmax[m * 8 + 2 * e + 1], fabsf(y[e].y));
+              cmax[m * 8 + 2 * e] = fmaxf(cmax[m * 8 + 2 * e], fabsf(x[e].x));
+              cmax[m * 8 + 2 * e + 1] = fmaxf(cmax[m * 8 + 2 * e + 1], fabsf(x[e].y));
             } else {
-              atomicMax(&colmax_s[c * 8 + 2 * e], __float_as_uint(fabsf(y[e].x)));
-              atomicMax(&colmax_s[c * 8 + 2 * e + 1], __float_as_uint(fabsf(y[e].y)));
+              atomicMax(&colmax_s[c * 8 + 2 * e], __float_as_uint(fabsf(x[e].x)));
+              atomicMax(&colmax_s[c * 8 + 2 * e + 1], __float_as_uint(fabsf(x[e].y)));
             }
           }
         });
       } else if constexpr (MODE == ROW_STATIC) {
         int8_t* qr = a.q + row * K;
-        for_chunks([&](int, int c, const float2 (&x)[4]) {
-          float2 y[4];
-          ychunk(c, x, y);
+        for_level(kLvlIn, [&](int, int c, float2 (&x)[4]) {
+          ytrans(c, x);
           uint32_t b[8];
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
-            b[2 * e] = qbits(y[e].x, static_inv, count, clipped);
-            b[2 * e + 1] = qbits(y[e].y, static_inv, count, clipped);
+            b[2 * e] = qbits(x[e].x, static_inv, count, clipped);
+            b[2 * e + 1] = qbits(x[e].y, static_inv, count, clipped);
           }
           store_codes(qr + c * 8, b);
         });
@@ -441,35 +520,36 @@ __global__ void __launch_bounds__(kThreads, 1) rowpipe_kernel(const Pipe P) {
         // peak magnitude with NaN propagated: a finite result means every
         // element is finite (and then it equals the NaN-ignoring peak)
         float mn = 0.0f;
-        for_chunks([&](int, int c, const float2 (&x)[4]) {
-          float2 y[4];
-          ychunk(c, x, y);
+        for_level(kLvlIn, [&](int, int c, float2 (&x)[4]) {
+          ytrans(c, x);  // now y
 #pragma unroll
-          for (int e = 0; e < 4; ++e) mn = maxabs_nan(maxabs_nan(mn, y[e].x), y[e].y);
+          for (int e = 0; e < 4; ++e) mn = maxabs_nan(maxabs_nan(mn, x[e].x), x[e].y);
         });
 #pragma unroll
         for (int o = 16; o >= 1; o >>= 1) mn = maxabs_nan(mn, __shfl_xor_sync(0xffffffffu, mn, o));
-        if (lane == 0) red[q][parity][2][v] = mn;
-        sync();
+        if constexpr (W > 1) {
+          if (lane == 0) red[q][parity][2][v] = mn;
+          sync();
 #pragma unroll
-        for (int t = 0; t < W; ++t) mn = maxabs_nan(mn, red[q][parity][2][t]);
+          for (int t = 0; t < W; ++t) mn = maxabs_nan(mn, red[q][parity][2][t]);
+        }
         float mx = fabsf(mn);
         const bool clean = mx < INFINITY;  // false for inf and NaN
         if (!clean) {
           // non-finite elements: the peak over the non-NaN values (fmaxf)
           float m2 = 0.0f;
-          for_chunks([&](int, int c, const float2 (&x)[4]) {
-            float2 y[4];
-            ychunk(c, x, y);
+          for_level(2, [&](int, int, float2 (&y)[4]) {
 #pragma unroll
             for (int e = 0; e < 4; ++e) m2 = fmaxf(fmaxf(m2, fabsf(y[e].x)), fabsf(y[e].y));
           });
           m2 = bmax(m2);
-          sync();  // everyone has read red[..][2] above
-          if (lane == 0) red[q][parity][2][v] = m2;
-          sync();
+          if constexpr (W > 1) {
+            sync();  // everyone has read red[..][2] above
+            if (lane == 0) red[q][parity][2][v] = m2;
+            sync();
 #pragma unroll
-          for (int t = 0; t < W; ++t) m2 = fmaxf(m2, red[q][parity][2][t]);
+            for (int t = 0; t < W; ++t) m2 = fmaxf(m2, red[q][parity][2][t]);
+          }
           mx = m2;
         }
         const float delta = __fdiv_rn(fmaxf(mx, 1e-7f), 127.0f);
@@ -480,9 +560,7 @@ __global__ void __launch_bounds__(kThreads, 1) rowpipe_kernel(const Pipe P) {
           // |y * inv| <= 127*(1 + 2^-23) < 127.5 for every element of a
           // finite row: round (1.5 * 2^23 addition) without clamping
           const float2 inv2 = make_float2(inv, inv);
-          for_chunks([&](int, int c, const float2 (&x)[4]) {
-            float2 y[4];
-            ychunk(c, x, y);
+          for_level(2, [&](int, int c, float2 (&y)[4]) {
             uint32_t b[8];
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
@@ -493,9 +571,7 @@ __global__ void __launch_bounds__(kThreads, 1) rowpipe_kernel(const Pipe P) {
             store_codes(qr + c * 8, b);
           });
         } else {
-          for_chunks([&](int, int c, const float2 (&x)[4]) {
-            float2 y[4];
-            ychunk(c, x, y);
+          for_level(2, [&](int, int c, float2 (&y)[4]) {
             uint32_t b[8];
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
@@ -506,8 +582,10 @@ __global__ void __launch_bounds__(kThreads, 1) rowpipe_kernel(const Pipe P) {
           });
         }
       }
-      sync();  // every thread of the slice is done with the slot
-      if (j == 0) tc::mbar_arrive(empty_bar(s));
+      if constexpr (SRC == kSrcSmem) {
+        __syncwarp();  // this warp is done with the slot
+        if (lane == 0) tc::mbar_arrive(empty_bar(s));
+      }
       parity ^= 1;
     }
     if constexpr (MODE == ROW_COLMAX && CM > 0) {
@@ -559,16 +637,15 @@ cudaError_t launch_t(const Pipe& P, size_t smem, int grid, cudaStream_t st) {
                                          (int)kSmemBudget);
   });
   if (attr_err[dev] != cudaSuccess) return attr_err[dev];
-  kern<<<grid, kThreads, smem, st>>>(P);
-  return cudaGetLastError();
+  return launch_pdl(kern, dim3(grid), dim3(kThreads), smem, st, P);
 }
 
-// Quantizing modes.  Slice width W (warps) is chosen by the host from the
-// ring depth: 2 warps (8 slices, 8 rows in process per SM) when 8 or more
-// slots fit, else 4, else -- only without a LayerNorm, whose fixed reduction
-// order needs W <= 4 -- 8 or 16.  The row is held packed in registers when
-// it spans at most 16 chunks per thread (bf16: 64 registers) or 8 (fp32);
-// else each pass re-reads shared memory.
+// Quantizing modes.  The host picks the slice width W (warps): the narrowest
+// whose threads hold at most 8 chunks each -- the row then sits in fp32
+// registers, worked on in place -- while every slice has a slot (W = 1 gives
+// 16 slices and reductions by warp shuffles alone; a LayerNorm's fixed
+// reduction order allows W <= 4).  Up to 16 bf16 chunks per thread are held
+// in storage form instead; beyond that each pass re-reads shared memory.
 template <typename T, int W, bool LN, int MODE>
 cudaError_t dispatch_quant_w(const Pipe& P, size_t smem, int grid, cudaStream_t st) {
   constexpr bool kBf16 = sizeof(T) == 2;
@@ -584,6 +661,7 @@ cudaError_t dispatch_quant_w(const Pipe& P, size_t smem, int grid, cudaStream_t 
 
 template <typename T, bool LN, int MODE>
 cudaError_t dispatch_quant(const Pipe& P, int w, size_t smem, int grid, cudaStream_t st) {
+  if (w == 1) return dispatch_quant_w<T, 1, LN, MODE>(P, smem, grid, st);
   if (w == 2) return dispatch_quant_w<T, 2, LN, MODE>(P, smem, grid, st);
   if (w == 4) return dispatch_quant_w<T, 4, LN, MODE>(P, smem, grid, st);
   if constexpr (!LN) {
@@ -594,20 +672,23 @@ cudaError_t dispatch_quant(const Pipe& P, int w, size_t smem, int grid, cudaStre
 }
 
 // Column-peak mode: 128-thread slices; the running peak of each owned
-// element stays in registers for up to 6 chunks per thread (4 for fp32).
+// element stays in registers for up to 4 chunks per thread (with the row in
+// fp32) or 6 (bf16, the row in storage form).
 template <typename T>
 cudaError_t dispatch_colmax(const Pipe& P, size_t smem, int grid, cudaStream_t st) {
   const int64_t per = (P.a.K / 8 + 127) / 128;
-  if (sizeof(T) == 4 && per > 4) return launch_t<T, 4, 0, true, ROW_COLMAX>(P, smem, grid, st);
   switch (per) {
     case 1: return launch_t<T, 4, 1, true, ROW_COLMAX>(P, smem, grid, st);
     case 2: return launch_t<T, 4, 2, true, ROW_COLMAX>(P, smem, grid, st);
     case 3: return launch_t<T, 4, 3, true, ROW_COLMAX>(P, smem, grid, st);
     case 4: return launch_t<T, 4, 4, true, ROW_COLMAX>(P, smem, grid, st);
-    case 5: return launch_t<T, 4, 5, true, ROW_COLMAX>(P, smem, grid, st);
-    case 6: return launch_t<T, 4, 6, true, ROW_COLMAX>(P, smem, grid, st);
-    default: return launch_t<T, 4, 0, true, ROW_COLMAX>(P, smem, grid, st);
+    default: break;
   }
+  if constexpr (sizeof(T) == 2) {  // bf16 rows held in storage form
+    if (per == 5) return launch_t<T, 4, 5, true, ROW_COLMAX>(P, smem, grid, st);
+    if (per == 6) return launch_t<T, 4, 6, true, ROW_COLMAX>(P, smem, grid, st);
+  }
+  return launch_t<T, 4, 0, true, ROW_COLMAX>(P, smem, grid, st);
 }
 
 template <typename T>
@@ -636,12 +717,25 @@ bool plan(int64_t K, sq_dtype xt, RowMode mode, bool ln, int* slots, int* w, siz
   int s = (int)((kSmemBudget - fixed) / rb);
   if (s > kMaxSlots) s = kMaxSlots;
   if (mode == ROW_COLMAX && !ln) return false;  // raw peaks: column strips (rowops.cu)
-  int ww;
-  if (mode == ROW_COLMAX) ww = 4;
-  else if (s >= 8) ww = 2;
-  else if (s >= 4) ww = 4;
-  else if (!ln) ww = 8;  // two slices of 8 warps share the (2 or 3) slots
-  else return false;
+  int ww = 0;
+  if (mode == ROW_COLMAX) {
+    ww = 4;
+  } else {
+    // the narrowest slice that holds its part of the row in fp32 registers
+    // (at most 8 chunks per thread) and has a slot per slice
+    const int64_t nch = K / 8;
+    for (int c = 1; c <= (ln ? 4 : 16); c *= 2)
+      if ((nch + 32 * c - 1) / (32 * c) <= 8 && s >= kConsumers / (32 * c)) {
+        ww = c;
+        break;
+      }
+    if (ww == 0) {
+      if (s >= 8) ww = 2;
+      else if (s >= 4) ww = 4;
+      else if (!ln) ww = 8;  // two slices of 8 warps share the (2 or 3) slots
+      else return false;
+    }
+  }
   const int ns = kConsumers / (32 * ww);
   if (s < ns || s < 2) return false;
   s = (s / ns) * ns;

@@ -88,4 +88,17 @@ __device__ __forceinline__ uint64_t global_ns() {
   return t;
 }
 
+// Programmatic dependent launch.  Every kernel of this library is launched
+// with programmatic stream serialization (launch_pdl, launch.cuh): it lets
+// the next kernel of the stream begin launching at once (that kernel's
+// blocks take SMs as they free up and run their data-free prologue), and it
+// waits for the previous kernel of the stream to complete -- with its
+// memory writes visible -- before its own first global-memory access.  Every
+// thread of every block executes pdl_wait() before touching global memory
+// and before it can exit, so completion stays transitive along the stream.
+__device__ __forceinline__ void pdl_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
 }  // namespace sq
