@@ -21,7 +21,7 @@ SOURCES = ["api.cpp", "status.cu", "rowops.cu", "rowpipe.cu", "gemm.cu"]
 # rounded (the INT8 codes are bit-exact against the oracle); its one intended
 # fused multiply-add is an explicit intrinsic, which this flag leaves alone.
 EXTRA_FLAGS = {"rowpipe.cu": ["-fmad=false"]}
-HEADERS = ["sq_internal.h", "sq_device.cuh", "tc_ptx.cuh"]
+HEADERS = ["sq_internal.h", "sq_device.cuh", "tc_ptx.cuh", "launch.cuh"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 NVCC_FLAGS = ["-O3", "-std=c++17", "-lineinfo", "-Xcompiler", "-fPIC",
               "-Xcompiler", "-Wall", "-I", INCLUDE, "-I", CSRC]

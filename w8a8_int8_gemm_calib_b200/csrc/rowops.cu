@@ -89,7 +89,9 @@ colmax_kernel(const T* __restrict__ x, int64_t T_, int64_t K, int64_t rows_per_s
 
 // Column strips stream the rows with plain 16-byte loads and no
 // synchronisation at all; measured faster here than staging whole rows
-// through the shared-memory ring (which pays a handshake per row).
+// through the shared-memory ring, where every row waits for all the warps
+// that share it before its slot is refilled (W of 12288 x 4096 bf16: 30.8 us
+// against 55 us).
 cudaError_t launch_colmax(const void* x, sq_dtype xt, int64_t T, int64_t K, float* out,
                           cudaStream_t st) {
   const int64_t strips = (K + 255) / 256;

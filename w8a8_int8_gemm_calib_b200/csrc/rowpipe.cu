@@ -44,6 +44,7 @@ constexpr int kConsumers = 512;        // consumer threads per CTA
 constexpr int kThreads = kConsumers + 32;
 constexpr int kMaxSlots = 24;
 constexpr size_t kSmemBudget = 226 * 1024;  // + static shared memory stays under the 227 KB per-block limit
+constexpr size_t kSmemBudget2 = 112 * 1024;  // two CTAs per SM (228 KB per SM)
 constexpr uint32_t kCopyPiece = 32768;
 constexpr uint64_t kWaitNs = 2000000000ull;
 constexpr uint64_t kDrainNs = 1000000000ull;
@@ -159,11 +160,22 @@ __device__ __forceinline__ float2 mul2(float2 a, float2 b) {
   return r;
 }
 
-// max(|m|, |y|) with NaN propagated (the sign bit of the result is not
-// meaningful: callers take the magnitude at the end)
-__device__ __forceinline__ float maxabs_nan(float m, float y) {
+// Maxima with NaN propagated: NaN if any operand is NaN.  The three-operand
+// form takes |a| and |b| as operand modifiers (one instruction for two
+// elements); the warp form is one redux over the 32 lanes' magnitudes.
+__device__ __forceinline__ float max_nan(float a, float b) {
   float r;
-  asm("max.NaN.xorsign.abs.f32 %0, %1, %2;" : "=f"(r) : "f"(m), "f"(y));
+  asm("max.NaN.f32 %0, %1, %2;" : "=f"(r) : "f"(a), "f"(b));
+  return r;
+}
+__device__ __forceinline__ float max_nan3(float a, float b, float c) {
+  float r;
+  asm("max.NaN.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
+__device__ __forceinline__ float warp_maxabs_nan(float v) {
+  float r;
+  asm volatile("redux.sync.max.abs.NaN.f32 %0, %1, 0xffffffff;" : "=f"(r) : "f"(v));
   return r;
 }
 
@@ -189,6 +201,43 @@ __device__ __forceinline__ void store_codes(int8_t* dst, const uint32_t (&b)[8])
   *reinterpret_cast<uint2*>(dst) = pk;
 }
 
+// Producer (one thread): streams rows r0 .. r0+R-1 of P.a.x into the ring,
+// row i into slot i mod S, each slot refilled once its consumers released it
+// (empty barrier).  On a time-out it lets every copy already issued land
+// before returning, so the CTA never exits with a bulk copy in flight.
+__device__ __forceinline__ void produce_rows(const Pipe& P, uint32_t ring_u32, uint64_t* bars,
+                                             int64_t r0, int64_t R, volatile int* abort_flag) {
+  const int S = P.slots;
+  const uint32_t RB = P.row_bytes;
+  auto full_bar = [&](int s) { return tc::smem_u32(bars + s); };
+  auto empty_bar = [&](int s) { return tc::smem_u32(bars + kMaxSlots + s); };
+  uint32_t issued = 0, issued_par = 0;
+  bool ok = true;
+  const uint8_t* src = reinterpret_cast<const uint8_t*>(P.a.x) + r0 * (int64_t)RB;
+  for (int64_t i = 0; i < R; ++i) {
+    const int s = (int)(i % S);
+    const int64_t u = i / S;
+    if (u > 0 && !tc::mbar_wait(empty_bar(s), (uint32_t)((u - 1) & 1), abort_flag, kWaitNs,
+                                P.status)) {
+      ok = false;
+      break;
+    }
+    tc::mbar_arrive_expect_tx(full_bar(s), RB);
+    for (uint32_t off = 0; off < RB; off += kCopyPiece) {
+      const uint32_t n = RB - off < kCopyPiece ? RB - off : kCopyPiece;
+      tc::bulk_load(ring_u32 + (uint32_t)s * RB + off, src + i * (int64_t)RB + off, n, full_bar(s));
+    }
+    issued |= 1u << s;
+    issued_par = (issued_par & ~(1u << s)) | ((uint32_t)(u & 1) << s);
+  }
+  if (!ok) {
+    int never = 0;
+    for (int s = 0; s < S; ++s)
+      if (issued & (1u << s))
+        tc::mbar_wait(full_bar(s), (issued_par >> s) & 1u, &never, kDrainNs, P.status);
+  }
+}
+
 // Ring ownership: slice q consumes the CTA's rows i = q, q + NS, ... and row
 // i sits in slot i mod S.  The host makes S a multiple of NS, so each slot
 // is consumed by exactly one slice, in order: a slice waits on a slot only
@@ -207,18 +256,19 @@ __device__ __forceinline__ void store_codes(int8_t* dst, const uint32_t (&b)[8])
 // same IEEE round-to-nearest operation as its scalar form; x - mu is
 // computed as x + (-mu), which IEEE defines identically.  The running sums of the
 // LayerNorm stay scalar (their order is fixed).
-template <typename T, int W, int CM, bool LN, int MODE>
-__global__ void __launch_bounds__(kThreads, 1) rowpipe_kernel(const Pipe P) {
+template <typename T, int W, int CM, bool LN, int MODE, int NB>
+__global__ void __launch_bounds__(kThreads, NB) rowpipe_kernel(const Pipe P) {
   constexpr int ST = 32 * W;            // threads per slice
   constexpr int NS = kConsumers / ST;   // slices per CTA
   constexpr int G = W <= 4 ? 4 / W : 1;  // slot groups per thread (LayerNorm modes: W <= 4)
   static_assert(!LN || W == 1 || W == 2 || W == 4, "the LayerNorm order needs 1-, 2- or 4-warp slices");
   static_assert(MODE != ROW_COLMAX || LN, "raw column peaks use the column-strip kernel");
   // where the row is kept while a slice works on it: fp32 registers (at most
-  // 64 per thread, with the column peaks when those are kept too), the
-  // storage form in registers, or the shared-memory slot itself
+  // 64 per thread with one CTA per SM, 32 with two; the column peaks count
+  // too when they are kept), the storage form in registers, or the
+  // shared-memory slot itself
   constexpr int SRC = CM == 0 ? kSrcSmem
-                      : CM * 8 * (MODE == ROW_COLMAX ? 2 : 1) <= 64 ? kSrcF32 : kSrcRaw;
+                      : CM * 8 * (MODE == ROW_COLMAX ? 2 : 1) <= 64 / NB ? kSrcF32 : kSrcRaw;
   extern __shared__ __align__(128) uint8_t smem[];
   __shared__ float red[NS][2][3][W];
   __shared__ int abort_s;
@@ -259,36 +309,7 @@ __global__ void __launch_bounds__(kThreads, 1) rowpipe_kernel(const Pipe P) {
   unsigned clipped = 0;
 
   if (tid >= kConsumers) {
-    // ------------------------------------------------------------ producer
-    // (starts streaming rows while the consumers stage the parameters)
-    if (tid == kConsumers) {
-      uint32_t issued = 0, issued_par = 0;
-      bool ok = true;
-      const uint8_t* src = reinterpret_cast<const uint8_t*>(a.x) + r0 * (int64_t)RB;
-      for (int64_t i = 0; i < R; ++i) {
-        const int s = (int)(i % S);
-        const int64_t u = i / S;
-        if (u > 0 && !tc::mbar_wait(empty_bar(s), (uint32_t)((u - 1) & 1), abort_flag, kWaitNs,
-                                    P.status)) {
-          ok = false;
-          break;
-        }
-        tc::mbar_arrive_expect_tx(full_bar(s), RB);
-        for (uint32_t off = 0; off < RB; off += kCopyPiece) {
-          const uint32_t n = RB - off < kCopyPiece ? RB - off : kCopyPiece;
-          tc::bulk_load(ring_u32 + (uint32_t)s * RB + off, src + i * (int64_t)RB + off, n,
-                        full_bar(s));
-        }
-        issued |= 1u << s;
-        issued_par = (issued_par & ~(1u << s)) | ((uint32_t)(u & 1) << s);
-      }
-      if (!ok) {
-        int never = 0;
-        for (int s = 0; s < S; ++s)
-          if (issued & (1u << s))
-            tc::mbar_wait(full_bar(s), (issued_par >> s) & 1u, &never, kDrainNs, P.status);
-      }
-    }
+    if (tid == kConsumers) produce_rows(P, ring_u32, bars, r0, R, abort_flag);
   } else {
     // ------------------------------------------------------------ consumers
     // per-column parameters into the split layout, with the global loads
@@ -518,22 +539,22 @@ __global__ void __launch_bounds__(kThreads, 1) rowpipe_kernel(const Pipe P) {
         });
       } else {
         // peak magnitude with NaN propagated: a finite result means every
-        // element is finite (and then it equals the NaN-ignoring peak)
-        float mn = 0.0f;
+        // element is finite (and then it equals the NaN-ignoring peak).  The
+        // maximum is exact in any order: four independent chains per thread.
+        float m4[4] = {0.0f, 0.0f, 0.0f, 0.0f};
         for_level(kLvlIn, [&](int, int c, float2 (&x)[4]) {
           ytrans(c, x);  // now y
 #pragma unroll
-          for (int e = 0; e < 4; ++e) mn = maxabs_nan(maxabs_nan(mn, x[e].x), x[e].y);
+          for (int e = 0; e < 4; ++e) m4[e] = max_nan3(m4[e], fabsf(x[e].x), fabsf(x[e].y));
         });
-#pragma unroll
-        for (int o = 16; o >= 1; o >>= 1) mn = maxabs_nan(mn, __shfl_xor_sync(0xffffffffu, mn, o));
+        float mn = warp_maxabs_nan(max_nan(max_nan3(m4[0], m4[1], m4[2]), m4[3]));
         if constexpr (W > 1) {
           if (lane == 0) red[q][parity][2][v] = mn;
           sync();
 #pragma unroll
-          for (int t = 0; t < W; ++t) mn = maxabs_nan(mn, red[q][parity][2][t]);
+          for (int t = 0; t < W; ++t) mn = max_nan(mn, red[q][parity][2][t]);
         }
-        float mx = fabsf(mn);
+        float mx = mn;  // >= 0, or NaN
         const bool clean = mx < INFINITY;  // false for inf and NaN
         if (!clean) {
           // non-finite elements: the peak over the non-NaN values (fmaxf)
@@ -622,9 +643,9 @@ size_t fixed_smem(int64_t K, bool ln, RowMode mode) {
   return b + 2 * kMaxSlots * 8;
 }
 
-template <typename T, int W, int CM, bool LN, int MODE>
+template <typename T, int W, int CM, bool LN, int MODE, int NB = 1>
 cudaError_t launch_t(const Pipe& P, size_t smem, int grid, cudaStream_t st) {
-  auto kern = rowpipe_kernel<T, W, CM, LN, MODE>;
+  auto kern = rowpipe_kernel<T, W, CM, LN, MODE, NB>;
   // the shared-memory limit is raised once per instantiation (and per
   // device), to the whole budget, so that launches stay free of driver calls
   static std::once_flag once[64];
@@ -634,7 +655,7 @@ cudaError_t launch_t(const Pipe& P, size_t smem, int grid, cudaStream_t st) {
   if (e != cudaSuccess || dev < 0 || dev >= 64) return e != cudaSuccess ? e : cudaErrorInvalidDevice;
   std::call_once(once[dev], [&] {
     attr_err[dev] = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)kSmemBudget);
+                                         (int)(NB == 2 ? kSmemBudget2 : kSmemBudget));
   });
   if (attr_err[dev] != cudaSuccess) return attr_err[dev];
   return launch_pdl(kern, dim3(grid), dim3(kThreads), smem, st, P);
@@ -647,9 +668,17 @@ cudaError_t launch_t(const Pipe& P, size_t smem, int grid, cudaStream_t st) {
 // reduction order allows W <= 4).  Up to 16 bf16 chunks per thread are held
 // in storage form instead; beyond that each pass re-reads shared memory.
 template <typename T, int W, bool LN, int MODE>
-cudaError_t dispatch_quant_w(const Pipe& P, size_t smem, int grid, cudaStream_t st) {
+cudaError_t dispatch_quant_w(const Pipe& P, int nb, size_t smem, int grid, cudaStream_t st) {
   constexpr bool kBf16 = sizeof(T) == 2;
   const int64_t per = (P.a.K / 8 + 32 * W - 1) / (32 * W);
+  if constexpr (!LN && W >= 2 && W <= 4) {
+    if (nb == 2) {  // two CTAs per SM: at most 4 chunks per thread
+      if (per <= 2) return launch_t<T, W, 2, LN, MODE, 2>(P, smem, grid, st);
+      if (per <= 4) return launch_t<T, W, 4, LN, MODE, 2>(P, smem, grid, st);
+      return cudaErrorInvalidValue;
+    }
+  }
+  if (nb != 1) return cudaErrorInvalidValue;
   if (per <= 2) return launch_t<T, W, 2, LN, MODE>(P, smem, grid, st);
   if (per <= 4) return launch_t<T, W, 4, LN, MODE>(P, smem, grid, st);
   if (per <= 8) return launch_t<T, W, 8, LN, MODE>(P, smem, grid, st);
@@ -660,13 +689,13 @@ cudaError_t dispatch_quant_w(const Pipe& P, size_t smem, int grid, cudaStream_t 
 }
 
 template <typename T, bool LN, int MODE>
-cudaError_t dispatch_quant(const Pipe& P, int w, size_t smem, int grid, cudaStream_t st) {
-  if (w == 1) return dispatch_quant_w<T, 1, LN, MODE>(P, smem, grid, st);
-  if (w == 2) return dispatch_quant_w<T, 2, LN, MODE>(P, smem, grid, st);
-  if (w == 4) return dispatch_quant_w<T, 4, LN, MODE>(P, smem, grid, st);
+cudaError_t dispatch_quant(const Pipe& P, int w, int nb, size_t smem, int grid, cudaStream_t st) {
+  if (w == 1) return dispatch_quant_w<T, 1, LN, MODE>(P, nb, smem, grid, st);
+  if (w == 2) return dispatch_quant_w<T, 2, LN, MODE>(P, nb, smem, grid, st);
+  if (w == 4) return dispatch_quant_w<T, 4, LN, MODE>(P, nb, smem, grid, st);
   if constexpr (!LN) {
-    if (w == 8) return dispatch_quant_w<T, 8, LN, MODE>(P, smem, grid, st);
-    if (w == 16) return dispatch_quant_w<T, 16, LN, MODE>(P, smem, grid, st);
+    if (w == 8) return dispatch_quant_w<T, 8, LN, MODE>(P, nb, smem, grid, st);
+    if (w == 16) return dispatch_quant_w<T, 16, LN, MODE>(P, nb, smem, grid, st);
   }
   return cudaErrorInvalidValue;
 }
@@ -692,38 +721,59 @@ cudaError_t dispatch_colmax(const Pipe& P, size_t smem, int grid, cudaStream_t s
 }
 
 template <typename T>
-cudaError_t dispatch_mode(const Pipe& P, RowMode mode, int w, size_t smem, int grid,
+cudaError_t dispatch_mode(const Pipe& P, RowMode mode, int w, int nb, size_t smem, int grid,
                           cudaStream_t st) {
   const bool ln = P.a.g != nullptr;
   switch (mode) {
     case ROW_DYNAMIC:
-      return ln ? dispatch_quant<T, true, ROW_DYNAMIC>(P, w, smem, grid, st)
-                : dispatch_quant<T, false, ROW_DYNAMIC>(P, w, smem, grid, st);
+      return ln ? dispatch_quant<T, true, ROW_DYNAMIC>(P, w, nb, smem, grid, st)
+                : dispatch_quant<T, false, ROW_DYNAMIC>(P, w, nb, smem, grid, st);
     case ROW_STATIC:
-      return ln ? dispatch_quant<T, true, ROW_STATIC>(P, w, smem, grid, st)
-                : dispatch_quant<T, false, ROW_STATIC>(P, w, smem, grid, st);
+      return ln ? dispatch_quant<T, true, ROW_STATIC>(P, w, nb, smem, grid, st)
+                : dispatch_quant<T, false, ROW_STATIC>(P, w, nb, smem, grid, st);
     case ROW_COLMAX:
-      return ln ? dispatch_colmax<T>(P, smem, grid, st) : cudaErrorInvalidValue;
+      return ln && nb == 1 ? dispatch_colmax<T>(P, smem, grid, st) : cudaErrorInvalidValue;
   }
   return cudaErrorInvalidValue;
 }
 
-// Ring depth and slice width: returns false when no valid pairing fits.
-// `slots` is a multiple of the slice count 16/w.
-bool plan(int64_t K, sq_dtype xt, RowMode mode, bool ln, int* slots, int* w, size_t* smem) {
+// Ring depth, slice width and CTAs per SM: returns false when no valid
+// combination fits.  `slots` is a multiple of the slice count 16/w.  Rows
+// without a LayerNorm (the weight fold, the plain quantizer) run two CTAs
+// per SM -- twice the resident warps -- when slices of at most 4 warps
+// hold the row with at most 4 chunks per thread and each slice still gets
+// two slots of look-ahead (measured: K = 4096 gains, wider rows, which
+// would need 8-warp slices and 4 slots, lose); everything else runs one
+// CTA per SM.
+bool plan(int64_t K, sq_dtype xt, RowMode mode, bool ln, int* slots, int* w, int* nb,
+          size_t* smem) {
   const size_t rb = (size_t)K * (xt == SQ_BF16 ? 2 : 4);
   const size_t fixed = fixed_smem(K, ln, mode);
+  const int64_t nch = K / 8;
+  if (mode == ROW_COLMAX && !ln) return false;  // raw peaks: column strips (rowops.cu)
+  if (!ln && mode != ROW_COLMAX && fixed + 2 * rb <= kSmemBudget2) {
+    int s2 = (int)((kSmemBudget2 - fixed) / rb);
+    if (s2 > kMaxSlots) s2 = kMaxSlots;
+    for (int c = 2; c <= 4; c *= 2) {
+      const int ns = kConsumers / (32 * c);
+      if ((nch + 32 * c - 1) / (32 * c) <= 4 && s2 >= 2 * ns) {
+        *slots = (s2 / ns) * ns;
+        *w = c;
+        *nb = 2;
+        *smem = (size_t)*slots * rb + fixed;
+        return true;
+      }
+    }
+  }
   if (fixed + 2 * rb > kSmemBudget) return false;
   int s = (int)((kSmemBudget - fixed) / rb);
   if (s > kMaxSlots) s = kMaxSlots;
-  if (mode == ROW_COLMAX && !ln) return false;  // raw peaks: column strips (rowops.cu)
   int ww = 0;
   if (mode == ROW_COLMAX) {
     ww = 4;
   } else {
     // the narrowest slice that holds its part of the row in fp32 registers
     // (at most 8 chunks per thread) and has a slot per slice
-    const int64_t nch = K / 8;
     for (int c = 1; c <= (ln ? 4 : 16); c *= 2)
       if ((nch + 32 * c - 1) / (32 * c) <= 8 && s >= kConsumers / (32 * c)) {
         ww = c;
@@ -741,6 +791,7 @@ bool plan(int64_t K, sq_dtype xt, RowMode mode, bool ln, int* slots, int* w, siz
   s = (s / ns) * ns;
   *slots = s;
   *w = ww;
+  *nb = 1;
   *smem = (size_t)s * rb + fixed;
   return true;
 }
@@ -748,19 +799,19 @@ bool plan(int64_t K, sq_dtype xt, RowMode mode, bool ln, int* slots, int* w, siz
 }  // namespace
 
 bool rowpipe_fits(int64_t K, sq_dtype xt, RowMode mode, bool ln) {
-  int slots, w;
+  int slots, w, nb;
   size_t smem;
-  return plan(K, xt, mode, ln, &slots, &w, &smem);
+  return plan(K, xt, mode, ln, &slots, &w, &nb, &smem);
 }
 
 cudaError_t launch_rowpipe(const RowArgs& a, sq_dtype xt, RowMode mode, cudaStream_t st) {
   const size_t rb = (size_t)a.K * (xt == SQ_BF16 ? 2 : 4);
-  int slots = 0, w = 0;
+  int slots = 0, w = 0, nb = 1;
   size_t smem = 0;
-  if (!plan(a.K, xt, mode, a.g != nullptr, &slots, &w, &smem)) return cudaErrorInvalidValue;
+  if (!plan(a.K, xt, mode, a.g != nullptr, &slots, &w, &nb, &smem)) return cudaErrorInvalidValue;
   unsigned int* sw = status_word();
   if (!sw) return cudaErrorInvalidDevice;
-  int grid = sm_count();
+  int grid = sm_count() * nb;
   if ((int64_t)grid > a.T) grid = (int)a.T;
   Pipe P{};
   P.a = a;
@@ -770,8 +821,8 @@ cudaError_t launch_rowpipe(const RowArgs& a, sq_dtype xt, RowMode mode, cudaStre
   P.slots = slots;
   P.count = a.n_clipped != nullptr;
   P.status = sw;
-  return xt == SQ_BF16 ? dispatch_mode<uint16_t>(P, mode, w, smem, grid, st)
-                       : dispatch_mode<float>(P, mode, w, smem, grid, st);
+  return xt == SQ_BF16 ? dispatch_mode<uint16_t>(P, mode, w, nb, smem, grid, st)
+                       : dispatch_mode<float>(P, mode, w, nb, smem, grid, st);
 }
 
 }  // namespace sq
