@@ -13,9 +13,12 @@ tcgen05 GEMM with the dequantizing epilogue.
 `value` is whole-job throughput in TOPS = 2*M*N*K per step (all ranks) over
 the device time of the timed steps, max over ranks.  Each step is one replay
 of a CUDA graph of the five calls, timed on the device by event nodes at the
-graph's two ends; a second graph with an event node between calls, replayed
-after the timed steps, gives the per-call breakdown.  L2 is flushed (a 256 MiB write) before every
-timed step, outside the timed events.  Inputs are resident in HBM.
+graph's two ends.  The per-call breakdown, taken after the timed steps,
+times graphs of the first 1..4 calls the same way: a call's time is what it
+adds to the step.  Before every timed replay L2 is flushed outside the timed
+events: a 256 MiB buffer is written, then another 256 MiB buffer is read, so
+that the timed work finds neither its data nor the flush's dirty lines in
+L2.  Inputs are resident in HBM.
 `e2e` is the same metric through the public Python API with pinned host
 buffers: every step copies its inputs host->device and its output back.
 `--impl reference` times the CPU oracle (tests-only code) on bounded samples
@@ -48,7 +51,10 @@ INT8_PER_BF16 = 2.0
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 # DRAM bytes (read + write) of one launch of the dominant kernel, from the ncu
 # capture summarised in profiles/ (null when the kernel has changed since)
-GEMM_DRAM_TRAFFIC = {}
+GEMM_DRAM_TRAFFIC = {
+    "opt6.7b_qkv_t2048": (75.44e6, "profiles/gemm_w8a8_tc_opt6.7b_qkv_t2048.md: "
+                          "dram__bytes_read.sum 58.82 MB + dram__bytes_write.sum 16.62 MB"),
+}
 
 
 def load_peaks():
@@ -91,8 +97,8 @@ def config_of(wl, lin, world):
         "layernorm": lin.ln, "alpha": lin.alpha,
         "act_quant": "per-token dynamic" if lin.per_token else "per-tensor static",
         "io_dtype": lin.dtype,
-        "l2": "flushed before every timed step (256 MiB write, outside the timed events)",
-        "timing": "CUDA graph per step, device events at its two ends; per-call times from a second graph with events between calls",
+        "l2": "flushed before every timed step, outside the timed events (256 MiB written, then another 256 MiB read)",
+        "timing": "CUDA graph per step, device events at its two ends; per-call times as differences of graphs of the step's first 1..5 calls",
         "parallelism": f"replicas x{world}",
     }
 
@@ -186,39 +192,53 @@ class Layer:
         self.act = torch.empty(M if lin.per_token else 1, dtype=f32, device=dev)
         self.y = torch.empty((M, N), dtype=io, device=dev)
         self.workspace = sq.Workspace(dev)
-        self.kernels_per_step = 7
+        # this library's kernels per step: calibration peak; column peak +
+        # eq. (4) factors; weight fold (+ LayerNorm fold); quantizer; GEMM
+        self.kernels_per_step = 7 if lin.ln else 6
 
-    def step(self, ev=None):
+    def step(self, ev=None, upto=5):
+        """The first `upto` of the five calls (all five: one step); ev = (start,
+        end) events recorded around them, or None."""
         sq, L = self.sq, self.lin
-        e = ev or [None] * 6
-
-        def rec(i):
-            if e[i] is not None:
-                e[i].record()
-
-        rec(0)
+        if ev is not None:
+            ev[0].record()
         self.amax.zero_()
         sq.sq_calib_absmax(self.x_cal, self.amax, self.gamma, self.beta, 1e-5)
-        rec(1)
-        sq.sq_smooth_scales(self.amax, self.w, L.alpha, self.s, self.inv_s,
-                            None if L.per_token else self.dA)
-        rec(2)
-        sq.sq_fuse_weights_q8(self.w, self.s, self.wq, self.ws, self.gamma, self.beta,
-                              self.g2, self.b2)
-        rec(3)
+        if upto >= 2:
+            sq.sq_smooth_scales(self.amax, self.w, L.alpha, self.s, self.inv_s,
+                                None if L.per_token else self.dA)
+        if upto >= 3:
+            sq.sq_fuse_weights_q8(self.w, self.s, self.wq, self.ws, self.gamma, self.beta,
+                                  self.g2, self.b2)
         act = self.act
-        if not L.per_token:
-            act.copy_(self.dA)
-        if L.ln:
-            sq.sq_ln_smooth_quant_act(self.x, self.xq, act, self.g2, self.b2, 1e-5,
-                                      per_token=L.per_token)
-        else:
-            sq.sq_ln_smooth_quant_act(self.x, self.xq, act, inv_s=self.inv_s,
-                                      per_token=L.per_token)
-        rec(4)
-        sq.sq_gemm_w8a8(self.xq, self.wq, act, self.ws, self.y, per_token=L.per_token,
-                        workspace=self.workspace)
-        rec(5)
+        if upto >= 4:
+            if not L.per_token:
+                act.copy_(self.dA)
+            if L.ln:
+                sq.sq_ln_smooth_quant_act(self.x, self.xq, act, self.g2, self.b2, 1e-5,
+                                          per_token=L.per_token)
+            else:
+                sq.sq_ln_smooth_quant_act(self.x, self.xq, act, inv_s=self.inv_s,
+                                          per_token=L.per_token)
+        if upto >= 5:
+            sq.sq_gemm_w8a8(self.xq, self.wq, act, self.ws, self.y, per_token=L.per_token,
+                            workspace=self.workspace)
+        if ev is not None:
+            ev[1].record()
+
+
+class L2Flush:
+    """Evicts L2 between timed iterations: writes a buffer twice the L2 size,
+    then reads another one, so that L2 holds clean lines of neither inputs
+    nor outputs and the timed work pays no write-back of the flush."""
+
+    def __init__(self, torch, dev):
+        self.w = torch.empty(FLUSH_BYTES // 4, dtype=torch.int32, device=dev)
+        self.r = torch.zeros(FLUSH_BYTES // 4, dtype=torch.int32, device=dev)
+
+    def __call__(self, i):
+        self.w.fill_(i)
+        self.sink = self.r.max()
 
 
 def max_over_ranks(value: float, world: int, device) -> float:
@@ -273,7 +293,7 @@ def run_ours(args):
     wl, lin = pick_linear(args)
     d = synth.make_linear_inputs(lin)
     layer = Layer(sq, torch, lin, d, dev)
-    flush = torch.empty(FLUSH_BYTES // 4, dtype=torch.int32, device=dev)
+    flush = L2Flush(torch, dev)
 
     def barrier():
         if world > 1:
@@ -283,49 +303,57 @@ def run_ours(args):
     for _ in range(max(3, args.warmup)):
         layer.step()
     sq.sq_sync_status()
-    # one CUDA graph per step: the five calls (seven kernels) replay without
-    # host launch gaps; event nodes inside the graph time each call on the
-    # device
     names = ["calib_absmax", "smooth_scales", "fuse_weights_q8", "ln_smooth_quant_act",
              "gemm_w8a8"]
-    # the timed graph has event nodes only at its two ends; a second graph
-    # with an event between every call gives the per-call breakdown (its
-    # replays run after the timed region)
-    ev_step = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(2)]
-    graph = torch.cuda.CUDAGraph()
-    with torch.cuda.graph(graph):
-        layer.step([ev_step[0], None, None, None, None, ev_step[1]])
-    evs = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(6)]
-    graph_calls = torch.cuda.CUDAGraph()
-    with torch.cuda.graph(graph_calls):
-        layer.step(evs)
+
+    def capture(upto):
+        ev = (torch.cuda.Event(enable_timing=True, external=True),
+              torch.cuda.Event(enable_timing=True, external=True))
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            layer.step(ev, upto)
+        return g, ev
+
+    # the timed graph: one whole step (five calls, seven kernels), event
+    # nodes only at its two ends
+    graph, ev_step = capture(5)
     for _ in range(max(3, args.warmup)):
         graph.replay()
-        graph_calls.replay()
     barrier()
 
     K = args.steps
-    per = {n: [] for n in names}
     step_ms = []
     clocks = ClockSampler(torch.cuda.current_device())
     with clocks:
         barrier()
         for i in range(K):
-            flush.fill_(i)  # evicts the previous step's data from L2
+            flush(i)  # evicts the previous step's data from L2
             graph.replay()
             torch.cuda.synchronize()
             step_ms.append(ev_step[0].elapsed_time(ev_step[1]))
         barrier()
-    for i in range(K):
-        flush.fill_(i)
-        graph_calls.replay()
-        torch.cuda.synchronize()
-        for j, n in enumerate(names):
-            per[n].append(evs[j].elapsed_time(evs[j + 1]))
     sq.sq_sync_status()
     total_ms = max_over_ranks(float(sum(step_ms)), world, dev)
     ops = 2.0 * lin.T * lin.N * lin.K
     value = throughput_tops(ops, K, world, total_ms)
+
+    # per-call breakdown (after the timed region): graphs of the first 1..4
+    # calls, timed like the step; a call's time is what it adds to the step
+    prefix_ms = {5: statistics.mean(step_ms)}
+    for upto in range(1, 5):
+        g, ev = capture(upto)
+        g.replay()
+        t = []
+        for i in range(K):
+            flush(i)
+            g.replay()
+            torch.cuda.synchronize()
+            t.append(ev[0].elapsed_time(ev[1]))
+        prefix_ms[upto] = statistics.mean(t)
+        del g
+    prefix_ms[0] = 0.0
+    per = {n: prefix_ms[j + 1] - prefix_ms[j] for j, n in enumerate(names)}
+    sq.sq_sync_status()
 
     # ---- e2e through the public API with pinned host buffers
     e2e = run_e2e(sq, torch, layer, lin, d, dev, args.e2e_steps, world, barrier)
@@ -334,13 +362,13 @@ def run_ours(args):
     peaks, peak_kind = load_peaks()
     bf16_peak = peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"])
     int8_peak = bf16_peak * INT8_PER_BF16
-    gemm_ms = statistics.mean(per["gemm_w8a8"])
+    gemm_ms = per["gemm_w8a8"]
     gemm_tops = ops / (gemm_ms * 1e-3) / 1e12
     ab = algorithmic_bytes(lin)
     hbm = peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"])
     kernels = {}
     for n in names:
-        ms = statistics.mean(per[n])
+        ms = per[n]
         k = {"ms": round(ms, 5), "gbs": round(ab[n] / (ms * 1e-3) / 1e9, 1),
              "hbm_frac": round(ab[n] / (ms * 1e-3) / 1e9 / hbm, 3)}
         if n == "gemm_w8a8":
@@ -419,7 +447,7 @@ def run_small_m(sq, torch, dev, flush, reps=20):
             e1.record()
         times = []
         for i in range(reps):
-            flush.fill_(i)
+            flush(i)
             graph.replay()
             torch.cuda.synchronize()
             times.append(e0.elapsed_time(e1))
