@@ -33,6 +33,7 @@ F32 = 0
 BF16 = 1
 PER_TENSOR_STATIC = 0
 PER_TOKEN_DYNAMIC = 1
+PER_TENSOR_DYNAMIC = 2
 
 CFLAGS = ["-O2", "-ffp-contract=off", "-fno-fast-math", "-std=c11",
           "-shared", "-fPIC", "-Wall"]
@@ -195,12 +196,16 @@ def fold_ln(gamma, beta, s):
 
 
 def quant_act(x, gamma_s=None, beta_s=None, eps=1e-5, inv_s=None,
-              per_token=True, static_delta=None):
-    """S5: returns (xq int8 [T,K], act_scale [T] or [1], n_clipped)."""
+              per_token=True, static_delta=None, per_tensor_dynamic=False):
+    """S5: returns (xq int8 [T,K], act_scale [T] or [1], n_clipped).
+    per_tensor_dynamic: one step from the peak of the whole call (O2)."""
     x, xt = _typed(x)
     T, K = x.shape
     gamma_s, beta_s, inv_s = _f32(gamma_s), _f32(beta_s), _f32(inv_s)
-    if per_token:
+    if per_tensor_dynamic:
+        act = np.zeros(1, np.float32)
+        gran = PER_TENSOR_DYNAMIC
+    elif per_token:
         act = np.empty(T, np.float32)
         gran = PER_TOKEN_DYNAMIC
     else:

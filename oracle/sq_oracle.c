@@ -260,7 +260,24 @@ void orc_quant_act(const void* x, int xtype, int64_t T, int64_t K,
   float* row = (float*)malloc(sizeof(float) * (size_t)K);
   float* y = (float*)malloc(sizeof(float) * (size_t)K);
   float static_inv = 0.0f;
-  if (gran == ORC_PER_TENSOR_STATIC) static_inv = 1.0f / act_scale[0];
+  if (gran == ORC_PER_TENSOR_DYNAMIC) {
+    /* first pass: the peak of |y| over every row of the call */
+    float m = 0.0f;
+    for (int64_t t = 0; t < T; ++t) {
+      for (int64_t k = 0; k < K; ++k) row[k] = load_elem(x, xtype, t * K + k);
+      if (gamma_s) {
+        orc_layernorm_row(row, K, gamma_s, beta_s, eps, y);
+      } else {
+        for (int64_t k = 0; k < K; ++k) y[k] = inv_s ? row[k] * inv_s[k] : row[k];
+      }
+      for (int64_t k = 0; k < K; ++k) {
+        float a = fabsf(y[k]);
+        if (a > m) m = a;
+      }
+    }
+    act_scale[0] = orc_delta(m);
+  }
+  if (gran != ORC_PER_TOKEN_DYNAMIC) static_inv = 1.0f / act_scale[0];
   for (int64_t t = 0; t < T; ++t) {
     for (int64_t k = 0; k < K; ++k) row[k] = load_elem(x, xtype, t * K + k);
     if (gamma_s) {

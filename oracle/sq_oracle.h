@@ -42,7 +42,7 @@ extern "C" {
  * 16-bit pattern and widened to fp32 exactly. */
 enum { ORC_F32 = 0, ORC_BF16 = 1 };
 /* Activation granularity ([review] §2.5, §2.6 Fig. 3, §6.3 O1/O3). */
-enum { ORC_PER_TENSOR_STATIC = 0, ORC_PER_TOKEN_DYNAMIC = 1 };
+enum { ORC_PER_TENSOR_STATIC = 0, ORC_PER_TOKEN_DYNAMIC = 1, ORC_PER_TENSOR_DYNAMIC = 2 };
 
 /* Quantization step of the symmetric INT8 quantizer ([review] §2.2):
  * delta = max(amax, 1e-7) / 127, in fp32. */
@@ -91,6 +91,9 @@ void orc_fold_ln(const float* gamma, const float* beta, const float* s,
 /* S5: runtime activation quantizer.  y = LN'(x) with (gamma_s, beta_s) when
  * gamma_s != NULL, else y = x * inv_s (inv_s NULL = 1).  Per-token: writes
  * act_scale[t] = delta(max_k |y[t,k]|).  Static: reads act_scale[0].
+ * Per-tensor dynamic (the review's SmoothQuant-O2, §6.3; dynamic steps §2.5):
+ * writes act_scale[0] = delta(max_{t,k} |y[t,k]|) over the whole call, then
+ * quantizes every row with it.  Peaks skip NaN (a NaN is never > m).
  * n_clipped (may be NULL) is incremented by the number of elements whose
  * rounded code fell outside [-127, 127] and was saturated. */
 void orc_quant_act(const void* x, int xtype, int64_t T, int64_t K,

@@ -325,6 +325,62 @@ def test_static_quant_saturates(orc):
     assert ncl == 8
 
 
+def test_per_tensor_dynamic_hand_example(orc):
+    """Per-tensor dynamic quantization ([review] §6.3 O2; dynamic steps §2.5):
+    one step from the peak of the whole call.  Peak 4 -> Delta = 4/127, 1/Delta
+    = 31.75 (to fp32), so 1 -> 31.75 -> 32, -3 -> -95.25 -> -95, 1.5 -> 47.625
+    -> 48, 4 -> 127, 0.25 -> 7.9375 -> 8, -1 -> -32, 0.5 -> 15.875 -> 16.  The
+    peak lies in the second row: a per-row step would code the first row
+    differently."""
+    x = np.array([[1.0, -3.0, 0.0, 1.5], [4.0, 0.25, -1.0, 0.5]], np.float32)
+    xq, act, ncl = orc.quant_act(x, per_tensor_dynamic=True)
+    assert act.shape == (1,) and act[0] == np.float32(4.0) / np.float32(127.0)
+    assert xq.tolist() == [[32, -95, 0, 48], [127, 8, -32, 16]]
+    assert ncl == 0
+    xq1, act1, _ = orc.quant_act(x, per_token=True)
+    assert xq1[0].tolist() != xq[0].tolist()  # row 0 alone peaks at 3
+
+
+def test_per_tensor_dynamic_relations(orc):
+    """O2 against O1 and O3 on outlier-structured data, with and without a
+    LayerNorm: Delta is monotone in the peak, so the per-tensor step equals
+    the largest per-token step exactly, the codes equal static quantization
+    with that step, the global peak maps to +-127, and a one-row call equals
+    per-token quantization."""
+    lin = synth.workloads()["tiny_k1024"].linears[0]
+    d = synth.make_linear_inputs(lin, T=24, T_cal=32, N=8)
+    rng = np.random.default_rng(21)
+    inv_s = rng.uniform(0.05, 2, 1024).astype(np.float32)
+    g = (1 + 0.1 * rng.standard_normal(1024)).astype(np.float32)
+    b = (0.02 * rng.standard_normal(1024)).astype(np.float32)
+    for kw in (dict(inv_s=inv_s), dict(gamma_s=g, beta_s=b)):
+        xq2, act2, ncl2 = orc.quant_act(d["x"], per_tensor_dynamic=True, **kw)
+        _, act1, _ = orc.quant_act(d["x"], per_token=True, **kw)
+        assert act2[0] == act1.max()
+        xq3, _, ncl3 = orc.quant_act(d["x"], per_token=False, static_delta=act2[0], **kw)
+        assert np.array_equal(xq2, xq3) and ncl2 == ncl3 == 0
+        assert np.abs(xq2).max() == 127
+        t_peak = int(np.argmax(act1))
+        assert np.abs(xq2[t_peak]).max() == 127
+        xq_one, act_one, _ = orc.quant_act(d["x"][5:6], per_tensor_dynamic=True, **kw)
+        xq_tok, act_tok, _ = orc.quant_act(d["x"][5:6], per_token=True, **kw)
+        assert act_one[0] == act_tok[0] and np.array_equal(xq_one, xq_tok)
+
+
+def test_per_tensor_dynamic_non_finite(orc):
+    """NaN elements are skipped by the peak and coded 0; an infinite element
+    makes the step infinite, so every finite element codes to 0.  Peak 2:
+    1/Delta rounds to exactly 63.5 in fp32, so 1 -> 63.5 -> 64 (tie to even)
+    and -2 -> -127."""
+    x = np.array([[1.0, np.nan, -2.0, 0.5], [0.25, 1.0, np.nan, -1.0]], np.float32)
+    xq, act, _ = orc.quant_act(x, per_tensor_dynamic=True)
+    assert act[0] == np.float32(2.0) / np.float32(127.0)
+    assert xq[0, 1] == 0 and xq[1, 2] == 0 and xq[0, 2] == -127 and xq[0, 0] == 64
+    x[1, 0] = np.inf
+    xq, act, _ = orc.quant_act(x, per_tensor_dynamic=True)
+    assert np.isinf(act[0]) and not xq.any()
+
+
 def _torch_bf16_bits(v):
     import torch
 
