@@ -358,6 +358,7 @@ def run_ours(args):
     # ---- e2e through the public API with pinned host buffers
     e2e = run_e2e(sq, torch, layer, lin, d, dev, args.e2e_steps, world, barrier)
     small_m = None if args.no_small_m else run_small_m(sq, torch, dev, flush)
+    next_rows = {"o2_per_tensor_dynamic_quant": run_o2(sq, torch, layer, lin, flush)}
 
     peaks, peak_kind = load_peaks()
     bf16_peak = peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"])
@@ -403,6 +404,7 @@ def run_ours(args):
         },
         "kernels": kernels,
         "small_m_decode": small_m,
+        "next_rows": next_rows,
         "e2e": e2e,
         "gpu_launches": layer.kernels_per_step * K,
         "clocks": clocks.summary(),
@@ -459,6 +461,51 @@ def run_small_m(sq, torch, dev, flush, reps=20):
                         "hbm_frac": round(gbs / hbm, 3), "bytes": int(nbytes)}
         del graph
     return out
+
+
+def run_o2(sq, torch, layer, lin, flush, reps=20):
+    """Per-tensor dynamic activation quantization (SmoothQuant-O2) on the
+    step's activations: one step from the peak of the whole call, two passes
+    over x.  One CUDA-graph replay per call, L2 flushed before each, device
+    events around it; GB/s over the algorithmic bytes (x read once, codes
+    written once), so the second read of x shows as a lower fraction."""
+    M, K = lin.T, lin.K
+    b = 2 if lin.dtype == "bf16" else 4
+    act = torch.empty(1, dtype=torch.float32, device=layer.x.device)
+
+    def call():
+        if lin.ln:
+            sq.sq_ln_smooth_quant_act(layer.x, layer.xq, act, layer.g2, layer.b2, 1e-5,
+                                      per_tensor_dynamic=True)
+        else:
+            sq.sq_ln_smooth_quant_act(layer.x, layer.xq, act, inv_s=layer.inv_s,
+                                      per_tensor_dynamic=True)
+
+    for _ in range(3):
+        call()
+    e0 = torch.cuda.Event(enable_timing=True, external=True)
+    e1 = torch.cuda.Event(enable_timing=True, external=True)
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        e0.record()
+        call()
+        e1.record()
+    times = []
+    for i in range(reps):
+        flush(i)
+        graph.replay()
+        torch.cuda.synchronize()
+        times.append(e0.elapsed_time(e1))
+    sq.sq_sync_status()
+    del graph
+    ms = statistics.mean(times)
+    nbytes = M * K * b + M * K + 4 + (8 * K if lin.ln else 4 * K)
+    hbm = load_peaks()[0].get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"])
+    gbs = nbytes / (ms * 1e-3) / 1e9
+    return {"shape": f"{M}x{K} {lin.dtype}{' + LayerNorm' if lin.ln else ''}",
+            "kernels": "peak pass, step, static quantizer pass (x read twice)",
+            "us": round(ms * 1e3, 2), "gbs": round(gbs, 1), "hbm_frac": round(gbs / hbm, 3),
+            "bytes": int(nbytes)}
 
 
 def run_e2e(sq, torch, layer, lin, d, dev, steps, world, barrier):

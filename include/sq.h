@@ -69,11 +69,14 @@ typedef enum {
 typedef enum { SQ_F32 = 0, SQ_BF16 = 1 } sq_dtype;
 
 /* Activation quantization granularity ([review] §2.5, §2.6 Fig. 3, §6.3):
- * per-tensor with a static step fixed at calibration (SmoothQuant-O3), or
- * per-token with a step computed from each token's peak at run time (O1). */
+ * per-tensor with a static step fixed at calibration (SmoothQuant-O3),
+ * per-token with a step computed from each token's peak at run time (O1),
+ * or per-tensor with one step computed at run time from the peak of the
+ * whole call's activations (O2). */
 typedef enum {
   SQ_ACT_PER_TENSOR_STATIC = 0,
-  SQ_ACT_PER_TOKEN_DYNAMIC = 1
+  SQ_ACT_PER_TOKEN_DYNAMIC = 1,
+  SQ_ACT_PER_TENSOR_DYNAMIC = 2
 } sq_act_gran;
 
 typedef struct CUstream_st* sq_stream; /* a cudaStream_t */
@@ -156,6 +159,11 @@ sq_status sq_fuse_weights_q8(const void* w, sq_dtype wt, int64_t N, int64_t K,
  *       [T] fp32), xq[t,k] = Q(y[t,k]; act_scale[t]);
  *   SQ_ACT_PER_TENSOR_STATIC: act_scale[0] is the calibrated step (input),
  *       xq[t,k] = Q(y[t,k]; act_scale[0]); values above it saturate.
+ *   SQ_ACT_PER_TENSOR_DYNAMIC: act_scale[0] = Delta(max_{t,k} |y[t,k]|)
+ *       (output, [1] fp32; NaN elements are skipped by the peak and code to
+ *       0), xq[t,k] = Q(y[t,k]; act_scale[0]).  Two passes over x: the peak
+ *       is accumulated in act_scale[0] itself, which holds the peak, not a
+ *       step, until the call's last kernel has run on the stream.
  *
  *   x [T,K] type xt; xq [T,K] int8 out.
  *   n_clipped: NULL, or an int64 counter in device memory to which the number

@@ -17,7 +17,7 @@ from __future__ import annotations
 import torch
 
 from . import _lib
-from ._lib import (SQ_ACT_PER_TENSOR_STATIC, SQ_ACT_PER_TOKEN_DYNAMIC, SQ_BF16,
+from ._lib import (SQ_ACT_PER_TENSOR_DYNAMIC, SQ_ACT_PER_TENSOR_STATIC, SQ_ACT_PER_TOKEN_DYNAMIC, SQ_BF16,
                    SQ_F32, SQError, check, lib)
 
 __all__ = [
@@ -77,10 +77,16 @@ def sq_fuse_weights_q8(w, s, wq, w_scale, gamma=None, beta=None, gamma_out=None,
 
 
 def sq_ln_smooth_quant_act(x, xq, act_scale, gamma_s=None, beta_s=None, ln_eps=1e-5,
-                           inv_s=None, per_token=True, n_clipped=None, stream=None):
-    """Fused LN + smoothing + symmetric INT8 quantizer -> xq (and act_scale)."""
+                           inv_s=None, per_token=True, n_clipped=None, stream=None,
+                           per_tensor_dynamic=False):
+    """Fused LN + smoothing + symmetric INT8 quantizer -> xq (and act_scale).
+    per_token: one step per token; else the step in act_scale[0] (static), or
+    with per_tensor_dynamic one step from the peak of the whole call."""
     T, K = x.shape
-    gran = SQ_ACT_PER_TOKEN_DYNAMIC if per_token else SQ_ACT_PER_TENSOR_STATIC
+    if per_tensor_dynamic:
+        gran = SQ_ACT_PER_TENSOR_DYNAMIC
+    else:
+        gran = SQ_ACT_PER_TOKEN_DYNAMIC if per_token else SQ_ACT_PER_TENSOR_STATIC
     check(lib.sq_ln_smooth_quant_act(_ptr(x), _dt(x), T, K, _ptr(gamma_s), _ptr(beta_s),
                                      ln_eps, _ptr(inv_s), gran, _ptr(act_scale), _ptr(xq),
                                      _ptr(n_clipped), _stream(stream)),

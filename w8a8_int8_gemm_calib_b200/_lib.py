@@ -28,6 +28,7 @@ SQ_F32 = 0
 SQ_BF16 = 1
 SQ_ACT_PER_TENSOR_STATIC = 0
 SQ_ACT_PER_TOKEN_DYNAMIC = 1
+SQ_ACT_PER_TENSOR_DYNAMIC = 2
 
 EXPORTS = [
     "sq_calib_absmax", "sq_smooth_scales", "sq_fuse_weights_q8",

@@ -158,7 +158,8 @@ sq_status sq_ln_smooth_quant_act(const void* x, sq_dtype xt, int64_t T, int64_t 
   const char* fn = "sq_ln_smooth_quant_act";
   g_last_error[0] = 0;
   SQ_TRY(check_dtype(xt, fn));
-  if (gran != SQ_ACT_PER_TENSOR_STATIC && gran != SQ_ACT_PER_TOKEN_DYNAMIC)
+  if (gran != SQ_ACT_PER_TENSOR_STATIC && gran != SQ_ACT_PER_TOKEN_DYNAMIC &&
+      gran != SQ_ACT_PER_TENSOR_DYNAMIC)
     return fail(SQ_ERR_INVALID_ARG, "%s: unknown granularity %d", fn, (int)gran);
   if (T < 0) return fail(SQ_ERR_SHAPE, "%s: T=%lld < 0", fn, (long long)T);
   SQ_TRY(check_k(K, fn));
@@ -179,8 +180,22 @@ sq_status sq_ln_smooth_quant_act(const void* x, sq_dtype xt, int64_t T, int64_t 
   RowArgs a{};
   a.x = x; a.T = T; a.K = K; a.g = gamma_s; a.b = beta_s; a.eps = ln_eps; a.mul = inv_s;
   a.scale = act_scale; a.q = xq; a.n_clipped = (unsigned long long*)n_clipped;
-  cudaError_t e = launch_row(a, xt, gran == SQ_ACT_PER_TOKEN_DYNAMIC ? ROW_DYNAMIC : ROW_STATIC,
-                             (cudaStream_t)stream);
+  const cudaStream_t st = (cudaStream_t)stream;
+  cudaError_t e;
+  if (gran == SQ_ACT_PER_TENSOR_DYNAMIC) {
+    // two passes over x: the peak of |y| over the call (into act_scale[0]),
+    // Delta of it in place, then the static quantizer with that step
+    RowArgs p = a;
+    p.q = nullptr;
+    p.n_clipped = nullptr;
+    p.peak = act_scale;
+    e = cudaMemsetAsync(act_scale, 0, sizeof(float), st);
+    if (e == cudaSuccess) e = launch_row(p, xt, ROW_PEAK, st);
+    if (e == cudaSuccess) e = launch_peak_to_delta(act_scale, st);
+    if (e == cudaSuccess) e = launch_row(a, xt, ROW_STATIC, st);
+  } else {
+    e = launch_row(a, xt, gran == SQ_ACT_PER_TOKEN_DYNAMIC ? ROW_DYNAMIC : ROW_STATIC, st);
+  }
   return e == cudaSuccess ? SQ_OK : cuda_fail(e, fn);
 }
 

@@ -282,6 +282,7 @@ row_kernel(RowArgs a) {
   if (MODE == ROW_STATIC) static_inv = __fdiv_rn(1.0f, __ldg(a.scale));
   unsigned clipped = 0;
   int parity = 0;
+  float peak = 0.0f;  // ROW_PEAK: this thread's running max of |y| (NaN skipped)
 
   const int64_t stride = (int64_t)gridDim.x * kSlices;
   int64_t row = (int64_t)blockIdx.x * kSlices + slice;
@@ -348,6 +349,13 @@ row_kernel(RowArgs a) {
           }
         }
       });
+    } else if constexpr (MODE == ROW_PEAK) {
+      for_chunks<MAXC>(cur, xr, j, nchunk, [&](int i, int64_t c, const float (&v)[8]) {
+        float g8[8], b8[8];
+        params(i, c, g8, b8);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) peak = fmaxf(peak, fabsf(yv(v[e], g8[e], b8[e])));
+      });
     } else {
       float inv = static_inv;
       if constexpr (MODE == ROW_DYNAMIC) {
@@ -410,6 +418,10 @@ row_kernel(RowArgs a) {
       for (int64_t k = threadIdx.x; k < K; k += blockDim.x)
         atomicMax((unsigned int*)a.colmax + k, colmax_s[k]);
     }
+  }
+  if constexpr (MODE == ROW_PEAK) {
+    peak = warp_max(peak);
+    if (lane == 0) atomicMax(reinterpret_cast<unsigned int*>(a.peak), __float_as_uint(peak));
   }
   if (COUNT && a.n_clipped) {
 #pragma unroll
@@ -480,6 +492,9 @@ static cudaError_t dispatch_mode(const RowArgs& a, RowMode mode, cudaStream_t st
                  : dispatch_maxc<T, false, ROW_STATIC, false>(a, st);
     case ROW_COLMAX:
       return dispatch_maxc<T, true, ROW_COLMAX, false>(a, st);
+    case ROW_PEAK:
+      return ln ? dispatch_maxc<T, true, ROW_PEAK, false>(a, st)
+                : dispatch_maxc<T, false, ROW_PEAK, false>(a, st);
   }
   return cudaErrorInvalidValue;
 }
@@ -551,6 +566,19 @@ cudaError_t launch_scales(const float* amax_x, int64_t K, float alpha, float* s,
   if (blocks > 4 * (int64_t)sm_count()) blocks = 4 * (int64_t)sm_count();
   return launch_pdl(scales_kernel, dim3((unsigned)blocks), dim3(kScaleThreads), 0, st, amax_x, K,
                     alpha, s, inv_s, (unsigned int*)delta_out);
+}
+
+// ============================================================ per-tensor step
+// The second step of per-tensor dynamic quantization: the peak folded into
+// act_scale[0] by the ROW_PEAK pass becomes Delta = max(peak, 1e-7) / 127.
+__global__ void peak_to_delta_kernel(float* act_scale) {
+  pdl_launch_dependents();
+  pdl_wait();
+  if (threadIdx.x == 0) act_scale[0] = __fdiv_rn(fmaxf(act_scale[0], 1e-7f), 127.0f);
+}
+
+cudaError_t launch_peak_to_delta(float* act_scale, cudaStream_t st) {
+  return launch_pdl(peak_to_delta_kernel, dim3(1), dim3(32), 0, st, act_scale);
 }
 
 // ============================================================ LayerNorm fold

@@ -357,6 +357,7 @@ __global__ void __launch_bounds__(kThreads, NB) rowpipe_kernel(const Pipe P) {
     float cmax[NC];
 #pragma unroll
     for (int i = 0; i < NC; ++i) cmax[i] = 0.0f;
+    float pk[4] = {0.0f, 0.0f, 0.0f, 0.0f};  // ROW_PEAK: running max of |y| (NaN skipped)
     const float static_inv = MODE == ROW_STATIC ? __fdiv_rn(1.0f, __ldg(a.scale)) : 0.0f;
     const bool count = P.count != 0;
     int parity = 0;
@@ -525,6 +526,12 @@ __global__ void __launch_bounds__(kThreads, NB) rowpipe_kernel(const Pipe P) {
             }
           }
         });
+      } else if constexpr (MODE == ROW_PEAK) {
+        for_level(kLvlIn, [&](int, int c, float2 (&x)[4]) {
+          ytrans(c, x);
+#pragma unroll
+          for (int e = 0; e < 4; ++e) pk[e] = fmaxf(fmaxf(pk[e], fabsf(x[e].x)), fabsf(x[e].y));
+        });
       } else if constexpr (MODE == ROW_STATIC) {
         int8_t* qr = a.q + row * K;
         for_level(kLvlIn, [&](int, int c, float2 (&x)[4]) {
@@ -608,6 +615,10 @@ __global__ void __launch_bounds__(kThreads, NB) rowpipe_kernel(const Pipe P) {
         if (lane == 0) tc::mbar_arrive(empty_bar(s));
       }
       parity ^= 1;
+    }
+    if constexpr (MODE == ROW_PEAK) {
+      const float m = bmax(fmaxf(fmaxf(pk[0], pk[1]), fmaxf(pk[2], pk[3])));
+      if (lane == 0) atomicMax(reinterpret_cast<unsigned int*>(a.peak), __float_as_uint(m));
     }
     if constexpr (MODE == ROW_COLMAX && CM > 0) {
 #pragma unroll
@@ -731,6 +742,9 @@ cudaError_t dispatch_mode(const Pipe& P, RowMode mode, int w, int nb, size_t sme
     case ROW_STATIC:
       return ln ? dispatch_quant<T, true, ROW_STATIC>(P, w, nb, smem, grid, st)
                 : dispatch_quant<T, false, ROW_STATIC>(P, w, nb, smem, grid, st);
+    case ROW_PEAK:
+      return ln ? dispatch_quant<T, true, ROW_PEAK>(P, w, nb, smem, grid, st)
+                : dispatch_quant<T, false, ROW_PEAK>(P, w, nb, smem, grid, st);
     case ROW_COLMAX:
       return ln && nb == 1 ? dispatch_colmax<T>(P, smem, grid, st) : cudaErrorInvalidValue;
   }

@@ -25,7 +25,9 @@ sq_status fail(sq_status st, const char* fmt, ...);
 cudaError_t launch_colmax(const void* x, sq_dtype xt, int64_t T, int64_t K,
                           float* out, cudaStream_t st);
 
-enum RowMode { ROW_DYNAMIC = 0, ROW_STATIC = 1, ROW_COLMAX = 2 };
+// ROW_PEAK: no codes; the peak of |y| over every row of the call is folded
+// into *peak (per-tensor dynamic quantization, first pass).
+enum RowMode { ROW_DYNAMIC = 0, ROW_STATIC = 1, ROW_COLMAX = 2, ROW_PEAK = 3 };
 
 struct RowArgs {
   const void* x;
@@ -38,6 +40,7 @@ struct RowArgs {
   int8_t* q;           // [T,K] codes out (quantizing modes)
   unsigned long long* n_clipped;  // may be NULL
   float* colmax;       // ROW_COLMAX: running max [K] (fp32 bits, atomic max)
+  float* peak;         // ROW_PEAK: running peak [1] (fp32 bits, atomic max)
 };
 
 cudaError_t launch_row(const RowArgs& a, sq_dtype xt, RowMode mode,
@@ -53,6 +56,9 @@ cudaError_t launch_rowpipe(const RowArgs& a, sq_dtype xt, RowMode mode,
 cudaError_t launch_scales(const float* amax_x, int64_t K, float alpha,
                           float* s, float* inv_s, float* delta_out,
                           cudaStream_t st);
+
+// act_scale[0] = Delta(act_scale[0]) = max(peak, 1e-7) / 127 (one thread).
+cudaError_t launch_peak_to_delta(float* act_scale, cudaStream_t st);
 
 cudaError_t launch_fold_ln(const float* gamma, const float* beta,
                            const float* s, int64_t K, float* gamma_out,
