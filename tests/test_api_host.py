@@ -96,6 +96,14 @@ def test_quant_act_checks(lib):
                                     None) == lib.SQ_ERR_SHAPE
     assert L.sq_ln_smooth_quant_act(A, 1, 0, 16, None, None, 1e-5, None, 1, A2, A2, None,
                                     None) == lib.SQ_OK
+    # per-tensor dynamic (2) is a granularity; 3 is not; its checks are the same
+    assert L.sq_ln_smooth_quant_act(A, 1, 4, 16, None, None, 1e-5, None, 3, A2, A2, None,
+                                    None) == lib.SQ_ERR_INVALID_ARG
+    assert L.sq_ln_smooth_quant_act(A, 1, 4, 16, None, None, 1e-5, None, 2, MIS, A2, None,
+                                    None) == lib.SQ_ERR_ALIGN
+    assert L.sq_ln_smooth_quant_act(A, 1, 0, 16, None, None, 1e-5, None, 2, A2, A2, None,
+                                    None) == lib.SQ_OK
+    assert lib.SQ_ACT_PER_TENSOR_DYNAMIC == 2
 
 
 def test_gemm_checks(lib):
