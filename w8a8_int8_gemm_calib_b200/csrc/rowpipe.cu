@@ -238,6 +238,49 @@ __device__ __forceinline__ void produce_rows(const Pipe& P, uint32_t ring_u32, u
   }
 }
 
+// Consumer threads stage the per-column parameters (gamma and beta, or the
+// column multiplier) into the split layout, the global loads batched so that
+// several are in flight per thread, and zero the per-CTA column peaks
+// (colmax_s, when given).
+template <bool LN>
+__device__ __forceinline__ void stage_params(const RowArgs& a, float* pg, float* pb,
+                                             unsigned int* colmax_s, int K, int tid) {
+  constexpr int U = 8;
+  const int khalf = K >> 1;
+  const bool has_mul = !LN && a.mul != nullptr;
+  for (int k0 = tid; k0 < K; k0 += U * kConsumers) {
+    float gv[U], bv[U];
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const int k = k0 + u * kConsumers;
+      gv[u] = 0.0f;
+      bv[u] = 0.0f;
+      if (k < K) {
+        if (LN) {
+          gv[u] = __ldg(a.g + k);
+          if (a.b) bv[u] = __ldg(a.b + k);
+        } else if (has_mul) {
+          gv[u] = __ldg(a.mul + k);
+        }
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const int k = k0 + u * kConsumers;
+      if (k < K) {
+        const int pk = param_index(k, khalf);
+        if (LN) {
+          pg[pk] = gv[u];
+          pb[pk] = bv[u];
+        } else if (has_mul) {
+          pg[pk] = gv[u];
+        }
+        if (colmax_s) colmax_s[k] = 0u;
+      }
+    }
+  }
+}
+
 // Ring ownership: slice q consumes the CTA's rows i = q, q + NS, ... and row
 // i sits in slot i mod S.  The host makes S a multiple of NS, so each slot
 // is consumed by exactly one slice, in order: a slice waits on a slot only
@@ -312,42 +355,7 @@ __global__ void __launch_bounds__(kThreads, NB) rowpipe_kernel(const Pipe P) {
     if (tid == kConsumers) produce_rows(P, ring_u32, bars, r0, R, abort_flag);
   } else {
     // ------------------------------------------------------------ consumers
-    // per-column parameters into the split layout, with the global loads
-    // batched so that several are in flight per thread
-    {
-      constexpr int U = 8;
-      for (int k0 = tid; k0 < (int)K; k0 += U * kConsumers) {
-        float gv[U], bv[U];
-#pragma unroll
-        for (int u = 0; u < U; ++u) {
-          const int k = k0 + u * kConsumers;
-          gv[u] = 0.0f;
-          bv[u] = 0.0f;
-          if (k < (int)K) {
-            if (LN) {
-              gv[u] = __ldg(a.g + k);
-              if (a.b) bv[u] = __ldg(a.b + k);
-            } else if (has_mul) {
-              gv[u] = __ldg(a.mul + k);
-            }
-          }
-        }
-#pragma unroll
-        for (int u = 0; u < U; ++u) {
-          const int k = k0 + u * kConsumers;
-          if (k < (int)K) {
-            const int pk = param_index(k, khalf);
-            if (LN) {
-              pg[pk] = gv[u];
-              pb[pk] = bv[u];
-            } else if (has_mul) {
-              pg[pk] = gv[u];
-            }
-            if (MODE == ROW_COLMAX) colmax_s[k] = 0u;
-          }
-        }
-      }
-    }
+    stage_params<LN>(a, pg, pb, MODE == ROW_COLMAX ? colmax_s : nullptr, (int)K, tid);
     asm volatile("bar.sync 9, %0;" ::"r"(kConsumers) : "memory");  // consumers only
 
     const int q = tid / ST, j = tid % ST;
