@@ -82,7 +82,7 @@ def _declare(L):
     L.orc_fuse_weights_q8.argtypes = [_p, _i, _i64, _i64, _p, _p, _p]
     L.orc_fold_ln.argtypes = [_p, _p, _p, _i64, _p, _p]
     L.orc_quant_act.argtypes = [_p, _i, _i64, _i64, _p, _p, _f, _p, _i, _p, _p, _p]
-    L.orc_gemm_w8a8.argtypes = [_p, _p, _i64, _i64, _i64, _p, _i, _p, _p, _i64,
+    L.orc_gemm_w8a8.argtypes = [_p, _p, _i64, _i64, _i64, _p, _i, _p, _p, _p, _i64,
                                 _p, _p, _p]
     for fn in ("orc_layernorm_row", "orc_calib_absmax", "orc_weight_colmax",
                "orc_smooth_scales", "orc_fuse_weights_q8", "orc_fold_ln",
@@ -219,21 +219,22 @@ def quant_act(x, gamma_s=None, beta_s=None, eps=1e-5, inv_s=None,
 
 
 def gemm_w8a8(xq, wq, act_scale, w_scale, per_token=True, rows=None,
-              out_bf16=False):
+              out_bf16=False, bias=None):
     """S6: returns (y, acc): y fp32 or bf16 bits (uint16), acc int32.
 
     rows: optional token indices; only those rows are computed (in order).
+    bias: optional [N] fp32 added after the dequantization.
     """
     xq = np.ascontiguousarray(xq, np.int8)
     wq = np.ascontiguousarray(wq, np.int8)
     M, K = xq.shape
     N = wq.shape[0]
-    act_scale, w_scale = _f32(act_scale), _f32(w_scale)
+    act_scale, w_scale, bias = _f32(act_scale), _f32(w_scale), _f32(bias)
     r = None if rows is None else np.ascontiguousarray(rows, np.int64)
     R = M if r is None else r.size
     acc = np.empty((R, N), np.int32)
     yf = None if out_bf16 else np.empty((R, N), np.float32)
     yb = np.empty((R, N), np.uint16) if out_bf16 else None
     lib().orc_gemm_w8a8(_ptr(xq), _ptr(wq), M, N, K, _ptr(act_scale), int(per_token),
-                        _ptr(w_scale), _ptr(r), R, _ptr(yf), _ptr(yb), _ptr(acc))
+                        _ptr(w_scale), _ptr(bias), _ptr(r), R, _ptr(yf), _ptr(yb), _ptr(acc))
     return (yb if out_bf16 else yf), acc

@@ -312,8 +312,8 @@ void orc_quant_act(const void* x, int xtype, int64_t T, int64_t K,
 
 void orc_gemm_w8a8(const int8_t* xq, const int8_t* wq, int64_t M, int64_t N,
                    int64_t K, const float* act_scale, int act_per_token,
-                   const float* w_scale, const int64_t* rows, int64_t nrows,
-                   float* y_f32, uint16_t* y_bf16, int32_t* acc) {
+                   const float* w_scale, const float* bias, const int64_t* rows,
+                   int64_t nrows, float* y_f32, uint16_t* y_bf16, int32_t* acc) {
   int64_t R = rows ? nrows : M;
   for (int64_t i = 0; i < R; ++i) {
     int64_t t = rows ? rows[i] : i;
@@ -325,6 +325,7 @@ void orc_gemm_w8a8(const int8_t* xq, const int8_t* wq, int64_t M, int64_t N,
       int32_t a32 = (int32_t)sum; /* |sum| <= 127*127*K < 2^31 for K <= 133136 */
       float scale = as * w_scale[n];
       float y = (float)a32 * scale;
+      if (bias) y = y + bias[n];
       if (acc) acc[i * N + n] = a32;
       if (y_f32) y_f32[i * N + n] = y;
       if (y_bf16) y_bf16[i * N + n] = orc_f32_to_bf16(y);

@@ -102,14 +102,16 @@ void orc_quant_act(const void* x, int xtype, int64_t T, int64_t K,
                    int8_t* xq, int64_t* n_clipped);
 
 /* S6: acc[t,n] = sum_k xq[t,k]*wq[n,k] (int32, exact);
- * y = (float)acc * (act_scale[t or 0] * w_scale[n]).  Only the rows listed
- * in rows[0..nrows) are computed (rows == NULL: all M rows, nrows ignored);
+ * y = (float)acc * (act_scale[t or 0] * w_scale[n]), then + bias[n] when
+ * bias != NULL (one more fp32 addition: the linear's bias is untouched by
+ * the smoothing, [review] §5.1 eq. (3)).  Only the rows listed in
+ * rows[0..nrows) are computed (rows == NULL: all M rows, nrows ignored);
  * output row i of y/acc corresponds to input row rows[i].  y_bf16 and acc
  * may be NULL; y_f32 may be NULL. */
 void orc_gemm_w8a8(const int8_t* xq, const int8_t* wq, int64_t M, int64_t N,
                    int64_t K, const float* act_scale, int act_per_token,
-                   const float* w_scale, const int64_t* rows, int64_t nrows,
-                   float* y_f32, uint16_t* y_bf16, int32_t* acc);
+                   const float* w_scale, const float* bias, const int64_t* rows,
+                   int64_t nrows, float* y_f32, uint16_t* y_bf16, int32_t* acc);
 
 #ifdef __cplusplus
 }

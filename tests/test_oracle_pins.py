@@ -236,6 +236,31 @@ def test_gemm_brute_force_tiny(orc):
                 assert y[t, n] == yref
 
 
+def test_gemm_bias_exact(orc):
+    """The bias is added after the dequantization, per output channel
+    ([review] §5.1 eq. (3): smoothing leaves a linear's bias untouched).  With
+    power-of-two scales (2^-3 x 2^-5) and biases on the same 2^-8 grid every
+    value is exact in fp32, so y = (acc + j) / 256 for bias[n] = j / 256 --
+    checked against Python integers; a zero bias changes nothing."""
+    r = np.random.default_rng(15)
+    M, N, K = 9, 13, 64
+    xq = r.integers(-127, 128, (M, K)).astype(np.int8)
+    wq = r.integers(-127, 128, (N, K)).astype(np.int8)
+    act = np.full(M, 2.0 ** -3, np.float32)
+    ws = np.full(N, 2.0 ** -5, np.float32)
+    j = r.integers(-1000, 1001, N)
+    bias = (j / 256.0).astype(np.float32)
+    y, acc = orc.gemm_w8a8(xq, wq, act, ws, per_token=True, bias=bias)
+    for t in range(M):
+        for n in range(N):
+            ref = sum(int(xq[t, k]) * int(wq[n, k]) for k in range(K))
+            assert acc[t, n] == ref
+            assert y[t, n] == np.float32((ref + int(j[n])) / 256.0)
+    y0, _ = orc.gemm_w8a8(xq, wq, act, ws, per_token=True, bias=np.zeros(N, np.float32))
+    y1, _ = orc.gemm_w8a8(xq, wq, act, ws, per_token=True)
+    assert np.array_equal(y0, y1)
+
+
 def test_gemm_saturation_closed_form(orc):
     """All-127 operands: acc = 127*127*K = 16129*K (K=20480 -> 330,321,920),
     the largest magnitude any layer in the workloads reaches."""
