@@ -51,10 +51,7 @@ INT8_PER_BF16 = 2.0
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 # DRAM bytes (read + write) of one launch of the dominant kernel, from the ncu
 # capture summarised in profiles/ (null when the kernel has changed since)
-GEMM_DRAM_TRAFFIC = {
-    "opt6.7b_qkv_t2048": (75.44e6, "profiles/gemm_w8a8_tc_opt6.7b_qkv_t2048.md: "
-                          "dram__bytes_read.sum 58.82 MB + dram__bytes_write.sum 16.62 MB"),
-}
+GEMM_DRAM_TRAFFIC = {}
 
 
 def load_peaks():
@@ -358,7 +355,8 @@ def run_ours(args):
     # ---- e2e through the public API with pinned host buffers
     e2e = run_e2e(sq, torch, layer, lin, d, dev, args.e2e_steps, world, barrier)
     small_m = None if args.no_small_m else run_small_m(sq, torch, dev, flush)
-    next_rows = {"o2_per_tensor_dynamic_quant": run_o2(sq, torch, layer, lin, flush)}
+    next_rows = {"o2_per_tensor_dynamic_quant": run_o2(sq, torch, layer, lin, flush),
+                 "gemm_bias_epilogue": run_gemm_bias(sq, torch, layer, lin, flush)}
 
     peaks, peak_kind = load_peaks()
     bf16_peak = peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"])
@@ -506,6 +504,45 @@ def run_o2(sq, torch, layer, lin, flush, reps=20):
             "kernels": "peak pass, step, static quantizer pass (x read twice)",
             "us": round(ms * 1e3, 2), "gbs": round(gbs, 1), "hbm_frac": round(gbs / hbm, 3),
             "bytes": int(nbytes)}
+
+
+def run_gemm_bias(sq, torch, layer, lin, flush, reps=20):
+    """The step's GEMM with the bias epilogue (y = dequantized acc + bias[n]),
+    timed like the decode GEMM: one CUDA-graph replay per call after an L2
+    flush, device events around it."""
+    M, N, K = lin.T, lin.N, lin.K
+    g = torch.Generator(device=layer.x.device).manual_seed(7)
+    bias = torch.randn(N, device=layer.x.device, generator=g) * 0.1
+
+    def call():
+        sq.sq_gemm_w8a8(layer.xq, layer.wq, layer.act, layer.ws, layer.y,
+                        per_token=lin.per_token, workspace=layer.workspace, bias=bias)
+
+    for _ in range(3):
+        call()
+    e0 = torch.cuda.Event(enable_timing=True, external=True)
+    e1 = torch.cuda.Event(enable_timing=True, external=True)
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        e0.record()
+        call()
+        e1.record()
+    times = []
+    for i in range(reps):
+        flush(i)
+        graph.replay()
+        torch.cuda.synchronize()
+        times.append(e0.elapsed_time(e1))
+    sq.sq_sync_status()
+    del graph
+    ms = statistics.mean(times)
+    peaks, _ = load_peaks()
+    int8_peak = peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]) * INT8_PER_BF16
+    tops = 2.0 * M * N * K / (ms * 1e-3) / 1e12
+    return {"shape": f"{M}x{N}x{K}", "us": round(ms * 1e3, 2), "tops": round(tops, 1),
+            "int8_frac": round(tops / int8_peak, 3),
+            "note": "one call after an L2 flush, launch included (the step's GEMM share "
+                    "overlaps its launch with the quantizer)"}
 
 
 def run_e2e(sq, torch, layer, lin, d, dev, steps, world, barrier):

@@ -210,6 +210,25 @@ sq_status sq_gemm_w8a8(const int8_t* xq, const int8_t* wq, int64_t M,
                        size_t workspace_bytes, sq_stream stream);
 
 /*
+ * sq_gemm_w8a8_bias -- sq_gemm_w8a8 followed by the linear's bias: the
+ * smoothing leaves a bias untouched ([review] §5.1 eq. (3): X W + b =
+ * (X diag(s)^-1)(diag(s) W) + b), so it is added to the dequantized output:
+ *
+ *   y[t,n] = (float)acc[t,n] * (as_t * w_scale[n]) + bias[n]
+ *
+ * as one more fp32 addition (never fused with the multiply), before the bf16
+ * conversion.  bias: [N] fp32 device memory, 16-byte aligned, or NULL (then
+ * identical to sq_gemm_w8a8).  All other arguments, errors and the workspace
+ * as for sq_gemm_w8a8.
+ */
+sq_status sq_gemm_w8a8_bias(const int8_t* xq, const int8_t* wq, int64_t M,
+                            int64_t N, int64_t K, const float* act_scale,
+                            int act_per_token, const float* w_scale,
+                            const float* bias, void* y, sq_dtype yt,
+                            int32_t* acc_out, void* workspace,
+                            size_t workspace_bytes, sq_stream stream);
+
+/*
  * sq_gemm_w8a8_noalloc -- sq_gemm_w8a8 for callers that cannot allocate
  * device memory.  (No counterpart on the pages: this is a property of the
  * library interface, not of the method.)

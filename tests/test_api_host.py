@@ -106,6 +106,17 @@ def test_quant_act_checks(lib):
     assert lib.SQ_ACT_PER_TENSOR_DYNAMIC == 2
 
 
+def test_gemm_bias_checks(lib):
+    L = lib.lib
+    assert L.sq_gemm_w8a8_bias(A, A, 4, 4, 16, A2, 1, A2, MIS, A2, 1, None, None, 0, None) == \
+        lib.SQ_ERR_ALIGN
+    assert L.sq_gemm_w8a8_bias(A, A, 4, 4, 24, A2, 1, A2, A2, A2, 1, None, None, 0, None) == \
+        lib.SQ_ERR_SHAPE
+    assert "sq_gemm_w8a8_bias" in lib.last_error()
+    assert L.sq_gemm_w8a8_bias(A, A, 0, 4, 16, A2, 1, A2, A2, A2, 1, None, None, 0, None) == \
+        lib.SQ_OK
+
+
 def test_gemm_checks(lib):
     L = lib.lib
     assert L.sq_gemm_w8a8(A, A, 4, 4, 24, A2, 1, A2, A2, 1, None, None, 0, None) == \

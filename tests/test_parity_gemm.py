@@ -147,3 +147,46 @@ def test_gemm_small_m_rejects_short_workspace(sq):
     with pytest.raises(sq.SQError) as ei:
         sq.sq_gemm_w8a8(dev(xq), dev(wq), dev(act), dev(ws), y, workspace=short)
     assert ei.value.status == 8  # SQ_ERR_WORKSPACE
+
+
+# Shapes for the bias epilogue: large-M tiles with the TMA-store epilogue
+# (N a multiple of 8), with direct stores (N % 8 != 0), fp32 and bf16 out,
+# and the weight-streaming path (M <= 128, stream-K splits).
+BIAS_SHAPES = [(300, 512, 1040), (257, 300, 272), (1024, 2048, 512), (1, 4096, 4096),
+               (33, 1000, 2064), (128, 520, 1024)]
+
+
+@pytest.mark.parametrize("M,N,K", BIAS_SHAPES)
+@pytest.mark.parametrize("out", ["f32", "bf16"])
+@pytest.mark.parametrize("per_token", [True, False])
+def test_gemm_bias(sq, orc, M, N, K, out, per_token):
+    """y = dequantized accumulator + bias[n], bit for bit against the oracle
+    (sampled rows for the larger shapes, every column)."""
+    xq, wq, act, ws = _operands(M, N, K, M * 17 + N * 3 + K)
+    bias = np.random.default_rng(M + N).normal(0, 0.5, N).astype(np.float32)
+    act_used = act if per_token else act[:1]
+    rows = np.unique(np.array([0, 1, 127, 128, M // 2, M - 1]).clip(0, M - 1)).astype(np.int64)
+    y_want, acc_want = orc.gemm_w8a8(xq, wq, act_used, ws, per_token=per_token, rows=rows,
+                                     out_bf16=(out == "bf16"), bias=bias)
+    y = torch.empty((M, N), dtype=torch.bfloat16 if out == "bf16" else torch.float32,
+                    device="cuda")
+    acc = torch.empty((M, N), dtype=torch.int32, device="cuda")
+    sq.sq_gemm_w8a8(dev(xq), dev(wq), dev(act_used), dev(ws), y, per_token=per_token,
+                    acc_out=acc, workspace=sq.Workspace(), bias=dev(bias))
+    sq.sq_sync_status()
+    r = torch.from_numpy(rows).cuda()
+    assert_bits_equal(host(acc[r]), acc_want, "acc")
+    assert_bits_equal(host(y[r]), y_want, "y")
+
+
+def test_gemm_zero_bias_is_no_bias(sq):
+    """A zero bias leaves every output bit unchanged (both paths)."""
+    for M, N, K in [(300, 512, 1040), (8, 1000, 2064)]:
+        xq, wq, act, ws = [dev(v) for v in _operands(M, N, K, 99)]
+        y0 = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
+        y1 = torch.empty_like(y0)
+        sq.sq_gemm_w8a8(xq, wq, act, ws, y0, workspace=sq.Workspace())
+        sq.sq_gemm_w8a8(xq, wq, act, ws, y1, workspace=sq.Workspace(),
+                        bias=torch.zeros(N, dtype=torch.float32, device="cuda"))
+        sq.sq_sync_status()
+        assert torch.equal(y0.view(torch.int16), y1.view(torch.int16))

@@ -115,8 +115,9 @@ class Workspace:
 
 
 def sq_gemm_w8a8(xq, wq, act_scale, w_scale, y, per_token=True, acc_out=None,
-                 workspace=None, stream=None):
-    """y = (float)(xq @ wq^T) * (act_scale[t] * w_scale[n]); y fp32 or bf16."""
+                 workspace=None, stream=None, bias=None):
+    """y = (float)(xq @ wq^T) * (act_scale[t] * w_scale[n]) (+ bias[n]);
+    y fp32 or bf16.  With a bias this calls sq_gemm_w8a8_bias."""
     M, K = xq.shape
     N = wq.shape[0]
     need = sq_gemm_workspace_bytes(M, N, K)
@@ -125,10 +126,16 @@ def sq_gemm_w8a8(xq, wq, act_scale, w_scale, y, per_token=True, acc_out=None,
         if workspace is None:
             raise ValueError(f"sq_gemm_w8a8 needs a workspace of {need} bytes")
         ws = workspace.get(need) if isinstance(workspace, Workspace) else workspace
-    check(lib.sq_gemm_w8a8(_ptr(xq), _ptr(wq), M, N, K, _ptr(act_scale), int(per_token),
-                           _ptr(w_scale), _ptr(y), _dt(y), _ptr(acc_out), _ptr(ws),
-                           0 if ws is None else ws.numel() * ws.element_size(),
-                           _stream(stream)), "sq_gemm_w8a8")
+    nbytes = 0 if ws is None else ws.numel() * ws.element_size()
+    if bias is None:
+        check(lib.sq_gemm_w8a8(_ptr(xq), _ptr(wq), M, N, K, _ptr(act_scale), int(per_token),
+                               _ptr(w_scale), _ptr(y), _dt(y), _ptr(acc_out), _ptr(ws),
+                               nbytes, _stream(stream)), "sq_gemm_w8a8")
+    else:
+        check(lib.sq_gemm_w8a8_bias(_ptr(xq), _ptr(wq), M, N, K, _ptr(act_scale),
+                                    int(per_token), _ptr(w_scale), _ptr(bias), _ptr(y), _dt(y),
+                                    _ptr(acc_out), _ptr(ws), nbytes, _stream(stream)),
+              "sq_gemm_w8a8_bias")
     return y
 
 

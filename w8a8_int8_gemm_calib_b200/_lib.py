@@ -34,7 +34,7 @@ EXPORTS = [
     "sq_calib_absmax", "sq_smooth_scales", "sq_fuse_weights_q8",
     "sq_ln_smooth_quant_act", "sq_gemm_workspace_bytes", "sq_gemm_w8a8",
     "sq_sync_status", "sq_status_string", "sq_last_error",
-    "sq_selftest_bounded_wait", "sq_gemm_w8a8_noalloc",
+    "sq_selftest_bounded_wait", "sq_gemm_w8a8_noalloc", "sq_gemm_w8a8_bias",
 ]
 
 
@@ -59,6 +59,7 @@ def _load() -> ctypes.CDLL:
     L.sq_gemm_workspace_bytes.argtypes = [i64, i64, i64]
     L.sq_gemm_workspace_bytes.restype = sz
     L.sq_gemm_w8a8.argtypes = [p, p, i64, i64, i64, p, i, p, p, i, p, p, sz, p]
+    L.sq_gemm_w8a8_bias.argtypes = [p, p, i64, i64, i64, p, i, p, p, p, i, p, p, sz, p]
     L.sq_sync_status.argtypes = [p]
     L.sq_status_string.argtypes = [st]
     L.sq_status_string.restype = ctypes.c_char_p
@@ -68,7 +69,7 @@ def _load() -> ctypes.CDLL:
     L.sq_gemm_w8a8_noalloc.argtypes = [p, p, i64, i64, i64, p, i, p, p, i, p, p]
     for fn in ("sq_calib_absmax", "sq_smooth_scales", "sq_fuse_weights_q8",
                "sq_ln_smooth_quant_act", "sq_gemm_w8a8", "sq_sync_status",
-               "sq_selftest_bounded_wait", "sq_gemm_w8a8_noalloc"):
+               "sq_selftest_bounded_wait", "sq_gemm_w8a8_noalloc", "sq_gemm_w8a8_bias"):
         getattr(L, fn).restype = st
     return L
 

@@ -204,11 +204,11 @@ size_t sq_gemm_workspace_bytes(int64_t M, int64_t N, int64_t K) {
   return gemm_workspace_bytes(M, N, K);
 }
 
-sq_status sq_gemm_w8a8(const int8_t* xq, const int8_t* wq, int64_t M, int64_t N, int64_t K,
-                       const float* act_scale, int act_per_token, const float* w_scale, void* y,
-                       sq_dtype yt, int32_t* acc_out, void* workspace, size_t workspace_bytes,
-                       sq_stream stream) {
-  const char* fn = "sq_gemm_w8a8";
+namespace {
+sq_status gemm_call(const char* fn, const int8_t* xq, const int8_t* wq, int64_t M, int64_t N,
+                    int64_t K, const float* act_scale, int act_per_token, const float* w_scale,
+                    const float* bias, void* y, sq_dtype yt, int32_t* acc_out, void* workspace,
+                    size_t workspace_bytes, sq_stream stream) {
   g_last_error[0] = 0;
   SQ_TRY(check_dtype(yt, fn));
   if (M < 0 || N < 0) return fail(SQ_ERR_SHAPE, "%s: M=%lld N=%lld must be >= 0", fn,
@@ -223,6 +223,7 @@ sq_status sq_gemm_w8a8(const int8_t* xq, const int8_t* wq, int64_t M, int64_t N,
   SQ_REQ(w_scale, fn);
   SQ_REQ(y, fn);
   SQ_OPT(acc_out, fn);
+  SQ_OPT(bias, fn);
   const size_t need = gemm_workspace_bytes(M, N, K);
   if (need) {
     if (!workspace || workspace_bytes < need)
@@ -232,9 +233,26 @@ sq_status sq_gemm_w8a8(const int8_t* xq, const int8_t* wq, int64_t M, int64_t N,
   }
   GemmArgs a{};
   a.xq = xq; a.wq = wq; a.M = M; a.N = N; a.K = K; a.act_scale = act_scale;
-  a.act_per_token = act_per_token ? 1 : 0; a.w_scale = w_scale; a.y = y; a.yt = yt;
-  a.acc_out = acc_out; a.workspace = workspace; a.workspace_bytes = workspace_bytes;
+  a.act_per_token = act_per_token ? 1 : 0; a.w_scale = w_scale; a.bias = bias; a.y = y;
+  a.yt = yt; a.acc_out = acc_out; a.workspace = workspace; a.workspace_bytes = workspace_bytes;
   return launch_gemm(a, (cudaStream_t)stream);
+}
+}  // namespace
+
+sq_status sq_gemm_w8a8(const int8_t* xq, const int8_t* wq, int64_t M, int64_t N, int64_t K,
+                       const float* act_scale, int act_per_token, const float* w_scale, void* y,
+                       sq_dtype yt, int32_t* acc_out, void* workspace, size_t workspace_bytes,
+                       sq_stream stream) {
+  return gemm_call("sq_gemm_w8a8", xq, wq, M, N, K, act_scale, act_per_token, w_scale, nullptr,
+                   y, yt, acc_out, workspace, workspace_bytes, stream);
+}
+
+sq_status sq_gemm_w8a8_bias(const int8_t* xq, const int8_t* wq, int64_t M, int64_t N, int64_t K,
+                            const float* act_scale, int act_per_token, const float* w_scale,
+                            const float* bias, void* y, sq_dtype yt, int32_t* acc_out,
+                            void* workspace, size_t workspace_bytes, sq_stream stream) {
+  return gemm_call("sq_gemm_w8a8_bias", xq, wq, M, N, K, act_scale, act_per_token, w_scale, bias,
+                   y, yt, acc_out, workspace, workspace_bytes, stream);
 }
 
 sq_status sq_gemm_w8a8_noalloc(const int8_t* xq, const int8_t* wq, int64_t M, int64_t N,

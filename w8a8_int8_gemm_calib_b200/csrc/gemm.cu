@@ -72,6 +72,7 @@ struct Params {
   const float* act_scale;
   int per_token;
   const float* w_scale;
+  const float* bias;  // [N] added after the dequantization, or NULL
   void* y;
   int32_t* acc;
   unsigned int* status;
@@ -87,6 +88,27 @@ __device__ __forceinline__ void tile_coords(int tile, int m_tiles, int n_tiles, 
   nb = r / gm;
 }
 
+// 32 per-column values (scales or bias) starting at col0; 0 past N.
+__device__ __forceinline__ void load_cols32(const float* src, int col0, int N, float (&v)[32]) {
+  if (col0 + 32 <= N) {
+    const float4* s4 = reinterpret_cast<const float4*>(src + col0);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const float4 t = __ldg(s4 + i);
+      v[4 * i] = t.x; v[4 * i + 1] = t.y; v[4 * i + 2] = t.z; v[4 * i + 3] = t.w;
+    }
+  } else {
+#pragma unroll
+    for (int i = 0; i < 32; ++i) v[i] = col0 + i < N ? __ldg(src + col0 + i) : 0.0f;
+  }
+}
+
+// (float)acc * (as * ws); a bias is added after it as a separate fp32
+// rounding (the intrinsics are never fused into a multiply-add)
+__device__ __forceinline__ float dequant(uint32_t acc, float as, float ws) {
+  return __fmul_rn(__int2float_rn((int)acc), __fmul_rn(as, ws));
+}
+
 // Store 32 consecutive outputs of one row.  Fast path: 16-byte vector stores
 // when the whole chunk is in range and rows stay 16-byte aligned.
 template <bool BF16>
@@ -94,21 +116,16 @@ __device__ __forceinline__ void store_chunk(const Params& p, int row, int col0,
                                             const uint32_t (&r)[32], float as) {
   const bool full = col0 + 32 <= p.N;
   float ws[32];
-  if (full) {
-    const float4* w4 = reinterpret_cast<const float4*>(p.w_scale + col0);
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      const float4 v = __ldg(w4 + i);
-      ws[4 * i] = v.x; ws[4 * i + 1] = v.y; ws[4 * i + 2] = v.z; ws[4 * i + 3] = v.w;
-    }
-  } else {
-#pragma unroll
-    for (int i = 0; i < 32; ++i) ws[i] = col0 + i < p.N ? __ldg(p.w_scale + col0 + i) : 0.0f;
-  }
+  load_cols32(p.w_scale, col0, p.N, ws);
   float yv[32];
 #pragma unroll
-  for (int i = 0; i < 32; ++i)
-    yv[i] = __fmul_rn(__int2float_rn((int)r[i]), __fmul_rn(as, ws[i]));
+  for (int i = 0; i < 32; ++i) yv[i] = dequant(r[i], as, ws[i]);
+  if (p.bias) {
+    float bs[32];
+    load_cols32(p.bias, col0, p.N, bs);
+#pragma unroll
+    for (int i = 0; i < 32; ++i) yv[i] = __fadd_rn(yv[i], bs[i]);
+  }
   const size_t base = (size_t)row * (size_t)p.N + (size_t)col0;
   if (BF16) {
     __nv_bfloat16* y = reinterpret_cast<__nv_bfloat16*>(p.y) + base;
@@ -303,23 +320,24 @@ gemm_w8a8_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
           continue;
         }
         // dequantize this lane's 32 outputs (row `row`, columns col0..+31)
-        float ws[32];
-        if (col0 + 32 <= p.N) {
-          const float4* w4 = reinterpret_cast<const float4*>(p.w_scale + col0);
+        float yv[32];
+        {
+          float ws[32];
+          load_cols32(p.w_scale, col0, p.N, ws);
 #pragma unroll
-          for (int i = 0; i < 8; ++i) {
-            const float4 v = __ldg(w4 + i);
-            ws[4 * i] = v.x; ws[4 * i + 1] = v.y; ws[4 * i + 2] = v.z; ws[4 * i + 3] = v.w;
-          }
-        } else {
+          for (int i = 0; i < 32; ++i) yv[i] = dequant(r[i], as, ws[i]);
+        }
+        if (p.bias) {
+          float bs[32];
+          load_cols32(p.bias, col0, p.N, bs);
 #pragma unroll
-          for (int i = 0; i < 32; ++i) ws[i] = col0 + i < p.N ? __ldg(p.w_scale + col0 + i) : 0.0f;
+          for (int i = 0; i < 32; ++i) yv[i] = __fadd_rn(yv[i], bs[i]);
         }
         uint32_t wv[BF16 ? 16 : 32];
 #pragma unroll
         for (int i = 0; i < 32; i += 2) {
-          const float y0 = __fmul_rn(__int2float_rn((int)r[i]), __fmul_rn(as, ws[i]));
-          const float y1 = __fmul_rn(__int2float_rn((int)r[i + 1]), __fmul_rn(as, ws[i + 1]));
+          const float y0 = yv[i];
+          const float y1 = yv[i + 1];
           if (BF16) {
             __nv_bfloat162 t = __floats2bfloat162_rn(y0, y1);
             wv[i / 2] = *reinterpret_cast<uint32_t*>(&t);
@@ -410,6 +428,7 @@ struct SmallParams {
   const float* act_scale;
   int per_token;
   const float* w_scale;
+  const float* bias;  // [N] added after the dequantization, or NULL
   void* y;
   int32_t* acc;
   int32_t* slots;           // [grid][2][M][128]
@@ -437,12 +456,14 @@ template <bool BF16, int CH>
 __device__ __forceinline__ void small_store(const SmallParams& p, int n, int t0, const int32_t (&v)[CH]) {
   if (n >= p.N) return;
   const float ws = __ldg(p.w_scale + n);
+  const float bn = p.bias ? __ldg(p.bias + n) : 0.0f;
 #pragma unroll
   for (int i = 0; i < CH; ++i) {
     const int t = t0 + i;
     if (t < p.M) {
       const float as = __ldg(p.act_scale + (p.per_token ? t : 0));
-      const float y = __fmul_rn(__int2float_rn(v[i]), __fmul_rn(as, ws));
+      float y = dequant((uint32_t)v[i], as, ws);
+      if (p.bias) y = __fadd_rn(y, bn);
       const size_t o = (size_t)t * (size_t)p.N + (size_t)n;
       if (BF16) reinterpret_cast<__nv_bfloat16*>(p.y)[o] = __float2bfloat16_rn(y);
       else reinterpret_cast<float*>(p.y)[o] = y;
@@ -867,6 +888,7 @@ sq_status launch_gemm(const GemmArgs& a, cudaStream_t st) {
     p.act_scale = a.act_scale;
     p.per_token = a.act_per_token;
     p.w_scale = a.w_scale;
+    p.bias = a.bias;
     p.y = a.y;
     p.acc = a.acc_out;
     p.counters = reinterpret_cast<unsigned int*>(a.workspace);
@@ -893,6 +915,7 @@ sq_status launch_gemm(const GemmArgs& a, cudaStream_t st) {
   p.act_scale = a.act_scale;
   p.per_token = a.act_per_token;
   p.w_scale = a.w_scale;
+  p.bias = a.bias;
   p.y = a.y;
   p.acc = a.acc_out;
   p.status = sw;

@@ -72,6 +72,7 @@ struct GemmArgs {
   const float* act_scale;
   int act_per_token;
   const float* w_scale;
+  const float* bias;  // [N] or NULL
   void* y;
   sq_dtype yt;
   int32_t* acc_out;
