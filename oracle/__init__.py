@@ -75,6 +75,9 @@ def _declare(L):
     L.orc_f32_to_bf16.restype = ctypes.c_uint16
     L.orc_layernorm_row.argtypes = [_p, _i64, _p, _p, _f, _p]
     L.orc_calib_absmax.argtypes = [_p, _i, _i64, _i64, _p, _p, _f, _p]
+    L.orc_rmsnorm_row.argtypes = [_p, _i64, _p, _f, _p]
+    L.orc_calib_absmax_rms.argtypes = [_p, _i, _i64, _i64, _p, _f, _p]
+    L.orc_quant_act_rms.argtypes = [_p, _i, _i64, _i64, _p, _f, _i, _p, _p, _p]
     L.orc_weight_colmax.argtypes = [_p, _i, _i64, _i64, _p]
     L.orc_smooth_scales.argtypes = [_p, _p, _i64, _f, _p, _p]
     L.orc_static_delta.argtypes = [_p, _p, _i64]
@@ -86,7 +89,8 @@ def _declare(L):
                                 _p, _p, _p]
     for fn in ("orc_layernorm_row", "orc_calib_absmax", "orc_weight_colmax",
                "orc_smooth_scales", "orc_fuse_weights_q8", "orc_fold_ln",
-               "orc_quant_act", "orc_gemm_w8a8"):
+               "orc_quant_act", "orc_gemm_w8a8", "orc_rmsnorm_row",
+               "orc_calib_absmax_rms", "orc_quant_act_rms"):
         getattr(L, fn).restype = None
 
 
@@ -138,6 +142,42 @@ def layernorm_row(x, g, b, eps=1e-5):
     y = np.empty_like(x)
     lib().orc_layernorm_row(_ptr(x), x.size, _ptr(g), _ptr(b), eps, _ptr(y))
     return y
+
+
+def rmsnorm_row(x, g, eps=1e-5):
+    x, g = _f32(x), _f32(g)
+    y = np.empty_like(x)
+    lib().orc_rmsnorm_row(_ptr(x), x.size, _ptr(g), eps, _ptr(y))
+    return y
+
+
+def calib_absmax_rms(x, gamma, eps=1e-5, amax=None):
+    """S1 through an RMSNorm with the original gamma."""
+    x, xt = _typed(x)
+    T, K = x.shape
+    amax = np.zeros(K, np.float32) if amax is None else np.array(amax, np.float32)
+    gamma = _f32(gamma)
+    lib().orc_calib_absmax_rms(_ptr(x), xt, T, K, _ptr(gamma), eps, _ptr(amax))
+    return amax
+
+
+def quant_act_rms(x, gamma_s, eps=1e-5, per_token=True, static_delta=None,
+                  per_tensor_dynamic=False):
+    """S5 with y = RMSNorm(x; gamma_s): (xq, act_scale, n_clipped)."""
+    x, xt = _typed(x)
+    T, K = x.shape
+    gamma_s = _f32(gamma_s)
+    if per_tensor_dynamic:
+        act, gran = np.zeros(1, np.float32), PER_TENSOR_DYNAMIC
+    elif per_token:
+        act, gran = np.empty(T, np.float32), PER_TOKEN_DYNAMIC
+    else:
+        act, gran = np.array([static_delta], np.float32), PER_TENSOR_STATIC
+    xq = np.empty((T, K), np.int8)
+    ncl = ctypes.c_int64(0)
+    lib().orc_quant_act_rms(_ptr(x), xt, T, K, _ptr(gamma_s), eps, gran, _ptr(act),
+                            _ptr(xq), ctypes.addressof(ncl))
+    return xq, act, int(ncl.value)
 
 
 def calib_absmax(x, gamma=None, beta=None, eps=1e-5, amax=None):

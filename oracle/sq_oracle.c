@@ -140,29 +140,63 @@ void orc_layernorm_row(const float* x, int64_t K, const float* g,
   }
 }
 
+/* RMSNorm: the mean of squares in the same slot order (each slot's update
+ * is fmaf(x, x, p)), rstd = 1 / sqrtf(ms + eps), y = (x * rstd) * g. */
+void orc_rmsnorm_row(const float* x, int64_t K, const float* g, float eps,
+                     float* y) {
+  float kf = (float)K;
+  float ms = canonical_row_sum(x, K, 0.0f, 1) / kf;
+  float rstd = 1.0f / sqrtf(ms + eps);
+  for (int64_t k = 0; k < K; ++k) {
+    float n = x[k] * rstd;
+    y[k] = n * g[k];
+  }
+}
+
+/* The linear's input y of one row: the preceding norm's output, or the row
+ * times inv_s (NULL: the row itself). */
+static void row_output(const float* row, int64_t K, int norm, const float* g,
+                       const float* b, float eps, const float* inv_s, float* y) {
+  if (norm == ORC_NORM_LAYER) {
+    orc_layernorm_row(row, K, g, b, eps, y);
+  } else if (norm == ORC_NORM_RMS) {
+    orc_rmsnorm_row(row, K, g, eps, y);
+  } else {
+    for (int64_t k = 0; k < K; ++k) y[k] = inv_s ? row[k] * inv_s[k] : row[k];
+  }
+}
+
 /* ------------------------------------------------------------------ */
 /* S1: calibration absmax ([explainer] §四; [review] §5.3 eq. (4))      */
 /* ------------------------------------------------------------------ */
 
-void orc_calib_absmax(const void* x, int xtype, int64_t T, int64_t K,
-                      const float* gamma, const float* beta, float eps,
-                      float* amax) {
+static void calib_absmax(const void* x, int xtype, int64_t T, int64_t K,
+                         int norm, const float* gamma, const float* beta,
+                         float eps, float* amax) {
   float* row = (float*)malloc(sizeof(float) * (size_t)K);
   float* y = (float*)malloc(sizeof(float) * (size_t)K);
   for (int64_t t = 0; t < T; ++t) {
     for (int64_t k = 0; k < K; ++k) row[k] = load_elem(x, xtype, t * K + k);
-    const float* v = row;
-    if (gamma) {
-      orc_layernorm_row(row, K, gamma, beta, eps, y);
-      v = y;
-    }
+    row_output(row, K, norm, gamma, beta, eps, NULL, y);
     for (int64_t k = 0; k < K; ++k) {
-      float a = fabsf(v[k]);
+      float a = fabsf(y[k]);
       if (a > amax[k]) amax[k] = a;
     }
   }
   free(row);
   free(y);
+}
+
+void orc_calib_absmax(const void* x, int xtype, int64_t T, int64_t K,
+                      const float* gamma, const float* beta, float eps,
+                      float* amax) {
+  calib_absmax(x, xtype, T, K, gamma ? ORC_NORM_LAYER : ORC_NORM_NONE, gamma, beta,
+               eps, amax);
+}
+
+void orc_calib_absmax_rms(const void* x, int xtype, int64_t T, int64_t K,
+                          const float* gamma, float eps, float* amax) {
+  calib_absmax(x, xtype, T, K, ORC_NORM_RMS, gamma, NULL, eps, amax);
 }
 
 void orc_weight_colmax(const void* w, int wtype, int64_t N, int64_t K,
@@ -253,10 +287,10 @@ void orc_fold_ln(const float* gamma, const float* beta, const float* s,
 /* §2.6, §6.3)                                                         */
 /* ------------------------------------------------------------------ */
 
-void orc_quant_act(const void* x, int xtype, int64_t T, int64_t K,
-                   const float* gamma_s, const float* beta_s, float eps,
-                   const float* inv_s, int gran, float* act_scale,
-                   int8_t* xq, int64_t* n_clipped) {
+static void quant_act(const void* x, int xtype, int64_t T, int64_t K, int norm,
+                      const float* gamma_s, const float* beta_s, float eps,
+                      const float* inv_s, int gran, float* act_scale,
+                      int8_t* xq, int64_t* n_clipped) {
   float* row = (float*)malloc(sizeof(float) * (size_t)K);
   float* y = (float*)malloc(sizeof(float) * (size_t)K);
   float static_inv = 0.0f;
@@ -265,11 +299,7 @@ void orc_quant_act(const void* x, int xtype, int64_t T, int64_t K,
     float m = 0.0f;
     for (int64_t t = 0; t < T; ++t) {
       for (int64_t k = 0; k < K; ++k) row[k] = load_elem(x, xtype, t * K + k);
-      if (gamma_s) {
-        orc_layernorm_row(row, K, gamma_s, beta_s, eps, y);
-      } else {
-        for (int64_t k = 0; k < K; ++k) y[k] = inv_s ? row[k] * inv_s[k] : row[k];
-      }
+      row_output(row, K, norm, gamma_s, beta_s, eps, inv_s, y);
       for (int64_t k = 0; k < K; ++k) {
         float a = fabsf(y[k]);
         if (a > m) m = a;
@@ -280,11 +310,7 @@ void orc_quant_act(const void* x, int xtype, int64_t T, int64_t K,
   if (gran != ORC_PER_TOKEN_DYNAMIC) static_inv = 1.0f / act_scale[0];
   for (int64_t t = 0; t < T; ++t) {
     for (int64_t k = 0; k < K; ++k) row[k] = load_elem(x, xtype, t * K + k);
-    if (gamma_s) {
-      orc_layernorm_row(row, K, gamma_s, beta_s, eps, y);
-    } else {
-      for (int64_t k = 0; k < K; ++k) y[k] = inv_s ? row[k] * inv_s[k] : row[k];
-    }
+    row_output(row, K, norm, gamma_s, beta_s, eps, inv_s, y);
     float inv;
     if (gran == ORC_PER_TOKEN_DYNAMIC) {
       float m = 0.0f;
@@ -302,6 +328,21 @@ void orc_quant_act(const void* x, int xtype, int64_t T, int64_t K,
   }
   free(row);
   free(y);
+}
+
+void orc_quant_act(const void* x, int xtype, int64_t T, int64_t K,
+                   const float* gamma_s, const float* beta_s, float eps,
+                   const float* inv_s, int gran, float* act_scale,
+                   int8_t* xq, int64_t* n_clipped) {
+  quant_act(x, xtype, T, K, gamma_s ? ORC_NORM_LAYER : ORC_NORM_NONE, gamma_s, beta_s,
+            eps, inv_s, gran, act_scale, xq, n_clipped);
+}
+
+void orc_quant_act_rms(const void* x, int xtype, int64_t T, int64_t K,
+                       const float* gamma_s, float eps, int gran,
+                       float* act_scale, int8_t* xq, int64_t* n_clipped) {
+  quant_act(x, xtype, T, K, ORC_NORM_RMS, gamma_s, NULL, eps, NULL, gran, act_scale, xq,
+            n_clipped);
 }
 
 /* ------------------------------------------------------------------ */

@@ -43,6 +43,7 @@ extern "C" {
 enum { ORC_F32 = 0, ORC_BF16 = 1 };
 /* Activation granularity ([review] §2.5, §2.6 Fig. 3, §6.3 O1/O3). */
 enum { ORC_PER_TENSOR_STATIC = 0, ORC_PER_TOKEN_DYNAMIC = 1, ORC_PER_TENSOR_DYNAMIC = 2 };
+enum { ORC_NORM_NONE = 0, ORC_NORM_LAYER = 1, ORC_NORM_RMS = 2 };
 
 /* Quantization step of the symmetric INT8 quantizer ([review] §2.2):
  * delta = max(amax, 1e-7) / 127, in fp32. */
@@ -83,6 +84,23 @@ float orc_static_delta(const float* amax_x, const float* s, int64_t K);
 /* S4: W_hat = W * s (per input channel); per-output-channel symmetric INT8. */
 void orc_fuse_weights_q8(const void* w, int wtype, int64_t N, int64_t K,
                          const float* s, int8_t* wq, float* w_scale);
+
+/* RMSNorm (the norm of models without a LayerNorm mean or beta): the mean
+ * of squares in the LayerNorm's slot order, each slot updated by
+ * fmaf(x, x, p); ms = sum / K; rstd = 1 / sqrtf(ms + eps);
+ * y = (x * rstd) * g.  Its smoothing fold is g' = g / s (no beta). */
+void orc_rmsnorm_row(const float* x, int64_t K, const float* g, float eps,
+                     float* y);
+
+/* S1 through an RMSNorm with the original gamma. */
+void orc_calib_absmax_rms(const void* x, int xtype, int64_t T, int64_t K,
+                          const float* gamma, float eps, float* amax);
+
+/* S5 with y = RMSNorm'(x) (gamma_s = gamma / s); granularities as
+ * orc_quant_act. */
+void orc_quant_act_rms(const void* x, int xtype, int64_t T, int64_t K,
+                       const float* gamma_s, float eps, int gran,
+                       float* act_scale, int8_t* xq, int64_t* n_clipped);
 
 /* S4: LayerNorm fold gamma' = gamma / s, beta' = beta / s ([embedded] §二). */
 void orc_fold_ln(const float* gamma, const float* beta, const float* s,

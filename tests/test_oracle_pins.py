@@ -458,6 +458,52 @@ def test_layernorm_exact_on_integer_rows(orc):
     assert np.array_equal(y, (x * rstd).astype(np.float32))
 
 
+def test_rmsnorm_matches_fp64(orc):
+    """Canonical-order RMSNorm against an fp64 RMSNorm (the norm of models
+    whose smoothing fold is gamma / s alone)."""
+    r = np.random.default_rng(12)
+    for K in (16, 48, 1040, 4096, 5120):
+        x = r.standard_normal(K).astype(np.float32)
+        x[r.integers(0, K, 3)] *= 80
+        g = (1 + 0.1 * r.standard_normal(K)).astype(np.float32)
+        y = orc.rmsnorm_row(x, g)
+        x64 = x.astype(np.float64)
+        ref = x64 / np.sqrt((x64 ** 2).mean() + 1e-5) * g
+        assert np.max(np.abs(y - ref)) <= 1e-5 * max(1.0, np.abs(ref).max())
+
+
+def test_rmsnorm_exact_closed_form(orc):
+    """Rows of +-2 with eps = 0: the mean of squares is exactly 4 in any
+    order, rstd = 1/2 exactly, so y = +-gamma exactly; a mean term (the
+    LayerNorm's) would make the +-2 pattern with a non-zero mean differ."""
+    K = 1024
+    r = np.random.default_rng(13)
+    x = np.where(r.random(K) < 0.7, 2.0, -2.0).astype(np.float32)
+    g = (1 + 0.1 * r.standard_normal(K)).astype(np.float32)
+    y = orc.rmsnorm_row(x, g, eps=0.0)
+    assert np.array_equal(y, np.where(x > 0, g, -g).astype(np.float32))
+    assert not np.array_equal(orc.layernorm_row(x, g, None, eps=0.0), y)
+
+
+def test_rmsnorm_fold_alpha_one(orc):
+    """Calibration through the RMSNorm, alpha = 1 (s = the peaks), the fold
+    gamma' = gamma / s: the smoothed calibration peaks are 1 within 2 ulp
+    (y' = ((x * rstd) * gamma) / s against (x * rstd) * (gamma / s)), and the
+    quantizer's per-token path equals its per-tensor-dynamic path on one row."""
+    lin = synth.workloads()["tiny_k1024"].linears[0]
+    d = synth.make_linear_inputs(lin, T=16, T_cal=64, N=8)
+    g = (1 + 0.1 * np.random.default_rng(14).standard_normal(1024)).astype(np.float32)
+    amax = orc.calib_absmax_rms(d["x_cal"], g)
+    s, _ = orc.smooth_scales(amax, np.ones(1024, np.float32), 1.0)
+    assert np.array_equal(s, np.maximum(amax, np.float32(1e-4)))
+    g2 = (g / s).astype(np.float32)
+    peak = orc.calib_absmax_rms(d["x_cal"], g2)
+    assert max(ulps(p, 1.0) for p in peak) <= 2
+    xq1, a1, _ = orc.quant_act_rms(d["x"][3:4], g2, per_token=True)
+    xq2, a2, _ = orc.quant_act_rms(d["x"][3:4], g2, per_tensor_dynamic=True)
+    assert a1[0] == a2[0] and np.array_equal(xq1, xq2)
+
+
 def test_calib_absmax_running_and_library(orc):
     """S1 raw mode equals numpy's max(|X|) over tokens, and a running max
     over two batches equals the max over their concatenation."""
