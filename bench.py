@@ -356,7 +356,8 @@ def run_ours(args):
     e2e = run_e2e(sq, torch, layer, lin, d, dev, args.e2e_steps, world, barrier)
     small_m = None if args.no_small_m else run_small_m(sq, torch, dev, flush)
     next_rows = {"o2_per_tensor_dynamic_quant": run_o2(sq, torch, layer, lin, flush),
-                 "gemm_bias_epilogue": run_gemm_bias(sq, torch, layer, lin, flush)}
+                 "gemm_bias_epilogue": run_gemm_bias(sq, torch, layer, lin, flush),
+                 "rmsnorm_quant_per_token": run_rms_quant(sq, torch, layer, lin, flush)}
 
     peaks, peak_kind = load_peaks()
     bf16_peak = peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"])
@@ -504,6 +505,46 @@ def run_o2(sq, torch, layer, lin, flush, reps=20):
             "kernels": "peak pass, step, static quantizer pass (x read twice)",
             "us": round(ms * 1e3, 2), "gbs": round(gbs, 1), "hbm_frac": round(gbs / hbm, 3),
             "bytes": int(nbytes)}
+
+
+def time_call(torch, call, flush, reps=20):
+    """Mean device time (ms) of one call: a CUDA-graph replay per call after
+    an L2 flush, device events around it."""
+    for _ in range(3):
+        call()
+    e0 = torch.cuda.Event(enable_timing=True, external=True)
+    e1 = torch.cuda.Event(enable_timing=True, external=True)
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        e0.record()
+        call()
+        e1.record()
+    times = []
+    for i in range(reps):
+        flush(i)
+        graph.replay()
+        torch.cuda.synchronize()
+        times.append(e0.elapsed_time(e1))
+    del graph
+    return statistics.mean(times)
+
+
+def run_rms_quant(sq, torch, layer, lin, flush):
+    """The quantizer behind an RMSNorm (gamma / s folded, no beta; NEXT-3) on
+    the step's activations, per-token; GB/s over x read once + codes and
+    scales written once."""
+    M, K = lin.T, lin.K
+    b = 2 if lin.dtype == "bf16" else 4
+    gs = layer.g2 if layer.g2 is not None else layer.inv_s
+    act = torch.empty(M, dtype=torch.float32, device=layer.x.device)
+    ms = time_call(torch, lambda: sq.sq_rms_smooth_quant_act(layer.x, layer.xq, act, gs),
+                   flush)
+    sq.sq_sync_status()
+    nbytes = M * K * b + M * K + 4 * M + 4 * K
+    hbm = load_peaks()[0].get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"])
+    gbs = nbytes / (ms * 1e-3) / 1e9
+    return {"shape": f"{M}x{K} {lin.dtype}", "us": round(ms * 1e3, 2), "gbs": round(gbs, 1),
+            "hbm_frac": round(gbs / hbm, 3), "bytes": int(nbytes)}
 
 
 def run_gemm_bias(sq, torch, layer, lin, flush, reps=20):

@@ -105,6 +105,23 @@ sq_status sq_calib_absmax(const void* x, sq_dtype xt, int64_t T, int64_t K,
                           float ln_eps, float* amax, sq_stream stream);
 
 /*
+ * sq_calib_absmax_rms -- sq_calib_absmax through an RMSNorm instead of a
+ * LayerNorm (the norm of models whose smoothing fold is gamma / s alone:
+ * the fold of [embedded] §二 without a beta; the pages define no RMSNorm, so
+ * the reduction order below is this library's):
+ *
+ *   ms = mean_k x[t,k]^2 in the LayerNorm's slot order (each slot updated by
+ *        one fused multiply-add), rstd = 1 / sqrt(ms + eps),
+ *   amax[k] = max(amax[k], max_t |(x[t,k] * rstd) * gamma[k]|).
+ *
+ *   gamma [K] fp32 (required); eps finite, >= 0.  Arguments, layouts and
+ *   errors otherwise as sq_calib_absmax.
+ */
+sq_status sq_calib_absmax_rms(const void* x, sq_dtype xt, int64_t T, int64_t K,
+                              const float* gamma, float eps, float* amax,
+                              sq_stream stream);
+
+/*
  * sq_smooth_scales -- smoothing factors of eq. (4) ([review] §5.3;
  * [explainer] §三):
  *
@@ -175,6 +192,24 @@ sq_status sq_ln_smooth_quant_act(const void* x, sq_dtype xt, int64_t T,
                                  const float* inv_s, sq_act_gran gran,
                                  float* act_scale, int8_t* xq,
                                  int64_t* n_clipped, sq_stream stream);
+
+/*
+ * sq_rms_smooth_quant_act -- the runtime quantizer behind an RMSNorm whose
+ * gamma carries the folded 1/s (gamma_s = gamma / s, from
+ * sq_fuse_weights_q8 with beta NULL):
+ *
+ *   y[t,k] = (x[t,k] * rstd_t) * gamma_s[k]   (rstd as sq_calib_absmax_rms)
+ *
+ * then quantized at granularity gran exactly as sq_ln_smooth_quant_act
+ * (per-token dynamic, per-tensor static, per-tensor dynamic).  gamma_s [K]
+ * fp32 (required).  Arguments, layouts and errors otherwise as
+ * sq_ln_smooth_quant_act.
+ */
+sq_status sq_rms_smooth_quant_act(const void* x, sq_dtype xt, int64_t T,
+                                  int64_t K, const float* gamma_s, float eps,
+                                  sq_act_gran gran, float* act_scale,
+                                  int8_t* xq, int64_t* n_clipped,
+                                  sq_stream stream);
 
 /*
  * sq_gemm_workspace_bytes -- device scratch sq_gemm_w8a8 needs for this

@@ -106,6 +106,23 @@ def test_quant_act_checks(lib):
     assert lib.SQ_ACT_PER_TENSOR_DYNAMIC == 2
 
 
+def test_rmsnorm_checks(lib):
+    L = lib.lib
+    # gamma is required; eps finite and >= 0; the rest as the LayerNorm calls
+    assert L.sq_calib_absmax_rms(A, 1, 4, 16, None, 1e-5, A2, None) == lib.SQ_ERR_INVALID_ARG
+    assert L.sq_calib_absmax_rms(A, 1, 4, 16, A2, -1.0, A2, None) == lib.SQ_ERR_INVALID_ARG
+    assert L.sq_calib_absmax_rms(A, 1, 4, 24, A2, 1e-5, A2, None) == lib.SQ_ERR_SHAPE
+    assert L.sq_calib_absmax_rms(A, 1, 0, 16, A2, 1e-5, A2, None) == lib.SQ_OK
+    assert L.sq_rms_smooth_quant_act(A, 1, 4, 16, None, 1e-5, 1, A2, A2, None, None) == \
+        lib.SQ_ERR_INVALID_ARG
+    assert "sq_rms_smooth_quant_act" in lib.last_error()
+    assert L.sq_rms_smooth_quant_act(A, 1, 4, 16, A2, 1e-5, 7, A2, A2, None, None) == \
+        lib.SQ_ERR_INVALID_ARG
+    assert L.sq_rms_smooth_quant_act(A, 1, 4, 16, MIS, 1e-5, 1, A2, A2, None, None) == \
+        lib.SQ_ERR_ALIGN
+    assert L.sq_rms_smooth_quant_act(A, 1, 0, 16, A2, 1e-5, 2, A2, A2, None, None) == lib.SQ_OK
+
+
 def test_gemm_bias_checks(lib):
     L = lib.lib
     assert L.sq_gemm_w8a8_bias(A, A, 4, 4, 16, A2, 1, A2, MIS, A2, 1, None, None, 0, None) == \

@@ -24,6 +24,7 @@ __all__ = [
     "sq_calib_absmax", "sq_smooth_scales", "sq_fuse_weights_q8",
     "sq_ln_smooth_quant_act", "sq_gemm_workspace_bytes", "sq_gemm_w8a8",
     "sq_sync_status", "sq_selftest_bounded_wait", "SQError", "Workspace",
+    "sq_calib_absmax_rms", "sq_rms_smooth_quant_act",
 ]
 
 
@@ -54,6 +55,14 @@ def sq_calib_absmax(x, amax, ln_gamma=None, ln_beta=None, ln_eps=1e-5, stream=No
     T, K = x.shape
     check(lib.sq_calib_absmax(_ptr(x), _dt(x), T, K, _ptr(ln_gamma), _ptr(ln_beta),
                               ln_eps, _ptr(amax), _stream(stream)), "sq_calib_absmax")
+    return amax
+
+
+def sq_calib_absmax_rms(x, amax, gamma, eps=1e-5, stream=None):
+    """Running per-input-channel peak of RMSNorm(X; gamma) over tokens."""
+    T, K = x.shape
+    check(lib.sq_calib_absmax_rms(_ptr(x), _dt(x), T, K, _ptr(gamma), eps, _ptr(amax),
+                                  _stream(stream)), "sq_calib_absmax_rms")
     return amax
 
 
@@ -91,6 +100,21 @@ def sq_ln_smooth_quant_act(x, xq, act_scale, gamma_s=None, beta_s=None, ln_eps=1
                                      ln_eps, _ptr(inv_s), gran, _ptr(act_scale), _ptr(xq),
                                      _ptr(n_clipped), _stream(stream)),
           "sq_ln_smooth_quant_act")
+    return xq, act_scale
+
+
+def sq_rms_smooth_quant_act(x, xq, act_scale, gamma_s, eps=1e-5, per_token=True,
+                            n_clipped=None, stream=None, per_tensor_dynamic=False):
+    """RMSNorm (gamma_s = gamma / s) + symmetric INT8 quantizer -> xq (and
+    act_scale), granularities as sq_ln_smooth_quant_act."""
+    T, K = x.shape
+    if per_tensor_dynamic:
+        gran = SQ_ACT_PER_TENSOR_DYNAMIC
+    else:
+        gran = SQ_ACT_PER_TOKEN_DYNAMIC if per_token else SQ_ACT_PER_TENSOR_STATIC
+    check(lib.sq_rms_smooth_quant_act(_ptr(x), _dt(x), T, K, _ptr(gamma_s), eps, gran,
+                                      _ptr(act_scale), _ptr(xq), _ptr(n_clipped),
+                                      _stream(stream)), "sq_rms_smooth_quant_act")
     return xq, act_scale
 
 

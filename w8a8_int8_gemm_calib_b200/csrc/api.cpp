@@ -65,21 +65,22 @@ using namespace sq;
 
 extern "C" {
 
-sq_status sq_calib_absmax(const void* x, sq_dtype xt, int64_t T, int64_t K,
-                          const float* ln_gamma, const float* ln_beta, float ln_eps,
-                          float* amax, sq_stream stream) {
-  const char* fn = "sq_calib_absmax";
+namespace {
+sq_status calib_call(const char* fn, const void* x, sq_dtype xt, int64_t T, int64_t K,
+                     const float* ln_gamma, const float* ln_beta, float ln_eps, int rms,
+                     float* amax, sq_stream stream) {
   g_last_error[0] = 0;
   SQ_TRY(check_dtype(xt, fn));
   if (T < 0) return fail(SQ_ERR_SHAPE, "%s: T=%lld < 0", fn, (long long)T);
   SQ_TRY(check_k(K, fn));
   SQ_REQ(x, fn);
   SQ_REQ(amax, fn);
+  if (rms) SQ_REQ(ln_gamma, fn);
   SQ_OPT(ln_gamma, fn);
   SQ_OPT(ln_beta, fn);
   if (ln_beta && !ln_gamma) return fail(SQ_ERR_INVALID_ARG, "%s: ln_beta given without ln_gamma", fn);
   if (ln_gamma && !(ln_eps >= 0.0f && isfinite(ln_eps)))
-    return fail(SQ_ERR_INVALID_ARG, "%s: ln_eps must be finite and >= 0", fn);
+    return fail(SQ_ERR_INVALID_ARG, "%s: eps must be finite and >= 0", fn);
   if (T == 0) return SQ_OK;
   cudaStream_t st = (cudaStream_t)stream;
   cudaError_t e;
@@ -87,11 +88,23 @@ sq_status sq_calib_absmax(const void* x, sq_dtype xt, int64_t T, int64_t K,
     e = launch_colmax(x, xt, T, K, amax, st);
   } else {
     RowArgs a{};
-    a.x = x; a.T = T; a.K = K; a.g = ln_gamma; a.b = ln_beta; a.eps = ln_eps;
+    a.x = x; a.T = T; a.K = K; a.g = ln_gamma; a.b = ln_beta; a.eps = ln_eps; a.rms = rms;
     a.colmax = amax;
     e = launch_row(a, xt, ROW_COLMAX, st);
   }
   return e == cudaSuccess ? SQ_OK : cuda_fail(e, fn);
+}
+}  // namespace
+
+sq_status sq_calib_absmax(const void* x, sq_dtype xt, int64_t T, int64_t K,
+                          const float* ln_gamma, const float* ln_beta, float ln_eps,
+                          float* amax, sq_stream stream) {
+  return calib_call("sq_calib_absmax", x, xt, T, K, ln_gamma, ln_beta, ln_eps, 0, amax, stream);
+}
+
+sq_status sq_calib_absmax_rms(const void* x, sq_dtype xt, int64_t T, int64_t K,
+                              const float* gamma, float eps, float* amax, sq_stream stream) {
+  return calib_call("sq_calib_absmax_rms", x, xt, T, K, gamma, nullptr, eps, 1, amax, stream);
 }
 
 sq_status sq_smooth_scales(const float* amax_x, const void* w, sq_dtype wt, int64_t N, int64_t K,
@@ -151,11 +164,11 @@ sq_status sq_fuse_weights_q8(const void* w, sq_dtype wt, int64_t N, int64_t K, c
   return e == cudaSuccess ? SQ_OK : cuda_fail(e, fn);
 }
 
-sq_status sq_ln_smooth_quant_act(const void* x, sq_dtype xt, int64_t T, int64_t K,
-                                 const float* gamma_s, const float* beta_s, float ln_eps,
-                                 const float* inv_s, sq_act_gran gran, float* act_scale,
-                                 int8_t* xq, int64_t* n_clipped, sq_stream stream) {
-  const char* fn = "sq_ln_smooth_quant_act";
+namespace {
+sq_status quant_call(const char* fn, const void* x, sq_dtype xt, int64_t T, int64_t K,
+                     const float* gamma_s, const float* beta_s, float ln_eps, int rms,
+                     const float* inv_s, sq_act_gran gran, float* act_scale, int8_t* xq,
+                     int64_t* n_clipped, sq_stream stream) {
   g_last_error[0] = 0;
   SQ_TRY(check_dtype(xt, fn));
   if (gran != SQ_ACT_PER_TENSOR_STATIC && gran != SQ_ACT_PER_TOKEN_DYNAMIC &&
@@ -166,6 +179,7 @@ sq_status sq_ln_smooth_quant_act(const void* x, sq_dtype xt, int64_t T, int64_t 
   SQ_REQ(x, fn);
   SQ_REQ(xq, fn);
   SQ_REQ(act_scale, fn);
+  if (rms) SQ_REQ(gamma_s, fn);
   SQ_OPT(gamma_s, fn);
   SQ_OPT(beta_s, fn);
   SQ_OPT(inv_s, fn);
@@ -175,10 +189,11 @@ sq_status sq_ln_smooth_quant_act(const void* x, sq_dtype xt, int64_t T, int64_t 
   if (gamma_s && inv_s)
     return fail(SQ_ERR_INVALID_ARG, "%s: inv_s is folded into gamma_s/beta_s when a LayerNorm precedes; pass one of them", fn);
   if (gamma_s && !(ln_eps >= 0.0f && isfinite(ln_eps)))
-    return fail(SQ_ERR_INVALID_ARG, "%s: ln_eps must be finite and >= 0", fn);
+    return fail(SQ_ERR_INVALID_ARG, "%s: eps must be finite and >= 0", fn);
   if (T == 0) return SQ_OK;
   RowArgs a{};
-  a.x = x; a.T = T; a.K = K; a.g = gamma_s; a.b = beta_s; a.eps = ln_eps; a.mul = inv_s;
+  a.x = x; a.T = T; a.K = K; a.g = gamma_s; a.b = beta_s; a.eps = ln_eps; a.rms = rms;
+  a.mul = inv_s;
   a.scale = act_scale; a.q = xq; a.n_clipped = (unsigned long long*)n_clipped;
   const cudaStream_t st = (cudaStream_t)stream;
   cudaError_t e;
@@ -197,6 +212,23 @@ sq_status sq_ln_smooth_quant_act(const void* x, sq_dtype xt, int64_t T, int64_t 
     e = launch_row(a, xt, gran == SQ_ACT_PER_TOKEN_DYNAMIC ? ROW_DYNAMIC : ROW_STATIC, st);
   }
   return e == cudaSuccess ? SQ_OK : cuda_fail(e, fn);
+}
+}  // namespace
+
+sq_status sq_ln_smooth_quant_act(const void* x, sq_dtype xt, int64_t T, int64_t K,
+                                 const float* gamma_s, const float* beta_s, float ln_eps,
+                                 const float* inv_s, sq_act_gran gran, float* act_scale,
+                                 int8_t* xq, int64_t* n_clipped, sq_stream stream) {
+  return quant_call("sq_ln_smooth_quant_act", x, xt, T, K, gamma_s, beta_s, ln_eps, 0, inv_s,
+                    gran, act_scale, xq, n_clipped, stream);
+}
+
+sq_status sq_rms_smooth_quant_act(const void* x, sq_dtype xt, int64_t T, int64_t K,
+                                  const float* gamma_s, float eps, sq_act_gran gran,
+                                  float* act_scale, int8_t* xq, int64_t* n_clipped,
+                                  sq_stream stream) {
+  return quant_call("sq_rms_smooth_quant_act", x, xt, T, K, gamma_s, nullptr, eps, 1, nullptr,
+                    gran, act_scale, xq, n_clipped, stream);
 }
 
 size_t sq_gemm_workspace_bytes(int64_t M, int64_t N, int64_t K) {

@@ -298,17 +298,19 @@ row_kernel(RowArgs a) {
 
     float mu = 0.0f, rstd = 0.0f;
     if constexpr (LN) {
-      float p = 0.0f;
-      for_chunks<MAXC>(cur, xr, j, nchunk, [&](int, int64_t, const float (&v)[8]) {
+      if (!a.rms) {  // RMSNorm: no mean (mu = 0, beta NULL)
+        float p = 0.0f;
+        for_chunks<MAXC>(cur, xr, j, nchunk, [&](int, int64_t, const float (&v)[8]) {
 #pragma unroll
-        for (int e = 0; e < 8; ++e) p = __fadd_rn(p, v[e]);
-      });
-      p = warp_sum_butterfly(p);
-      if (lane == 0) red[slice][parity][0][w] = p;
-      slice_bar(slice);
-      const float s0 = __fadd_rn(__fadd_rn(red[slice][parity][0][0], red[slice][parity][0][2]),
-                                 __fadd_rn(red[slice][parity][0][1], red[slice][parity][0][3]));
-      mu = __fdiv_rn(s0, kf);
+          for (int e = 0; e < 8; ++e) p = __fadd_rn(p, v[e]);
+        });
+        p = warp_sum_butterfly(p);
+        if (lane == 0) red[slice][parity][0][w] = p;
+        slice_bar(slice);
+        const float s0 = __fadd_rn(__fadd_rn(red[slice][parity][0][0], red[slice][parity][0][2]),
+                                   __fadd_rn(red[slice][parity][0][1], red[slice][parity][0][3]));
+        mu = __fdiv_rn(s0, kf);
+      }
       float q = 0.0f;
       for_chunks<MAXC>(cur, xr, j, nchunk, [&](int, int64_t, const float (&v)[8]) {
 #pragma unroll

@@ -494,16 +494,21 @@ __global__ void __launch_bounds__(kThreads, NB) rowpipe_kernel(const Pipe P) {
 
       if constexpr (LN) {
         float p[G];
+        // RMSNorm has no mean: mu = 0 makes x - mu = x below, the variance
+        // pass the mean of squares, and y = ((x * rstd) * g) + 0 (beta NULL)
+        float mu = 0.0f;
+        if (!a.rms) {
 #pragma unroll
-        for (int g = 0; g < G; ++g) p[g] = 0.0f;
-        for_level(0, [&](int m, int, float2 (&x)[4]) {
+          for (int g = 0; g < G; ++g) p[g] = 0.0f;
+          for_level(0, [&](int m, int, float2 (&x)[4]) {
 #pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            p[m % G] = __fadd_rn(p[m % G], x[e].x);
-            p[m % G] = __fadd_rn(p[m % G], x[e].y);
-          }
-        });
-        const float mu = __fdiv_rn(slot_sum(p, 0), kf);
+            for (int e = 0; e < 4; ++e) {
+              p[m % G] = __fadd_rn(p[m % G], x[e].x);
+              p[m % G] = __fadd_rn(p[m % G], x[e].y);
+            }
+          });
+          mu = __fdiv_rn(slot_sum(p, 0), kf);
+        }
         negmu2 = make_float2(-mu, -mu);
 #pragma unroll
         for (int g = 0; g < G; ++g) p[g] = 0.0f;

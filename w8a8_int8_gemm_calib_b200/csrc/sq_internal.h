@@ -35,6 +35,7 @@ struct RowArgs {
   const float* g;      // LayerNorm gamma (NULL: no LayerNorm)
   const float* b;      // LayerNorm beta (may be NULL)
   float eps;
+  int rms;             // with g: RMSNorm (no mean; b must be NULL) instead of LayerNorm
   const float* mul;    // per-column multiplier when there is no LayerNorm (may be NULL)
   float* scale;        // ROW_DYNAMIC: out [T]; ROW_STATIC: in [1]
   int8_t* q;           // [T,K] codes out (quantizing modes)
