@@ -84,13 +84,14 @@ def _declare(L):
     L.orc_static_delta.restype = _f
     L.orc_fuse_weights_q8.argtypes = [_p, _i, _i64, _i64, _p, _p, _p]
     L.orc_fold_ln.argtypes = [_p, _p, _p, _i64, _p, _p]
+    L.orc_fold_into_producer.argtypes = [_p, _i64, _p, _p]
     L.orc_quant_act.argtypes = [_p, _i, _i64, _i64, _p, _p, _f, _p, _i, _p, _p, _p]
     L.orc_gemm_w8a8.argtypes = [_p, _p, _i64, _i64, _i64, _p, _i, _p, _p, _p, _i64,
                                 _p, _p, _p]
     for fn in ("orc_layernorm_row", "orc_calib_absmax", "orc_weight_colmax",
                "orc_smooth_scales", "orc_fuse_weights_q8", "orc_fold_ln",
                "orc_quant_act", "orc_gemm_w8a8", "orc_rmsnorm_row",
-               "orc_calib_absmax_rms", "orc_quant_act_rms"):
+               "orc_calib_absmax_rms", "orc_quant_act_rms", "orc_fold_into_producer"):
         getattr(L, fn).restype = None
 
 
@@ -223,6 +224,15 @@ def fuse_weights_q8(w, s):
     ws = np.empty(N, np.float32)
     lib().orc_fuse_weights_q8(_ptr(w), wt, N, K, _ptr(s), _ptr(wq), _ptr(ws))
     return wq, ws
+
+
+def fold_into_producer(s, w_scale, bias=None):
+    """The producer's per-output-channel scale (and bias) divided by s."""
+    s = _f32(s)
+    ws = np.array(w_scale, np.float32)
+    b = None if bias is None else np.array(bias, np.float32)
+    lib().orc_fold_into_producer(_ptr(s), s.size, _ptr(ws), _ptr(b))
+    return ws, b
 
 
 def fold_ln(gamma, beta, s):

@@ -274,6 +274,13 @@ void orc_fuse_weights_q8(const void* w, int wtype, int64_t N, int64_t K,
   free(what);
 }
 
+void orc_fold_into_producer(const float* s, int64_t K, float* w_scale, float* bias) {
+  for (int64_t k = 0; k < K; ++k) {
+    w_scale[k] = w_scale[k] / s[k];
+    if (bias) bias[k] = bias[k] / s[k];
+  }
+}
+
 void orc_fold_ln(const float* gamma, const float* beta, const float* s,
                  int64_t K, float* gamma_out, float* beta_out) {
   for (int64_t k = 0; k < K; ++k) {

@@ -102,6 +102,14 @@ void orc_quant_act_rms(const void* x, int xtype, int64_t T, int64_t K,
                        const float* gamma_s, float eps, int gran,
                        float* act_scale, int8_t* xq, int64_t* n_clipped);
 
+/* The fold into a producing linear ([review] §5.5: s folds into the
+ * previous layer's parameters): the producer's output channel k feeds the
+ * consumer's input channel k, so its per-output-channel scale and bias are
+ * divided by s_k (one fp32 division each): w_scale[k] /= s[k],
+ * bias[k] /= s[k] (bias may be NULL).  With s > 0 a ReLU between the two
+ * commutes with the division. */
+void orc_fold_into_producer(const float* s, int64_t K, float* w_scale, float* bias);
+
 /* S4: LayerNorm fold gamma' = gamma / s, beta' = beta / s ([embedded] §二). */
 void orc_fold_ln(const float* gamma, const float* beta, const float* s,
                  int64_t K, float* gamma_out, float* beta_out);

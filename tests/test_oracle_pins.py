@@ -504,6 +504,43 @@ def test_rmsnorm_fold_alpha_one(orc):
     assert a1[0] == a2[0] and np.array_equal(xq1, xq2)
 
 
+def test_fold_into_producer(orc):
+    """Folding 1/s into the producing linear ([review] §5.5): with
+    power-of-two s the divisions are exact; on general data the producer's
+    output with the folded scale and bias equals its original output divided
+    by s within 2 ulp (fp64 reference), a ReLU in between commutes (s > 0),
+    and the consumer then needs no 1/s: quantizing the folded output with
+    inv_s NULL equals quantizing the original output times 1/s on all but
+    last-bit ties."""
+    r = np.random.default_rng(31)
+    K = 64
+    s2 = (2.0 ** r.integers(-6, 7, K)).astype(np.float32)
+    ws = r.uniform(1e-4, 1e-2, K).astype(np.float32)
+    b = r.normal(0, 0.5, K).astype(np.float32)
+    ws2, b2 = orc.fold_into_producer(s2, ws, b)
+    assert np.array_equal(ws2, ws / s2) and np.array_equal(b2, b / s2)
+    # producer: M x Kp -> K outputs (its output channels = consumer inputs)
+    M, Kp = 24, 96
+    xq = r.integers(-127, 128, (M, Kp)).astype(np.int8)
+    wq = r.integers(-127, 128, (K, Kp)).astype(np.int8)
+    act = r.uniform(1e-3, 1e-1, M).astype(np.float32)
+    s = r.uniform(0.05, 20.0, K).astype(np.float32)
+    y, acc = orc.gemm_w8a8(xq, wq, act, ws, bias=b)
+    wsf, bf = orc.fold_into_producer(s, ws, b)
+    yf, acc_f = orc.gemm_w8a8(xq, wq, act, wsf, bias=bf)
+    assert np.array_equal(acc, acc_f)
+    term = acc.astype(np.float64) * act[:, None] * ws[None, :] / s[None, :]
+    ref = term + b[None, :] / s[None, :]
+    # four fp32 roundings, each relative to the terms (a sum may cancel)
+    bound = 4 * F32_EPS * (np.abs(term) + np.abs(b / s)[None, :])
+    assert np.all(np.abs(yf - ref) <= bound)
+    assert np.array_equal(np.maximum(yf, 0) > 0, np.maximum(ref, 0) > 0)
+    xq_f, a_f, _ = orc.quant_act(np.maximum(yf, 0).astype(np.float32), per_token=True)
+    xq_o, a_o, _ = orc.quant_act(np.maximum(y, 0).astype(np.float32),
+                                 inv_s=(1.0 / s).astype(np.float32), per_token=True)
+    assert np.mean(xq_f == xq_o) > 0.99 and np.max(np.abs(xq_f.astype(int) - xq_o)) <= 1
+
+
 def test_calib_absmax_running_and_library(orc):
     """S1 raw mode equals numpy's max(|X|) over tokens, and a running max
     over two batches equals the max over their concatenation."""
