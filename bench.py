@@ -51,7 +51,10 @@ INT8_PER_BF16 = 2.0
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 # DRAM bytes (read + write) of one launch of the dominant kernel, from the ncu
 # capture summarised in profiles/ (null when the kernel has changed since)
-GEMM_DRAM_TRAFFIC = {}
+GEMM_DRAM_TRAFFIC = {
+    "opt6.7b_qkv_t2048": (75.33e6, "profiles/gemm_w8a8_tc_opt6.7b_qkv_t2048.md: "
+                          "dram__bytes_read.sum 58.82 MB + dram__bytes_write.sum 16.51 MB"),
+}
 
 
 def load_peaks():

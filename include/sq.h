@@ -164,6 +164,26 @@ sq_status sq_fuse_weights_q8(const void* w, sq_dtype wt, int64_t N, int64_t K,
                              sq_stream stream);
 
 /*
+ * sq_fold_into_producer -- fold 1/s into the linear that produces this
+ * layer's input instead of into a norm or the quantizer ([review] §5.5: the
+ * smoothing factor folds into the previous layer's parameters).  The
+ * producer's output channel k is this layer's input channel k and has its
+ * own per-output-channel scale (from sq_fuse_weights_q8 on the producer) and
+ * bias, so
+ *
+ *   w_scale[k] = w_scale[k] / s[k],   bias[k] = bias[k] / s[k]
+ *
+ * (one fp32 division each, in place) makes the producer emit X diag(s)^-1
+ * directly (a ReLU in between commutes, s > 0), and this layer's quantizer
+ * then takes inv_s = NULL.  s [K] fp32 (from sq_smooth_scales of this
+ * layer); w_scale [K] fp32 in/out; bias [K] fp32 in/out or NULL; all device
+ * memory, 16-byte aligned.  Errors: SQ_ERR_SHAPE (K < 0),
+ * SQ_ERR_INVALID_ARG / SQ_ERR_ALIGN for the pointers; K = 0 does nothing.
+ */
+sq_status sq_fold_into_producer(const float* s, int64_t K, float* w_scale,
+                                float* bias, sq_stream stream);
+
+/*
  * sq_ln_smooth_quant_act -- runtime fused LayerNorm + smoothing + symmetric
  * INT8 activation quantizer ([embedded] §二: the modified LayerNorm emits the
  * smoothed activation, which is quantized per tensor and fed to the INT8

@@ -123,6 +123,15 @@ def test_rmsnorm_checks(lib):
     assert L.sq_rms_smooth_quant_act(A, 1, 0, 16, A2, 1e-5, 2, A2, A2, None, None) == lib.SQ_OK
 
 
+def test_fold_into_producer_checks(lib):
+    L = lib.lib
+    assert L.sq_fold_into_producer(None, 16, A2, None, None) == lib.SQ_ERR_INVALID_ARG
+    assert L.sq_fold_into_producer(A, 16, None, None, None) == lib.SQ_ERR_INVALID_ARG
+    assert L.sq_fold_into_producer(A, 16, A2, MIS, None) == lib.SQ_ERR_ALIGN
+    assert L.sq_fold_into_producer(A, -1, A2, None, None) == lib.SQ_ERR_SHAPE
+    assert L.sq_fold_into_producer(A, 0, A2, None, None) == lib.SQ_OK
+
+
 def test_gemm_bias_checks(lib):
     L = lib.lib
     assert L.sq_gemm_w8a8_bias(A, A, 4, 4, 16, A2, 1, A2, MIS, A2, 1, None, None, 0, None) == \

@@ -24,7 +24,7 @@ __all__ = [
     "sq_calib_absmax", "sq_smooth_scales", "sq_fuse_weights_q8",
     "sq_ln_smooth_quant_act", "sq_gemm_workspace_bytes", "sq_gemm_w8a8",
     "sq_sync_status", "sq_selftest_bounded_wait", "SQError", "Workspace",
-    "sq_calib_absmax_rms", "sq_rms_smooth_quant_act",
+    "sq_calib_absmax_rms", "sq_rms_smooth_quant_act", "sq_fold_into_producer",
 ]
 
 
@@ -116,6 +116,14 @@ def sq_rms_smooth_quant_act(x, xq, act_scale, gamma_s, eps=1e-5, per_token=True,
                                       _ptr(act_scale), _ptr(xq), _ptr(n_clipped),
                                       _stream(stream)), "sq_rms_smooth_quant_act")
     return xq, act_scale
+
+
+def sq_fold_into_producer(s, w_scale, bias=None, stream=None):
+    """1/s folded into the producing linear: w_scale /= s, bias /= s (in place)."""
+    K = s.numel()
+    check(lib.sq_fold_into_producer(_ptr(s), K, _ptr(w_scale), _ptr(bias), _stream(stream)),
+          "sq_fold_into_producer")
+    return w_scale, bias
 
 
 def sq_gemm_workspace_bytes(M, N, K) -> int:

@@ -215,6 +215,19 @@ sq_status quant_call(const char* fn, const void* x, sq_dtype xt, int64_t T, int6
 }
 }  // namespace
 
+sq_status sq_fold_into_producer(const float* s, int64_t K, float* w_scale, float* bias,
+                                sq_stream stream) {
+  const char* fn = "sq_fold_into_producer";
+  g_last_error[0] = 0;
+  if (K < 0) return fail(SQ_ERR_SHAPE, "%s: K=%lld < 0", fn, (long long)K);
+  SQ_REQ(s, fn);
+  SQ_REQ(w_scale, fn);
+  SQ_OPT(bias, fn);
+  if (K == 0) return SQ_OK;
+  cudaError_t e = launch_fold_producer(s, K, w_scale, bias, (cudaStream_t)stream);
+  return e == cudaSuccess ? SQ_OK : cuda_fail(e, fn);
+}
+
 sq_status sq_ln_smooth_quant_act(const void* x, sq_dtype xt, int64_t T, int64_t K,
                                  const float* gamma_s, const float* beta_s, float ln_eps,
                                  const float* inv_s, sq_act_gran gran, float* act_scale,

@@ -583,6 +583,29 @@ cudaError_t launch_peak_to_delta(float* act_scale, cudaStream_t st) {
   return launch_pdl(peak_to_delta_kernel, dim3(1), dim3(32), 0, st, act_scale);
 }
 
+// ============================================================ producer fold
+// 1/s folded into a producing linear: its per-output-channel scale and bias
+// divided by s (one fp32 division each, [review] §5.5).
+__global__ void fold_producer_kernel(const float* __restrict__ s, int64_t K, float* w_scale,
+                                     float* bias) {
+  pdl_launch_dependents();
+  pdl_wait();
+  for (int64_t k = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; k < K;
+       k += (int64_t)gridDim.x * blockDim.x) {
+    const float sk = s[k];
+    w_scale[k] = __fdiv_rn(w_scale[k], sk);
+    if (bias) bias[k] = __fdiv_rn(bias[k], sk);
+  }
+}
+
+cudaError_t launch_fold_producer(const float* s, int64_t K, float* w_scale, float* bias,
+                                 cudaStream_t st) {
+  int64_t blocks = (K + 255) / 256;
+  if (blocks > 1024) blocks = 1024;
+  return launch_pdl(fold_producer_kernel, dim3((unsigned)blocks), dim3(256), 0, st, s, K,
+                    w_scale, bias);
+}
+
 // ============================================================ LayerNorm fold
 // gamma' = gamma / s, beta' = beta / s ([embedded] §二), fp32 division.
 __global__ void fold_ln_kernel(const float* __restrict__ gamma, const float* __restrict__ beta,

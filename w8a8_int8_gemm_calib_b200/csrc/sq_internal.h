@@ -61,6 +61,10 @@ cudaError_t launch_scales(const float* amax_x, int64_t K, float alpha,
 // act_scale[0] = Delta(act_scale[0]) = max(peak, 1e-7) / 127 (one thread).
 cudaError_t launch_peak_to_delta(float* act_scale, cudaStream_t st);
 
+// w_scale[k] /= s[k], bias[k] /= s[k] (bias may be NULL).
+cudaError_t launch_fold_producer(const float* s, int64_t K, float* w_scale, float* bias,
+                                 cudaStream_t st);
+
 cudaError_t launch_fold_ln(const float* gamma, const float* beta,
                            const float* s, int64_t K, float* gamma_out,
                            float* beta_out, cudaStream_t st);
