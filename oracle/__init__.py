@@ -19,6 +19,7 @@ bit patterns in ``np.uint16`` and widened exactly inside the C code.
 from __future__ import annotations
 
 import ctypes
+import math
 import os
 import subprocess
 
@@ -288,3 +289,34 @@ def gemm_w8a8(xq, wq, act_scale, w_scale, per_token=True, rows=None,
     lib().orc_gemm_w8a8(_ptr(xq), _ptr(wq), M, N, K, _ptr(act_scale), int(per_token),
                         _ptr(w_scale), _ptr(bias), _ptr(r), R, _ptr(yf), _ptr(yb), _ptr(acc))
     return (yb if out_bf16 else yf), acc
+
+
+def output_error(y, y_ref):
+    """Relative Frobenius error ||y - y_ref|| / ||y_ref||, sums in fp64 (the
+    layer-output error that alpha is chosen by)."""
+    y = np.asarray(y, np.float64)
+    r = np.asarray(y_ref, np.float64)
+    num = float(np.sum((y - r) ** 2))
+    den = float(np.sum(r * r))
+    if den > 0:
+        return math.sqrt(num / den)
+    return math.inf if num > 0 else 0.0
+
+
+def alpha_error(amax_x, w, x, y_ref, alpha, gamma=None, beta=None, eps=1e-5,
+                gran="token"):
+    """The smoothed W8A8 layer at one alpha, built from the calibration peaks
+    amax_x: eq. (4), the fold, the quantizer at granularity gran ("token",
+    "static", "tensor"), the GEMM in fp32; returns its output_error against
+    y_ref."""
+    s, inv_s = smooth_scales(amax_x, weight_colmax(w), alpha)
+    wq, ws = fuse_weights_q8(w, s)
+    kw = dict(per_token=gran == "token", per_tensor_dynamic=gran == "tensor",
+              static_delta=static_delta(amax_x, s) if gran == "static" else None)
+    if gamma is not None:
+        g2, b2 = fold_ln(gamma, beta, s)
+        xq, act, _ = quant_act(x, g2, b2, eps, **kw)
+    else:
+        xq, act, _ = quant_act(x, inv_s=inv_s, **kw)
+    y, _ = gemm_w8a8(xq, wq, act, ws, per_token=gran == "token")
+    return output_error(y, y_ref)

@@ -541,6 +541,38 @@ def test_fold_into_producer(orc):
     assert np.mean(xq_f == xq_o) > 0.99 and np.max(np.abs(xq_f.astype(int) - xq_o)) <= 1
 
 
+def test_output_error_closed_forms(orc):
+    """The layer-output error metric: 0 for y = y_ref, 1 for y = 2 y_ref or
+    y = 0, and scale-invariant."""
+    r = np.random.default_rng(41).normal(0, 3, (7, 5)).astype(np.float32)
+    assert orc.output_error(r, r) == 0.0
+    assert orc.output_error(2 * r, r) == pytest.approx(1.0, rel=1e-15)
+    assert orc.output_error(np.zeros_like(r), r) == 1.0
+    assert orc.output_error(8 * r + 8, 8 * r) == pytest.approx(orc.output_error(r + 1, r),
+                                                                rel=1e-12)
+
+
+def test_alpha_sweep_u_shape(orc):
+    """Layer-output error against alpha on outlier-structured data ([review]
+    §5.3 eq. (4) and its alpha discussion: alpha = 0 leaves the activation
+    outliers in X, alpha = 1 moves them all into W; the paper's sweep, Fig. 10,
+    has its sweet spot in between).  Reference: the unquantized layer in
+    fp64.  The error at 0.5 is below both ends, for per-token and static
+    activations, with and without a LayerNorm."""
+    lin = synth.workloads()["tiny_k1024"].linears[0]
+    d = synth.make_linear_inputs(lin, T=64, T_cal=256, N=256)
+    x, x_cal, w = d["x"], d["x_cal"], d["w"]
+    for ln in (False, True):
+        g, b = (d["gamma"], d["beta"]) if ln else (None, None)
+        amax = orc.calib_absmax(x_cal, g, b)
+        f = (orc.layernorm_row(x[t], g, b) for t in range(x.shape[0])) if ln else iter(x)
+        fx = np.stack(list(f)).astype(np.float64)
+        y_ref = (fx @ w.astype(np.float64).T).astype(np.float32)
+        for gran in ("token", "static"):
+            e = {a: orc.alpha_error(amax, w, x, y_ref, a, g, b, gran=gran) for a in (0.0, 0.5, 1.0)}
+            assert e[0.5] < e[0.0] and e[0.5] < e[1.0], (ln, gran, e)
+
+
 def test_calib_absmax_running_and_library(orc):
     """S1 raw mode equals numpy's max(|X|) over tokens, and a running max
     over two batches equals the max over their concatenation."""
