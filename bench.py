@@ -360,7 +360,8 @@ def run_ours(args):
     small_m = None if args.no_small_m else run_small_m(sq, torch, dev, flush)
     next_rows = {"o2_per_tensor_dynamic_quant": run_o2(sq, torch, layer, lin, flush),
                  "gemm_bias_epilogue": run_gemm_bias(sq, torch, layer, lin, flush),
-                 "rmsnorm_quant_per_token": run_rms_quant(sq, torch, layer, lin, flush)}
+                 "rmsnorm_quant_per_token": run_rms_quant(sq, torch, layer, lin, flush),
+                 "alpha_sweep": run_alpha_sweep(sq, torch, layer, lin, flush)}
 
     peaks, peak_kind = load_peaks()
     bf16_peak = peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"])
@@ -530,6 +531,33 @@ def time_call(torch, call, flush, reps=20):
         times.append(e0.elapsed_time(e1))
     del graph
     return statistics.mean(times)
+
+
+def run_alpha_sweep(sq, torch, layer, lin, flush, alphas=(0.0, 0.25, 0.5, 0.75, 1.0)):
+    """alpha chosen by the layer's output error (NEXT-2): the whole smoothed
+    layer at five alphas on the step's tokens (eq. (4), fold, quantizer,
+    GEMM in fp32, fp64 error), against the unquantized layer in fp32 (the
+    reference is computed once with torch, outside the timing)."""
+    import torch.nn.functional as F
+
+    xf = layer.x.float()
+    if lin.ln:
+        xf = F.layer_norm(xf, (lin.K,), layer.gamma, layer.beta, 1e-5)
+    y_ref = xf @ layer.w.float().t()
+    ws = sq.Workspace(layer.x.device)
+    out = {}
+
+    def call():
+        out["err"] = sq.sq_alpha_sweep(layer.amax, layer.w, layer.x, y_ref, list(alphas),
+                                       layer.gamma, layer.beta, per_token=lin.per_token,
+                                       workspace=ws)
+
+    ms = time_call(torch, call, flush, reps=5)
+    sq.sq_sync_status()
+    err = out["err"].cpu().tolist()
+    del y_ref
+    return {"shape": f"{lin.T}x{lin.N}x{lin.K}", "alphas": list(alphas),
+            "rel_error": [round(e, 6) for e in err], "us_per_alpha": round(ms * 1e3 / len(alphas), 1)}
 
 
 def run_rms_quant(sq, torch, layer, lin, flush):

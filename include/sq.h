@@ -317,6 +317,41 @@ sq_status sq_gemm_w8a8_noalloc(const int8_t* xq, const int8_t* wq, int64_t M,
                                sq_stream stream);
 
 /*
+ * sq_alpha_sweep -- choose the migration strength alpha by the layer's
+ * output error (eq. (4)'s alpha, [review] §5.3; the paper sweeps it and
+ * finds a sweet spot between the activation side, alpha = 0, and the weight
+ * side, alpha = 1).  For each alphas[i] the whole smoothed W8A8 layer runs
+ * on the GPU with this library's kernels -- eq. (4) from the calibration
+ * peaks amax_x and the weight column peaks (computed once), the fold
+ * (W * s -> INT8 and, with a LayerNorm, gamma / s, beta / s), the runtime
+ * quantizer at granularity gran on the evaluation tokens x, the INT8 GEMM
+ * in fp32 -- and
+ *
+ *   err[i] = ||y - y_ref||_F / ||y_ref||_F      (sums in fp64)
+ *
+ * against the caller's reference output y_ref (typically the unquantized
+ * layer, f(x) W^T in fp32 or better).
+ *
+ *   amax_x [K] fp32 (from sq_calib_absmax, with the LayerNorm when one
+ *   precedes); w [N,K] of type wt; x [M,K] of type xt; ln_gamma / ln_beta
+ *   [K] fp32 or NULL (no LayerNorm: the quantizer multiplies by 1/s);
+ *   y_ref [M,N] fp32; alphas: HOST array of n_alpha values in [0,1];
+ *   err: DEVICE array of n_alpha doubles (out); workspace: at least
+ *   sq_alpha_sweep_workspace_bytes(M,N,K) bytes of device memory, 16-byte
+ *   aligned (holds every intermediate of one alpha, reused for the next).
+ *   Errors as the calls it composes, SQ_ERR_WORKSPACE for a short
+ *   workspace; n_alpha = 0 does nothing.
+ */
+size_t sq_alpha_sweep_workspace_bytes(int64_t M, int64_t N, int64_t K);
+sq_status sq_alpha_sweep(const float* amax_x, const void* w, sq_dtype wt,
+                         int64_t N, int64_t K, const void* x, sq_dtype xt,
+                         int64_t M, const float* ln_gamma,
+                         const float* ln_beta, float ln_eps,
+                         const float* y_ref, const float* alphas, int n_alpha,
+                         sq_act_gran gran, double* err, void* workspace,
+                         size_t workspace_bytes, sq_stream stream);
+
+/*
  * sq_sync_status -- synchronize `stream`, then return and clear the status
  * word of the current device: SQ_OK, or SQ_ERR_TIMEOUT when a kernel gave up
  * a bounded wait (its outputs are then undefined), or SQ_ERR_CUDA when the

@@ -132,6 +132,23 @@ def test_fold_into_producer_checks(lib):
     assert L.sq_fold_into_producer(A, 0, A2, None, None) == lib.SQ_OK
 
 
+def test_alpha_sweep_checks(lib):
+    import ctypes as C
+
+    L = lib.lib
+    need = L.sq_alpha_sweep_workspace_bytes(64, 256, 1024)
+    assert need > 256 * 1024 + 64 * 1024 + 4 * 64 * 256
+    assert L.sq_alpha_sweep_workspace_bytes(0, 256, 1024) == 0
+    good = (C.c_float * 2)(0.0, 0.5)
+    bad = (C.c_float * 2)(0.5, 1.5)
+    args = lambda al, n, gran, ws_bytes: (A, A, 1, 256, 1024, A, 1, 64, None, None, 1e-5, A,
+                                          al, n, gran, A2, A2, ws_bytes, None)
+    assert L.sq_alpha_sweep(*args(bad, 2, 1, need)) == lib.SQ_ERR_INVALID_ARG
+    assert L.sq_alpha_sweep(*args(good, 2, 5, need)) == lib.SQ_ERR_INVALID_ARG
+    assert L.sq_alpha_sweep(*args(good, 2, 1, need - 1)) == lib.SQ_ERR_WORKSPACE
+    assert L.sq_alpha_sweep(*args(good, 0, 1, need)) == lib.SQ_OK
+
+
 def test_gemm_bias_checks(lib):
     L = lib.lib
     assert L.sq_gemm_w8a8_bias(A, A, 4, 4, 16, A2, 1, A2, MIS, A2, 1, None, None, 0, None) == \

@@ -14,6 +14,8 @@ Sources:
 """
 from __future__ import annotations
 
+import ctypes
+
 import torch
 
 from . import _lib
@@ -25,6 +27,7 @@ __all__ = [
     "sq_ln_smooth_quant_act", "sq_gemm_workspace_bytes", "sq_gemm_w8a8",
     "sq_sync_status", "sq_selftest_bounded_wait", "SQError", "Workspace",
     "sq_calib_absmax_rms", "sq_rms_smooth_quant_act", "sq_fold_into_producer",
+    "sq_alpha_sweep_workspace_bytes", "sq_alpha_sweep",
 ]
 
 
@@ -124,6 +127,33 @@ def sq_fold_into_producer(s, w_scale, bias=None, stream=None):
     check(lib.sq_fold_into_producer(_ptr(s), K, _ptr(w_scale), _ptr(bias), _stream(stream)),
           "sq_fold_into_producer")
     return w_scale, bias
+
+
+def sq_alpha_sweep_workspace_bytes(M, N, K) -> int:
+    return int(lib.sq_alpha_sweep_workspace_bytes(M, N, K))
+
+
+def sq_alpha_sweep(amax_x, w, x, y_ref, alphas, ln_gamma=None, ln_beta=None, ln_eps=1e-5,
+                   per_token=True, per_tensor_dynamic=False, workspace=None, stream=None):
+    """Layer-output error of the smoothed W8A8 layer at each alpha: a CUDA
+    tensor of len(alphas) doubles, ||y - y_ref|| / ||y_ref||."""
+    N, K = w.shape
+    M = x.shape[0]
+    if per_tensor_dynamic:
+        gran = SQ_ACT_PER_TENSOR_DYNAMIC
+    else:
+        gran = SQ_ACT_PER_TOKEN_DYNAMIC if per_token else SQ_ACT_PER_TENSOR_STATIC
+    need = sq_alpha_sweep_workspace_bytes(M, N, K)
+    ws = workspace.get(need) if isinstance(workspace, Workspace) else workspace
+    if ws is None:
+        ws = torch.empty(need, dtype=torch.uint8, device=x.device)
+    a = (ctypes.c_float * len(alphas))(*[float(v) for v in alphas])
+    err = torch.empty(len(alphas), dtype=torch.float64, device=x.device)
+    check(lib.sq_alpha_sweep(_ptr(amax_x), _ptr(w), _dt(w), N, K, _ptr(x), _dt(x), M,
+                             _ptr(ln_gamma), _ptr(ln_beta), ln_eps, _ptr(y_ref), a, len(alphas),
+                             gran, _ptr(err), _ptr(ws), ws.numel() * ws.element_size(),
+                             _stream(stream)), "sq_alpha_sweep")
+    return err
 
 
 def sq_gemm_workspace_bytes(M, N, K) -> int:

@@ -165,6 +165,24 @@ sq_status sq_fuse_weights_q8(const void* w, sq_dtype wt, int64_t N, int64_t K, c
 }
 
 namespace {
+// The quantizer at granularity gran on validated arguments (a.scale is
+// act_scale).  Per-tensor dynamic: two passes over x -- the peak of |y| over
+// the call (into act_scale[0]), Delta of it in place, then the static
+// quantizer with that step.
+cudaError_t run_quant(const RowArgs& a, sq_dtype xt, sq_act_gran gran, cudaStream_t st) {
+  if (gran != SQ_ACT_PER_TENSOR_DYNAMIC)
+    return launch_row(a, xt, gran == SQ_ACT_PER_TOKEN_DYNAMIC ? ROW_DYNAMIC : ROW_STATIC, st);
+  RowArgs p = a;
+  p.q = nullptr;
+  p.n_clipped = nullptr;
+  p.peak = a.scale;
+  cudaError_t e = cudaMemsetAsync(a.scale, 0, sizeof(float), st);
+  if (e == cudaSuccess) e = launch_row(p, xt, ROW_PEAK, st);
+  if (e == cudaSuccess) e = launch_peak_to_delta(a.scale, st);
+  if (e == cudaSuccess) e = launch_row(a, xt, ROW_STATIC, st);
+  return e;
+}
+
 sq_status quant_call(const char* fn, const void* x, sq_dtype xt, int64_t T, int64_t K,
                      const float* gamma_s, const float* beta_s, float ln_eps, int rms,
                      const float* inv_s, sq_act_gran gran, float* act_scale, int8_t* xq,
@@ -195,22 +213,7 @@ sq_status quant_call(const char* fn, const void* x, sq_dtype xt, int64_t T, int6
   a.x = x; a.T = T; a.K = K; a.g = gamma_s; a.b = beta_s; a.eps = ln_eps; a.rms = rms;
   a.mul = inv_s;
   a.scale = act_scale; a.q = xq; a.n_clipped = (unsigned long long*)n_clipped;
-  const cudaStream_t st = (cudaStream_t)stream;
-  cudaError_t e;
-  if (gran == SQ_ACT_PER_TENSOR_DYNAMIC) {
-    // two passes over x: the peak of |y| over the call (into act_scale[0]),
-    // Delta of it in place, then the static quantizer with that step
-    RowArgs p = a;
-    p.q = nullptr;
-    p.n_clipped = nullptr;
-    p.peak = act_scale;
-    e = cudaMemsetAsync(act_scale, 0, sizeof(float), st);
-    if (e == cudaSuccess) e = launch_row(p, xt, ROW_PEAK, st);
-    if (e == cudaSuccess) e = launch_peak_to_delta(act_scale, st);
-    if (e == cudaSuccess) e = launch_row(a, xt, ROW_STATIC, st);
-  } else {
-    e = launch_row(a, xt, gran == SQ_ACT_PER_TOKEN_DYNAMIC ? ROW_DYNAMIC : ROW_STATIC, st);
-  }
+  const cudaError_t e = run_quant(a, xt, gran, (cudaStream_t)stream);
   return e == cudaSuccess ? SQ_OK : cuda_fail(e, fn);
 }
 }  // namespace
@@ -324,6 +327,134 @@ sq_status sq_gemm_w8a8_noalloc(const int8_t* xq, const int8_t* wq, int64_t M, in
   a.act_per_token = act_per_token ? 1 : 0; a.w_scale = w_scale; a.y = y; a.yt = yt;
   a.acc_out = acc_out;
   return launch_gemm_noalloc(a, (cudaStream_t)stream);
+}
+
+namespace {
+// Workspace of sq_alpha_sweep, carved in this order (each piece 256-byte
+// aligned): wmax, s, inv_s, Delta_A [K|K|K|4] fp32; gamma', beta' [K|K];
+// w_scale [N]; act_scale [M]; wq [N,K]; xq [M,K]; y [M,N] fp32; the error
+// reduction's per-block fp64 sums; then the GEMM's own workspace.
+struct SweepLayout {
+  size_t wmax, s, inv_s, dA, g2, b2, ws, act, wq, xq, y, sums, gemm, total;
+};
+SweepLayout sweep_layout(int64_t M, int64_t N, int64_t K) {
+  auto al = [](size_t v) { return (v + 255) & ~(size_t)255; };
+  SweepLayout L{};
+  size_t o = 0;
+  L.wmax = o; o += al(4 * (size_t)K);
+  L.s = o; o += al(4 * (size_t)K);
+  L.inv_s = o; o += al(4 * (size_t)K);
+  L.dA = o; o += al(16);
+  L.g2 = o; o += al(4 * (size_t)K);
+  L.b2 = o; o += al(4 * (size_t)K);
+  L.ws = o; o += al(4 * (size_t)N);
+  L.act = o; o += al(4 * (size_t)M);
+  L.wq = o; o += al((size_t)N * (size_t)K);
+  L.xq = o; o += al((size_t)M * (size_t)K);
+  L.y = o; o += al(4 * (size_t)M * (size_t)N);
+  L.sums = o; o += al(output_error_scratch_bytes());
+  L.gemm = o; o += al(gemm_workspace_bytes(M, N, K));
+  L.total = o;
+  return L;
+}
+}  // namespace
+
+size_t sq_alpha_sweep_workspace_bytes(int64_t M, int64_t N, int64_t K) {
+  if (M <= 0 || N <= 0 || K <= 0) return 0;
+  return sweep_layout(M, N, K).total;
+}
+
+sq_status sq_alpha_sweep(const float* amax_x, const void* w, sq_dtype wt, int64_t N, int64_t K,
+                         const void* x, sq_dtype xt, int64_t M, const float* ln_gamma,
+                         const float* ln_beta, float ln_eps, const float* y_ref,
+                         const float* alphas, int n_alpha, sq_act_gran gran, double* err,
+                         void* workspace, size_t workspace_bytes, sq_stream stream) {
+  const char* fn = "sq_alpha_sweep";
+  g_last_error[0] = 0;
+  SQ_TRY(check_dtype(wt, fn));
+  SQ_TRY(check_dtype(xt, fn));
+  if (gran != SQ_ACT_PER_TENSOR_STATIC && gran != SQ_ACT_PER_TOKEN_DYNAMIC &&
+      gran != SQ_ACT_PER_TENSOR_DYNAMIC)
+    return fail(SQ_ERR_INVALID_ARG, "%s: unknown granularity %d", fn, (int)gran);
+  if (M <= 0 || N <= 0) return fail(SQ_ERR_SHAPE, "%s: M=%lld N=%lld must be >= 1", fn,
+                                    (long long)M, (long long)N);
+  if (M > (int64_t)1 << 31 || N > (int64_t)1 << 31)
+    return fail(SQ_ERR_SHAPE, "%s: M and N must be below 2^31", fn);
+  SQ_TRY(check_k(K, fn));
+  if (n_alpha < 0) return fail(SQ_ERR_INVALID_ARG, "%s: n_alpha=%d < 0", fn, n_alpha);
+  if (n_alpha > 0 && !alphas) return fail(SQ_ERR_INVALID_ARG, "%s: alphas is NULL", fn);
+  for (int i = 0; i < n_alpha; ++i)
+    if (!(alphas[i] >= 0.0f && alphas[i] <= 1.0f))
+      return fail(SQ_ERR_INVALID_ARG, "%s: alphas[%d] = %g is not in [0, 1]", fn, i,
+                  (double)alphas[i]);
+  SQ_REQ(amax_x, fn);
+  SQ_REQ(w, fn);
+  SQ_REQ(x, fn);
+  SQ_REQ(y_ref, fn);
+  SQ_REQ(err, fn);
+  SQ_OPT(ln_gamma, fn);
+  SQ_OPT(ln_beta, fn);
+  if (ln_beta && !ln_gamma) return fail(SQ_ERR_INVALID_ARG, "%s: ln_beta given without ln_gamma", fn);
+  if (ln_gamma && !(ln_eps >= 0.0f && isfinite(ln_eps)))
+    return fail(SQ_ERR_INVALID_ARG, "%s: ln_eps must be finite and >= 0", fn);
+  const SweepLayout L = sweep_layout(M, N, K);
+  if (!workspace || workspace_bytes < L.total)
+    return fail(SQ_ERR_WORKSPACE, "%s: workspace of %zu bytes needed, %zu given", fn, L.total,
+                workspace ? workspace_bytes : (size_t)0);
+  SQ_OPT(workspace, fn);
+  if (n_alpha == 0) return SQ_OK;
+  uint8_t* base = (uint8_t*)workspace;
+  float* wmax = (float*)(base + L.wmax);
+  float* s = (float*)(base + L.s);
+  float* inv_s = (float*)(base + L.inv_s);
+  float* dA = (float*)(base + L.dA);
+  float* g2 = (float*)(base + L.g2);
+  float* b2 = (float*)(base + L.b2);
+  float* ws = (float*)(base + L.ws);
+  float* act = (float*)(base + L.act);
+  int8_t* wq = (int8_t*)(base + L.wq);
+  int8_t* xq = (int8_t*)(base + L.xq);
+  float* y = (float*)(base + L.y);
+  double* sums = (double*)(base + L.sums);
+  const cudaStream_t st = (cudaStream_t)stream;
+  const bool stat = gran == SQ_ACT_PER_TENSOR_STATIC;
+  // the weight column peaks do not depend on alpha
+  cudaError_t e = cudaMemsetAsync(wmax, 0, 4 * (size_t)K, st);
+  if (e == cudaSuccess) e = launch_colmax(w, wt, N, K, wmax, st);
+  for (int i = 0; e == cudaSuccess && i < n_alpha; ++i) {
+    // eq. (4) (and the static step); scales_kernel reads the peaks from s
+    e = cudaMemcpyAsync(s, wmax, 4 * (size_t)K, cudaMemcpyDeviceToDevice, st);
+    if (e == cudaSuccess) e = launch_scales(amax_x, K, alphas[i], s, inv_s, stat ? dA : nullptr, st);
+    // the fold: W * s -> wq, w_scale; gamma / s, beta / s
+    RowArgs f{};
+    f.x = w; f.T = N; f.K = K; f.mul = s; f.scale = ws; f.q = wq;
+    if (e == cudaSuccess) e = launch_row(f, wt, ROW_DYNAMIC, st);
+    if (e == cudaSuccess && ln_gamma)
+      e = launch_fold_ln(ln_gamma, ln_beta, s, K, g2, ln_beta ? b2 : nullptr, st);
+    // the quantizer
+    RowArgs q{};
+    q.x = x; q.T = M; q.K = K; q.eps = ln_eps; q.scale = act; q.q = xq;
+    if (ln_gamma) {
+      q.g = g2;
+      q.b = ln_beta ? b2 : nullptr;
+    } else {
+      q.mul = inv_s;
+    }
+    if (e == cudaSuccess && stat)
+      e = cudaMemcpyAsync(act, dA, sizeof(float), cudaMemcpyDeviceToDevice, st);
+    if (e == cudaSuccess) e = run_quant(q, xt, gran, st);
+    // the GEMM in fp32, then the error against y_ref
+    GemmArgs g{};
+    g.xq = xq; g.wq = wq; g.M = M; g.N = N; g.K = K; g.act_scale = act;
+    g.act_per_token = gran == SQ_ACT_PER_TOKEN_DYNAMIC ? 1 : 0; g.w_scale = ws; g.y = y;
+    g.yt = SQ_F32; g.workspace = base + L.gemm; g.workspace_bytes = L.total - L.gemm;
+    if (e == cudaSuccess) {
+      const sq_status gs = launch_gemm(g, st);
+      if (gs != SQ_OK) return gs;
+    }
+    if (e == cudaSuccess) e = launch_output_error(y, y_ref, M * N, sums, err + i, st);
+  }
+  return e == cudaSuccess ? SQ_OK : cuda_fail(e, fn);
 }
 
 sq_status sq_sync_status(sq_stream stream) {

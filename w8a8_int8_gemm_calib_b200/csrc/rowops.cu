@@ -583,6 +583,84 @@ cudaError_t launch_peak_to_delta(float* act_scale, cudaStream_t st) {
   return launch_pdl(peak_to_delta_kernel, dim3(1), dim3(32), 0, st, act_scale);
 }
 
+// ============================================================ output error
+// sum (y - r)^2 and sum r^2 in fp64, deterministic: each thread accumulates
+// a grid-stride share, warps and blocks reduce, each block writes its two
+// partial sums to its own slot, and one thread adds the slots in block
+// order.
+constexpr int kErrThreads = 256;
+
+int output_error_blocks(int64_t n) {
+  int64_t blocks = (n + kErrThreads - 1) / kErrThreads;
+  const int64_t cap = 8 * (int64_t)sm_count();
+  if (blocks > cap) blocks = cap;
+  return blocks < 1 ? 1 : (int)blocks;
+}
+
+size_t output_error_scratch_bytes() { return 2 * sizeof(double) * 8 * (size_t)sm_count(); }
+
+__device__ __forceinline__ double warp_sum_d(double v) {
+#pragma unroll
+  for (int o = 16; o >= 1; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+
+__global__ void __launch_bounds__(kErrThreads)
+output_error_kernel(const float* __restrict__ y, const float* __restrict__ r, int64_t n,
+                    double* part_out) {
+  __shared__ double part[2][kErrThreads / 32];
+  pdl_launch_dependents();
+  pdl_wait();
+  double num = 0.0, den = 0.0;
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n;
+       i += (int64_t)gridDim.x * blockDim.x) {
+    const double a = (double)__ldg(y + i), b = (double)__ldg(r + i);
+    const double d = a - b;
+    num += d * d;
+    den += b * b;
+  }
+  num = warp_sum_d(num);
+  den = warp_sum_d(den);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (lane == 0) {
+    part[0][warp] = num;
+    part[1][warp] = den;
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    double a = 0.0, b = 0.0;
+    for (int w = 0; w < kErrThreads / 32; ++w) {
+      a += part[0][w];
+      b += part[1][w];
+    }
+    part_out[2 * blockIdx.x] = a;
+    part_out[2 * blockIdx.x + 1] = b;
+  }
+}
+
+__global__ void output_error_final_kernel(const double* part, int nblocks, double* err) {
+  pdl_launch_dependents();
+  pdl_wait();
+  if (threadIdx.x == 0) {
+    double num = 0.0, den = 0.0;
+    for (int i = 0; i < nblocks; ++i) {
+      num += part[2 * i];
+      den += part[2 * i + 1];
+    }
+    *err = den > 0.0 ? sqrt(num / den) : (num > 0.0 ? (double)INFINITY : 0.0);
+  }
+}
+
+cudaError_t launch_output_error(const float* y, const float* y_ref, int64_t n, double* scratch,
+                                double* err, cudaStream_t st) {
+  const int blocks = output_error_blocks(n);
+  cudaError_t e = launch_pdl(output_error_kernel, dim3((unsigned)blocks), dim3(kErrThreads), 0,
+                             st, y, y_ref, n, scratch);
+  if (e != cudaSuccess) return e;
+  return launch_pdl(output_error_final_kernel, dim3(1), dim3(32), 0, st,
+                    (const double*)scratch, blocks, err);
+}
+
 // ============================================================ producer fold
 // 1/s folded into a producing linear: its per-output-channel scale and bias
 // divided by s (one fp32 division each, [review] §5.5).

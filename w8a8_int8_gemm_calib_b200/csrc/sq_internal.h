@@ -65,6 +65,13 @@ cudaError_t launch_peak_to_delta(float* act_scale, cudaStream_t st);
 cudaError_t launch_fold_producer(const float* s, int64_t K, float* w_scale, float* bias,
                                  cudaStream_t st);
 
+// Relative Frobenius error of y against y_ref (n fp32 values each), in
+// fp64 and deterministic: *err = sqrt(sum (y - r)^2 / sum r^2) (0 / 0 = 0,
+// x / 0 = inf).  scratch: output_error_scratch_bytes() of device memory.
+size_t output_error_scratch_bytes();
+cudaError_t launch_output_error(const float* y, const float* y_ref, int64_t n, double* scratch,
+                                double* err, cudaStream_t st);
+
 cudaError_t launch_fold_ln(const float* gamma, const float* beta,
                            const float* s, int64_t K, float* gamma_out,
                            float* beta_out, cudaStream_t st);
