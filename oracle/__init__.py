@@ -227,6 +227,25 @@ def fuse_weights_q8(w, s):
     return wq, ws
 
 
+def bmm_w8a8(xq, wq, act_scale, w_scale, per_token=True, w_per_channel=True, out_bf16=False):
+    """S6 applied to each batch b of xq [B, M, K] and wq [B, N, K]: act_scale
+    [B*M] (per token) or [B]; w_scale [B*N] (per channel) or [B].  Returns
+    (y [B, M, N], acc [B, M, N])."""
+    xq = np.ascontiguousarray(xq, np.int8)
+    wq = np.ascontiguousarray(wq, np.int8)
+    B, M, _ = xq.shape
+    N = wq.shape[1]
+    act_scale, w_scale = _f32(act_scale), _f32(w_scale)
+    ys, accs = [], []
+    for b in range(B):
+        a = act_scale[b * M:(b + 1) * M] if per_token else act_scale[b:b + 1]
+        w = w_scale[b * N:(b + 1) * N] if w_per_channel else np.full(N, w_scale[b], np.float32)
+        y, acc = gemm_w8a8(xq[b], wq[b], a, w, per_token=per_token, out_bf16=out_bf16)
+        ys.append(y)
+        accs.append(acc)
+    return np.stack(ys), np.stack(accs)
+
+
 def fold_into_producer(s, w_scale, bias=None):
     """The producer's per-output-channel scale (and bias) divided by s."""
     s = _f32(s)

@@ -261,6 +261,32 @@ def test_gemm_bias_exact(orc):
     assert np.array_equal(y0, y1)
 
 
+def test_bmm_brute_force_tiny(orc):
+    """The batched form (attention's INT8 matmuls, [review] §5.6 Fig. 6):
+    every batch against Python-integer triple loops and a once-rounded fp64
+    dequantization, with per-token / per-tensor activation steps and
+    per-channel / per-batch weight steps; a scale taken from the wrong batch
+    or axis fails."""
+    r = np.random.default_rng(17)
+    B, M, N, K = 3, 5, 7, 48
+    xq = r.integers(-127, 128, (B, M, K)).astype(np.int8)
+    wq = r.integers(-127, 128, (B, N, K)).astype(np.int8)
+    for per_token in (True, False):
+        for per_channel in (True, False):
+            act = r.uniform(1e-3, 1.0, B * M if per_token else B).astype(np.float32)
+            ws = r.uniform(1e-4, 1e-2, B * N if per_channel else B).astype(np.float32)
+            y, acc = orc.bmm_w8a8(xq, wq, act, ws, per_token, per_channel)
+            for b in range(B):
+                for t in range(M):
+                    for n in range(N):
+                        ref = sum(int(xq[b, t, k]) * int(wq[b, n, k]) for k in range(K))
+                        assert acc[b, t, n] == ref
+                        a = act[b * M + t] if per_token else act[b]
+                        w = ws[b * N + n] if per_channel else ws[b]
+                        scale = np.float32(np.float64(a) * np.float64(w))
+                        assert y[b, t, n] == np.float32(np.float64(np.float32(ref)) * scale)
+
+
 def test_gemm_saturation_closed_form(orc):
     """All-127 operands: acc = 127*127*K = 16129*K (K=20480 -> 330,321,920),
     the largest magnitude any layer in the workloads reaches."""
