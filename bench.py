@@ -361,7 +361,8 @@ def run_ours(args):
     next_rows = {"o2_per_tensor_dynamic_quant": run_o2(sq, torch, layer, lin, flush),
                  "gemm_bias_epilogue": run_gemm_bias(sq, torch, layer, lin, flush),
                  "rmsnorm_quant_per_token": run_rms_quant(sq, torch, layer, lin, flush),
-                 "alpha_sweep": run_alpha_sweep(sq, torch, layer, lin, flush)}
+                 "alpha_sweep": run_alpha_sweep(sq, torch, layer, lin, flush),
+                 "attention_bmm": run_attention_bmm(sq, torch, layer.x.device, flush)}
 
     peaks, peak_kind = load_peaks()
     bf16_peak = peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"])
@@ -558,6 +559,30 @@ def run_alpha_sweep(sq, torch, layer, lin, flush, alphas=(0.0, 0.25, 0.5, 0.75, 
     del y_ref
     return {"shape": f"{lin.T}x{lin.N}x{lin.K}", "alphas": list(alphas),
             "rel_error": [round(e, 6) for e in err], "us_per_alpha": round(ms * 1e3 / len(alphas), 1)}
+
+
+def run_attention_bmm(sq, torch, dev, flush, heads=32, tokens=2048, head_dim=128):
+    """Attention's INT8 matmuls (NEXT-4) at OPT-6.7B shapes, one batched
+    launch over the heads each: scores = Q K^T (per-token Q steps, one K step
+    per head) and P V (V^T as the K-major operand), bf16 out."""
+    g = torch.Generator(device=dev).manual_seed(11)
+    peaks, _ = load_peaks()
+    int8_peak = peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]) * INT8_PER_BF16
+    out = {}
+    for name, (M, N, K) in (("scores_qk", (tokens, tokens, head_dim)),
+                            ("pv", (tokens, head_dim, tokens))):
+        xq = torch.randint(-127, 128, (heads, M, K), dtype=torch.int8, device=dev, generator=g)
+        wq = torch.randint(-127, 128, (heads, N, K), dtype=torch.int8, device=dev, generator=g)
+        act = torch.rand(heads * M, device=dev, generator=g) * 0.01 + 1e-4
+        ws = torch.rand(heads, device=dev, generator=g) * 0.01 + 1e-4
+        y = torch.empty((heads, M, N), dtype=torch.bfloat16, device=dev)
+        ms = time_call(torch, lambda: sq.sq_bmm_w8a8(xq, wq, act, ws, y, per_token=True,
+                                                     w_per_channel=False), flush)
+        sq.sq_sync_status()
+        tops = 2.0 * heads * M * N * K / (ms * 1e-3) / 1e12
+        out[name] = {"shape": f"{heads}x{M}x{N}x{K}", "us": round(ms * 1e3, 2),
+                     "tops": round(tops, 1), "int8_frac": round(tops / int8_peak, 3)}
+    return out
 
 
 def run_rms_quant(sq, torch, layer, lin, flush):

@@ -317,6 +317,30 @@ sq_status sq_gemm_w8a8_noalloc(const int8_t* xq, const int8_t* wq, int64_t M,
                                sq_stream stream);
 
 /*
+ * sq_bmm_w8a8 -- batched INT8 matrix multiplication for the attention block
+ * (SmoothQuant quantizes the batched matmuls of attention to INT8 as well,
+ * [review] §5.6 Fig. 6): for every b in [0, batch)
+ *
+ *   acc[b,t,n] = sum_k xq[b,t,k] * wq[b,n,k]                (exact INT32)
+ *   y[b,t,n]   = (float)acc[b,t,n] * (as * ws)               (fp32, RNE)
+ *   as = act_scale[b*M + t] if act_per_token else act_scale[b]
+ *   ws = w_scale[b*N + n]   if w_per_channel else w_scale[b]
+ *
+ * e.g. scores = Q K^T with xq = Q [heads, T, d] and wq = K [heads, T, d],
+ * or P V with xq = P [heads, T, T] and wq = V^T [heads, d, T].  Both
+ * operands are K-major (K contiguous, a multiple of 16); the batches are
+ * stored back to back: xq [batch, M, K], wq [batch, N, K], y and acc_out
+ * [batch, M, N].  One persistent tcgen05 launch covers every batch.
+ * No workspace.  Errors as sq_gemm_w8a8 (no bias); batch times the number
+ * of 128 x 128 tiles must stay below 2^31.
+ */
+sq_status sq_bmm_w8a8(const int8_t* xq, const int8_t* wq, int64_t batch,
+                      int64_t M, int64_t N, int64_t K, const float* act_scale,
+                      int act_per_token, const float* w_scale,
+                      int w_per_channel, void* y, sq_dtype yt, int32_t* acc_out,
+                      sq_stream stream);
+
+/*
  * sq_alpha_sweep -- choose the migration strength alpha by the layer's
  * output error (eq. (4)'s alpha, [review] §5.3; the paper sweeps it and
  * finds a sweet spot between the activation side, alpha = 0, and the weight

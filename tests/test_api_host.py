@@ -149,6 +149,17 @@ def test_alpha_sweep_checks(lib):
     assert L.sq_alpha_sweep(*args(good, 0, 1, need)) == lib.SQ_OK
 
 
+def test_bmm_checks(lib):
+    L = lib.lib
+    assert L.sq_bmm_w8a8(A, A, 2, 4, 4, 24, A2, 1, A2, 1, A2, 1, None, None) == lib.SQ_ERR_SHAPE
+    assert L.sq_bmm_w8a8(A, A, -1, 4, 4, 16, A2, 1, A2, 1, A2, 1, None, None) == lib.SQ_ERR_SHAPE
+    assert L.sq_bmm_w8a8(A, None, 2, 4, 4, 16, A2, 1, A2, 1, A2, 1, None, None) == \
+        lib.SQ_ERR_INVALID_ARG
+    assert L.sq_bmm_w8a8(A, A, 2, 4, 4, 16, A2, 1, A2, 1, MIS, 1, None, None) == lib.SQ_ERR_ALIGN
+    assert L.sq_bmm_w8a8(A, A, 2, 4, 4, 16, A2, 1, A2, 1, A2, 9, None, None) == lib.SQ_ERR_DTYPE
+    assert L.sq_bmm_w8a8(A, A, 0, 4, 4, 16, A2, 1, A2, 1, A2, 1, None, None) == lib.SQ_OK
+
+
 def test_gemm_bias_checks(lib):
     L = lib.lib
     assert L.sq_gemm_w8a8_bias(A, A, 4, 4, 16, A2, 1, A2, MIS, A2, 1, None, None, 0, None) == \

@@ -27,7 +27,7 @@ __all__ = [
     "sq_ln_smooth_quant_act", "sq_gemm_workspace_bytes", "sq_gemm_w8a8",
     "sq_sync_status", "sq_selftest_bounded_wait", "SQError", "Workspace",
     "sq_calib_absmax_rms", "sq_rms_smooth_quant_act", "sq_fold_into_producer",
-    "sq_alpha_sweep_workspace_bytes", "sq_alpha_sweep",
+    "sq_alpha_sweep_workspace_bytes", "sq_alpha_sweep", "sq_bmm_w8a8",
 ]
 
 
@@ -154,6 +154,18 @@ def sq_alpha_sweep(amax_x, w, x, y_ref, alphas, ln_gamma=None, ln_beta=None, ln_
                              gran, _ptr(err), _ptr(ws), ws.numel() * ws.element_size(),
                              _stream(stream)), "sq_alpha_sweep")
     return err
+
+
+def sq_bmm_w8a8(xq, wq, act_scale, w_scale, y, per_token=True, w_per_channel=True,
+                acc_out=None, stream=None):
+    """Batched INT8 GEMM: y[b] = (float)(xq[b] @ wq[b]^T) * (as * ws), xq
+    [batch, M, K], wq [batch, N, K], y [batch, M, N]."""
+    B, M, K = xq.shape
+    N = wq.shape[1]
+    check(lib.sq_bmm_w8a8(_ptr(xq), _ptr(wq), B, M, N, K, _ptr(act_scale), int(per_token),
+                          _ptr(w_scale), int(w_per_channel), _ptr(y), _dt(y), _ptr(acc_out),
+                          _stream(stream)), "sq_bmm_w8a8")
+    return y
 
 
 def sq_gemm_workspace_bytes(M, N, K) -> int:

@@ -303,6 +303,36 @@ sq_status sq_gemm_w8a8_bias(const int8_t* xq, const int8_t* wq, int64_t M, int64
                    y, yt, acc_out, workspace, workspace_bytes, stream);
 }
 
+sq_status sq_bmm_w8a8(const int8_t* xq, const int8_t* wq, int64_t batch, int64_t M, int64_t N,
+                      int64_t K, const float* act_scale, int act_per_token, const float* w_scale,
+                      int w_per_channel, void* y, sq_dtype yt, int32_t* acc_out,
+                      sq_stream stream) {
+  const char* fn = "sq_bmm_w8a8";
+  g_last_error[0] = 0;
+  SQ_TRY(check_dtype(yt, fn));
+  if (batch < 0 || M < 0 || N < 0)
+    return fail(SQ_ERR_SHAPE, "%s: batch=%lld M=%lld N=%lld must be >= 0", fn, (long long)batch,
+                (long long)M, (long long)N);
+  SQ_TRY(check_k(K, fn));
+  if (batch == 0 || M == 0 || N == 0) return SQ_OK;
+  const int64_t tiles = batch * ((M + 127) / 128) * ((N + 127) / 128);
+  if (M > (int64_t)1 << 31 || N > (int64_t)1 << 31 || tiles > ((int64_t)1 << 31) - 1 ||
+      batch > ((int64_t)1 << 31) - 1)
+    return fail(SQ_ERR_SHAPE, "%s: batch x tiles must stay below 2^31", fn);
+  SQ_REQ(xq, fn);
+  SQ_REQ(wq, fn);
+  SQ_REQ(act_scale, fn);
+  SQ_REQ(w_scale, fn);
+  SQ_REQ(y, fn);
+  SQ_OPT(acc_out, fn);
+  BmmArgs a{};
+  a.xq = xq; a.wq = wq; a.batch = batch; a.M = M; a.N = N; a.K = K;
+  a.act_scale = act_scale; a.act_per_token = act_per_token ? 1 : 0;
+  a.w_scale = w_scale; a.w_per_channel = w_per_channel ? 1 : 0;
+  a.y = y; a.yt = yt; a.acc_out = acc_out;
+  return launch_bmm(a, (cudaStream_t)stream);
+}
+
 sq_status sq_gemm_w8a8_noalloc(const int8_t* xq, const int8_t* wq, int64_t M, int64_t N,
                                int64_t K, const float* act_scale, int act_per_token,
                                const float* w_scale, void* y, sq_dtype yt, int32_t* acc_out,

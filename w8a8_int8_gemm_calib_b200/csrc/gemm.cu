@@ -59,7 +59,8 @@ template <int TBN>
 struct TcCfg {
   static constexpr int B_BYTES = TBN * BK;
   static constexpr int STAGE = A_BYTES + B_BYTES;
-  static constexpr int STAGES = TBN == 256 ? 4 : 5;
+  // as many stages as fit in 200 KB: 4 at 256 columns, 5 at 192, 6 at 128
+  static constexpr int STAGES = (200 * 1024) / STAGE;
   static constexpr uint32_t TMEM_COLS = 2 * TBN <= 256 ? 256 : 512;  // power of two
   static constexpr size_t SMEM = 1024 + (size_t)STAGES * STAGE + EPI_BYTES + 256;
   static_assert(SMEM <= 227 * 1024, "shared memory");
@@ -68,6 +69,8 @@ struct TcCfg {
 struct Params {
   int M, N, K;
   int m_tiles, n_tiles, num_tiles, nk;
+  int tiles_per_batch;  // m_tiles * n_tiles (num_tiles = batch * tiles_per_batch)
+  int w_per_tensor;     // batched: one weight step per batch (w_scale[b])
   int tma_store;  // outputs leave through shared memory and TMA stores
   const float* act_scale;
   int per_token;
@@ -90,7 +93,7 @@ __device__ __forceinline__ void tile_coords(int tile, int m_tiles, int n_tiles, 
 
 // 32 per-column values (scales or bias) starting at col0; 0 past N.
 __device__ __forceinline__ void load_cols32(const float* src, int col0, int N, float (&v)[32]) {
-  if (col0 + 32 <= N) {
+  if (col0 + 32 <= N && ((reinterpret_cast<uintptr_t>(src + col0) & 15) == 0)) {
     const float4* s4 = reinterpret_cast<const float4*>(src + col0);
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
@@ -109,24 +112,39 @@ __device__ __forceinline__ float dequant(uint32_t acc, float as, float ws) {
   return __fmul_rn(__int2float_rn((int)acc), __fmul_rn(as, ws));
 }
 
-// Store 32 consecutive outputs of one row.  Fast path: 16-byte vector stores
-// when the whole chunk is in range and rows stay 16-byte aligned.
-template <bool BF16>
-__device__ __forceinline__ void store_chunk(const Params& p, int row, int col0,
-                                            const uint32_t (&r)[32], float as) {
-  const bool full = col0 + 32 <= p.N;
+// The 32 outputs of one row from columns col0..col0+31 of batch b:
+// (float)acc * (as * ws[n]) (+ bias[n]); ws per output channel (batch b's
+// row of w_scale) or, for a batch with one weight step, w_scale[b].
+template <bool BATCH>
+__device__ __forceinline__ void dequant_chunk(const Params& p, int b, int col0,
+                                              const uint32_t (&r)[32], float as,
+                                              float (&yv)[32]) {
   float ws[32];
-  load_cols32(p.w_scale, col0, p.N, ws);
-  float yv[32];
+  if (BATCH && p.w_per_tensor) {
+    const float w = __ldg(p.w_scale + b);
+#pragma unroll
+    for (int i = 0; i < 32; ++i) ws[i] = w;
+  } else {
+    load_cols32(p.w_scale + (BATCH ? (size_t)b * (size_t)p.N : (size_t)0), col0, p.N, ws);
+  }
 #pragma unroll
   for (int i = 0; i < 32; ++i) yv[i] = dequant(r[i], as, ws[i]);
-  if (p.bias) {
+  if (p.bias) {  // never with a batch
     float bs[32];
     load_cols32(p.bias, col0, p.N, bs);
 #pragma unroll
     for (int i = 0; i < 32; ++i) yv[i] = __fadd_rn(yv[i], bs[i]);
   }
-  const size_t base = (size_t)row * (size_t)p.N + (size_t)col0;
+}
+
+// Store 32 consecutive outputs (and accumulators) of output row yrow.  Fast
+// path: 16-byte vector stores when the whole chunk is in range and rows
+// stay 16-byte aligned.
+template <bool BF16>
+__device__ __forceinline__ void store_chunk(const Params& p, size_t yrow, int col0,
+                                            const uint32_t (&r)[32], const float (&yv)[32]) {
+  const bool full = col0 + 32 <= p.N;
+  const size_t base = yrow * (size_t)p.N + (size_t)col0;
   if (BF16) {
     __nv_bfloat16* y = reinterpret_cast<__nv_bfloat16*>(p.y) + base;
     if (full && (p.N % 8) == 0) {
@@ -171,7 +189,7 @@ __device__ __forceinline__ void store_chunk(const Params& p, int row, int col0,
   }
 }
 
-template <bool BF16, int TBN>
+template <bool BF16, int TBN, bool BATCH>
 __global__ void __launch_bounds__(THREADS, 1)
 gemm_w8a8_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                     const __grid_constant__ CUtensorMap tmY, const Params p) {
@@ -231,15 +249,25 @@ gemm_w8a8_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
       bool ok = true;
       for (int tile = blockIdx.x; ok && tile < p.num_tiles; tile += gridDim.x) {
         int mb, nb;
-        tile_coords(tile, p.m_tiles, p.n_tiles, mb, nb);
+        const int b = BATCH ? tile / p.tiles_per_batch : 0;
+        tile_coords(tile - b * p.tiles_per_batch, p.m_tiles, p.n_tiles, mb, nb);
         for (int kb = 0; kb < p.nk; ++kb) {
           if (!tc::mbar_wait(empty_bar(stage), phase ^ 1u, abort_flag, kWaitNs, p.status)) {
             ok = false;
             break;
           }
           tc::mbar_arrive_expect_tx(full_bar(stage), STAGE_BYTES);
-          tc::tma_load_2d(tc::smem_u32(sA + stage * A_BYTES), &tmA, kb * BK, mb * BM, full_bar(stage));
-          tc::tma_load_2d(tc::smem_u32(sB + stage * B_BYTES), &tmB, kb * BK, nb * BN, full_bar(stage));
+          if constexpr (BATCH) {
+            tc::tma_load_3d(tc::smem_u32(sA + stage * A_BYTES), &tmA, kb * BK, mb * BM, b,
+                            full_bar(stage));
+            tc::tma_load_3d(tc::smem_u32(sB + stage * B_BYTES), &tmB, kb * BK, nb * BN, b,
+                            full_bar(stage));
+          } else {
+            tc::tma_load_2d(tc::smem_u32(sA + stage * A_BYTES), &tmA, kb * BK, mb * BM,
+                            full_bar(stage));
+            tc::tma_load_2d(tc::smem_u32(sB + stage * B_BYTES), &tmB, kb * BK, nb * BN,
+                            full_bar(stage));
+          }
           issued |= 1u << stage;
           issued_par = (issued_par & ~(1u << stage)) | (phase << stage);
           if (++stage == STAGES) { stage = 0; phase ^= 1u; }
@@ -301,13 +329,16 @@ gemm_w8a8_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
     uint32_t abuf = 0, aphase = 0;
     for (int tile = blockIdx.x; tile < p.num_tiles; tile += gridDim.x) {
       int mb, nb;
-      tile_coords(tile, p.m_tiles, p.n_tiles, mb, nb);
+      const int b = BATCH ? tile / p.tiles_per_batch : 0;
+      tile_coords(tile - b * p.tiles_per_batch, p.m_tiles, p.n_tiles, mb, nb);
       if (!tc::mbar_wait(tfull_bar(abuf), aphase, abort_flag, kWaitNs, p.status)) break;
       tc::tc_fence_after();
       const int row0 = mb * BM + quarter * 32;
       const int row = row0 + lane;
       const bool row_ok = row < p.M;
-      const float as = p.per_token ? (row_ok ? __ldg(p.act_scale + row) : 0.0f) : __ldg(p.act_scale);
+      const size_t yrow = (size_t)b * (size_t)p.M + (size_t)row;  // output row of [batch*M, N]
+      const float as = p.per_token ? (row_ok ? __ldg(p.act_scale + yrow) : 0.0f)
+                                   : __ldg(p.act_scale + b);
       const uint32_t taddr = tmem_base + abuf * BN + ((uint32_t)(quarter * 32) << 16);
 #pragma unroll 1
       for (int c = 0; c < BN / 32; ++c) {
@@ -315,23 +346,12 @@ gemm_w8a8_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
         tc::tmem_ld32(taddr + c * 32, r);
         tc::tmem_ld_wait();
         const int col0 = nb * BN + c * 32;
-        if (!p.tma_store) {
-          if (row_ok && col0 < p.N) store_chunk<BF16>(p, row, col0, r, as);
-          continue;
-        }
         // dequantize this lane's 32 outputs (row `row`, columns col0..+31)
         float yv[32];
-        {
-          float ws[32];
-          load_cols32(p.w_scale, col0, p.N, ws);
-#pragma unroll
-          for (int i = 0; i < 32; ++i) yv[i] = dequant(r[i], as, ws[i]);
-        }
-        if (p.bias) {
-          float bs[32];
-          load_cols32(p.bias, col0, p.N, bs);
-#pragma unroll
-          for (int i = 0; i < 32; ++i) yv[i] = __fadd_rn(yv[i], bs[i]);
+        dequant_chunk<BATCH>(p, b, col0, r, as, yv);
+        if (!p.tma_store) {
+          if (row_ok && col0 < p.N) store_chunk<BF16>(p, yrow, col0, r, yv);
+          continue;
         }
         uint32_t wv[BF16 ? 16 : 32];
 #pragma unroll
@@ -347,7 +367,7 @@ gemm_w8a8_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
           }
         }
         if (p.acc && row_ok && col0 < p.N) {
-          int32_t* a = p.acc + (size_t)row * p.N + col0;
+          int32_t* a = p.acc + yrow * p.N + col0;
 #pragma unroll
           for (int i = 0; i < 32; ++i)
             if (col0 + i < p.N) a[i] = (int)r[i];
@@ -372,7 +392,10 @@ gemm_w8a8_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
           __syncwarp();
           if (lane == 0) {
             const int cx = col0 + h * 16;
-            if (any && cx < p.N) tc::tma_store_2d(&tmY, tc::smem_u32(buf), cx, row0);
+            if (any && cx < p.N) {
+              if constexpr (BATCH) tc::tma_store_3d(&tmY, tc::smem_u32(buf), cx, row0, b);
+              else tc::tma_store_2d(&tmY, tc::smem_u32(buf), cx, row0);
+            }
             tc::bulk_commit();
           }
           ++nstore;
@@ -738,7 +761,40 @@ bool make_tmap_out(CUtensorMap* m, void* base, uint64_t cols, uint64_t rows, boo
   return r == CUDA_SUCCESS;
 }
 
-template <bool BF16, int TBN>
+// Batched operands: [batch, rows, inner] int8 (K-major rows), box
+// [1, box_rows, 128 bytes], 128-byte swizzle, zero fill past each batch's
+// rows and inner extent.
+bool make_tmap3(CUtensorMap* m, const void* base, uint64_t inner, uint64_t rows, uint64_t batch,
+                uint32_t box_rows) {
+  auto enc = encode_fn();
+  if (!enc) return false;
+  cuuint64_t dims[3] = {inner, rows, batch};
+  cuuint64_t strides[2] = {inner, inner * rows};
+  cuuint32_t box[3] = {(cuuint32_t)BK, box_rows, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void*>(base), dims, strides, box,
+                   estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+// Batched output [batch, rows, cols]: stores clipped at each batch's edges.
+bool make_tmap_out3(CUtensorMap* m, void* base, uint64_t cols, uint64_t rows, uint64_t batch,
+                    bool bf16) {
+  auto enc = encode_fn();
+  if (!enc) return false;
+  const uint64_t esz = bf16 ? 2 : 4;
+  cuuint64_t dims[3] = {cols, rows, batch};
+  cuuint64_t strides[2] = {cols * esz, cols * rows * esz};
+  cuuint32_t box[3] = {(cuuint32_t)(64 / esz), 32, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = enc(m, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3,
+                   base, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                   CU_TENSOR_MAP_SWIZZLE_64B, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+template <bool BF16, int TBN, bool BATCH = false>
 cudaError_t launch_tc(const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& ty,
                       const Params& p, int grid, cudaStream_t st) {
   static std::once_flag once[64];
@@ -747,24 +803,25 @@ cudaError_t launch_tc(const CUtensorMap& ta, const CUtensorMap& tb, const CUtens
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess || dev < 0 || dev >= 64) return e != cudaSuccess ? e : cudaErrorInvalidDevice;
   std::call_once(once[dev], [&] {
-    attr_err[dev] = cudaFuncSetAttribute(gemm_w8a8_tc_kernel<BF16, TBN>,
+    attr_err[dev] = cudaFuncSetAttribute(gemm_w8a8_tc_kernel<BF16, TBN, BATCH>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)TcCfg<TBN>::SMEM);
   });
   if (attr_err[dev] != cudaSuccess) return attr_err[dev];
-  return launch_pdl(gemm_w8a8_tc_kernel<BF16, TBN>, dim3(grid), dim3(THREADS), TcCfg<TBN>::SMEM, st,
-                    ta, tb, ty, p);
+  return launch_pdl(gemm_w8a8_tc_kernel<BF16, TBN, BATCH>, dim3(grid), dim3(THREADS),
+                    TcCfg<TBN>::SMEM, st, ta, tb, ty, p);
 }
 
 // Tile width for the large-M kernel: the per-tile time grows with the width,
 // and a partly filled last wave costs a whole tile time, so take the width
 // with the smaller (waves x width) -- plus a fixed per-tile cost.
-int pick_tile_n(int64_t M, int64_t N, int sms) {
+int pick_tile_n(int64_t M, int64_t N, int sms, int64_t batch = 1, bool narrow = false) {
   const int64_t mt = (M + BM - 1) / BM;
   int best = 256;
   int64_t best_cost = -1;
-  for (int tbn : {256, 192}) {
-    const int64_t tiles = mt * ((N + tbn - 1) / tbn);
+  for (int tbn : {256, 192, 128}) {
+    if (tbn == 128 && !narrow) continue;
+    const int64_t tiles = batch * mt * ((N + tbn - 1) / tbn);
     const int64_t waves = (tiles + sms - 1) / sms;
     const int64_t cost = waves * (tbn + 16);
     if (best_cost < 0 || cost < best_cost) { best = tbn; best_cost = cost; }
@@ -911,6 +968,7 @@ sq_status launch_gemm(const GemmArgs& a, cudaStream_t st) {
   p.m_tiles = (int)((a.M + BM - 1) / BM);
   p.n_tiles = (int)((a.N + tbn - 1) / tbn);
   p.num_tiles = p.m_tiles * p.n_tiles;
+  p.tiles_per_batch = p.num_tiles;
   p.nk = (int)((a.K + BK - 1) / BK);
   p.act_scale = a.act_scale;
   p.per_token = a.act_per_token;
@@ -932,6 +990,48 @@ sq_status launch_gemm(const GemmArgs& a, cudaStream_t st) {
                               : (bf16 ? launch_tc<true, 192>(ta, tb, ty, p, grid, st)
                                       : launch_tc<false, 192>(ta, tb, ty, p, grid, st));
   if (e != cudaSuccess) return fail(SQ_ERR_CUDA, "sq_gemm_w8a8: %s", cudaGetErrorString(e));
+  return SQ_OK;
+}
+
+sq_status launch_bmm(const BmmArgs& a, cudaStream_t st) {
+  unsigned int* sw = status_word();
+  if (!sw) return fail(SQ_ERR_CUDA, "sq_bmm_w8a8: device status word unavailable");
+  const int sms = sm_count();
+  const int tbn = pick_tile_n(a.M, a.N, sms, a.batch, true);
+  CUtensorMap ta, tb;
+  if (!make_tmap3(&ta, a.xq, (uint64_t)a.K, (uint64_t)a.M, (uint64_t)a.batch, BM) ||
+      !make_tmap3(&tb, a.wq, (uint64_t)a.K, (uint64_t)a.N, (uint64_t)a.batch, (uint32_t)tbn))
+    return fail(SQ_ERR_CUDA, "sq_bmm_w8a8: cuTensorMapEncodeTiled failed");
+  Params p{};
+  p.M = (int)a.M; p.N = (int)a.N; p.K = (int)a.K;
+  p.m_tiles = (int)((a.M + BM - 1) / BM);
+  p.n_tiles = (int)((a.N + tbn - 1) / tbn);
+  p.tiles_per_batch = p.m_tiles * p.n_tiles;
+  p.num_tiles = (int)(a.batch * p.tiles_per_batch);
+  p.nk = (int)((a.K + BK - 1) / BK);
+  p.w_per_tensor = a.w_per_channel ? 0 : 1;
+  p.act_scale = a.act_scale;
+  p.per_token = a.act_per_token;
+  p.w_scale = a.w_scale;
+  p.bias = nullptr;
+  p.y = a.y;
+  p.acc = a.acc_out;
+  p.status = sw;
+  CUtensorMap ty;
+  memset(&ty, 0, sizeof ty);
+  const bool bf16 = a.yt == SQ_BF16;
+  p.tma_store = (a.N % (bf16 ? 8 : 4)) == 0 &&
+                make_tmap_out3(&ty, a.y, (uint64_t)a.N, (uint64_t)a.M, (uint64_t)a.batch, bf16);
+  int grid = sms;
+  if (grid > p.num_tiles) grid = p.num_tiles;
+  cudaError_t e;
+  if (tbn == 256) e = bf16 ? launch_tc<true, 256, true>(ta, tb, ty, p, grid, st)
+                           : launch_tc<false, 256, true>(ta, tb, ty, p, grid, st);
+  else if (tbn == 192) e = bf16 ? launch_tc<true, 192, true>(ta, tb, ty, p, grid, st)
+                                : launch_tc<false, 192, true>(ta, tb, ty, p, grid, st);
+  else e = bf16 ? launch_tc<true, 128, true>(ta, tb, ty, p, grid, st)
+                : launch_tc<false, 128, true>(ta, tb, ty, p, grid, st);
+  if (e != cudaSuccess) return fail(SQ_ERR_CUDA, "sq_bmm_w8a8: %s", cudaGetErrorString(e));
   return SQ_OK;
 }
 

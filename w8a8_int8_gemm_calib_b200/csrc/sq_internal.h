@@ -92,6 +92,23 @@ struct GemmArgs {
   size_t workspace_bytes;
 };
 
+// Batched INT8 GEMM (attention BMMs): y[b] = xq[b] wq[b]^T dequantized
+// per batch; act_scale [batch*M] (per token) or [batch]; w_scale [batch*N]
+// (per channel) or [batch]; y, acc_out [batch, M, N].
+struct BmmArgs {
+  const int8_t* xq;
+  const int8_t* wq;
+  int64_t batch, M, N, K;
+  const float* act_scale;
+  int act_per_token;
+  const float* w_scale;
+  int w_per_channel;
+  void* y;
+  sq_dtype yt;
+  int32_t* acc_out;
+};
+sq_status launch_bmm(const BmmArgs& a, cudaStream_t st);
+
 size_t gemm_workspace_bytes(int64_t M, int64_t N, int64_t K);
 sq_status launch_gemm(const GemmArgs& a, cudaStream_t st);
 
