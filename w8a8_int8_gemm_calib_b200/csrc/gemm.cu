@@ -35,34 +35,33 @@ namespace sq {
 namespace {
 
 constexpr int BM = 128;     // token rows per tile (MMA M)
-constexpr int BN = 256;     // output channels per tile (MMA N)
 constexpr int BK = 128;     // bytes of K per stage = one 128B swizzle row
 constexpr int UK = 32;      // K per tcgen05.mma kind::i8
-constexpr int STAGES = 4;
 constexpr int A_BYTES = BM * BK;
-constexpr int B_BYTES = BN * BK;
-constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
 constexpr int THREADS = 192;
-constexpr uint32_t TMEM_COLS = 2 * BN;
 constexpr int GROUP_M = 16;  // tile raster: 16 row blocks share each column sweep
 constexpr uint64_t kWaitNs = 4000000000ull;   // 4 s: far above any pipeline step
 constexpr uint64_t kDrainNs = 1000000000ull;  // waits for copies already in flight
-// Output staging for the TMA-store epilogue: per epilogue warp, two buffers
-// of 32 rows x 64 bytes (32 bf16 or 16 fp32 columns), 64-byte swizzled.
+// Output staging for the TMA-store epilogue: per epilogue warp, buffers of
+// 32 rows x 64 bytes (32 bf16 or 16 fp32 columns), 64-byte swizzled.
 constexpr int EPI_BUF = 32 * 64;
-constexpr int EPI_BYTES = 4 * 2 * EPI_BUF;
-constexpr size_t SMEM_BYTES = 1024 + (size_t)STAGES * STAGE_BYTES + EPI_BYTES + 256;
 
-// Large-M tile shapes: 128 x TBN outputs per tile, TBN in {256, 192}; the
-// host picks the one that fills the last wave of SMs best.
-template <int TBN>
+// Large-M tile shapes: 128 x TBN outputs per tile, TBN in {256, 192, 128};
+// the host picks the one that fills the last wave of SMs best.  EPI_NB
+// output staging buffers per epilogue warp (EPI_NB - 1 TMA stores in flight
+// per warp; deeper staging was measured not to speed up output-bound
+// shapes, whose epilogue is latency-bound instead).
+template <int TBN, int EPI_NB = 2>
 struct TcCfg {
   static constexpr int B_BYTES = TBN * BK;
   static constexpr int STAGE = A_BYTES + B_BYTES;
-  // as many stages as fit in 200 KB: 4 at 256 columns, 5 at 192, 6 at 128
-  static constexpr int STAGES = (200 * 1024) / STAGE;
+  static constexpr int EPI_BYTES = 4 * EPI_NB * EPI_BUF;
+  // as many stages as fit: with 2 staging buffers 4 at 256 columns, 5 at
+  // 192, 6 at 128
+  static constexpr int STAGES = (224 * 1024 - 2048 - EPI_BYTES) / STAGE;
   static constexpr uint32_t TMEM_COLS = 2 * TBN <= 256 ? 256 : 512;  // power of two
   static constexpr size_t SMEM = 1024 + (size_t)STAGES * STAGE + EPI_BYTES + 256;
+  static_assert(STAGES >= 2, "two main-loop stages at least");
   static_assert(SMEM <= 227 * 1024, "shared memory");
 };
 
@@ -189,11 +188,11 @@ __device__ __forceinline__ void store_chunk(const Params& p, size_t yrow, int co
   }
 }
 
-template <bool BF16, int TBN, bool BATCH>
+template <bool BF16, int TBN, bool BATCH, int EPI_NB>
 __global__ void __launch_bounds__(THREADS, 1)
 gemm_w8a8_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                     const __grid_constant__ CUtensorMap tmY, const Params p) {
-  using C = TcCfg<TBN>;
+  using C = TcCfg<TBN, EPI_NB>;
   constexpr int STAGES = C::STAGES;
   constexpr int B_BYTES = C::B_BYTES;
   constexpr int STAGE_BYTES = C::STAGE;
@@ -204,7 +203,7 @@ gemm_w8a8_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
   uint8_t* sA = smem;
   uint8_t* sB = smem + STAGES * A_BYTES;
   uint8_t* sEpi = smem + STAGES * STAGE_BYTES;  // 1024-aligned
-  uint64_t* bars = reinterpret_cast<uint64_t*>(sEpi + EPI_BYTES);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sEpi + C::EPI_BYTES);
   // bars: full[STAGES], empty[STAGES], tfull[2], tempty[2], drain
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * STAGES + 5);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
@@ -324,7 +323,7 @@ gemm_w8a8_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
   } else {
     // ------------------------------------------------------------ epilogue
     const int quarter = warp & 3;  // this warp may read TMEM lanes 32*quarter..+31
-    uint8_t* ebuf = sEpi + (warp - 2) * 2 * EPI_BUF;
+    uint8_t* ebuf = sEpi + (warp - 2) * EPI_NB * EPI_BUF;
     uint32_t nstore = 0;  // TMA stores issued by this warp (selects the buffer)
     uint32_t abuf = 0, aphase = 0;
     for (int tile = blockIdx.x; tile < p.num_tiles; tile += gridDim.x) {
@@ -376,8 +375,9 @@ gemm_w8a8_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
         const bool any = row0 < p.M && col0 < p.N;  // warp-uniform
 #pragma unroll
         for (int h = 0; h < (BF16 ? 1 : 2); ++h) {
-          uint8_t* buf = ebuf + (nstore & 1) * EPI_BUF;
-          if (lane == 0) tc::bulk_wait_read<1>();  // the store that last read `buf` is done
+          uint8_t* buf = ebuf + (nstore % EPI_NB) * EPI_BUF;
+          // the store that last read `buf` (EPI_NB stores ago) is done
+          if (lane == 0) tc::bulk_wait_read<EPI_NB - 1>();
           __syncwarp();
           // row `lane`, 16-byte chunk k at chunk k ^ ((lane >> 1) & 3): the
           // 64-byte swizzle the tensor map undoes (conflict-free writes)
@@ -794,22 +794,23 @@ bool make_tmap_out3(CUtensorMap* m, void* base, uint64_t cols, uint64_t rows, ui
   return r == CUDA_SUCCESS;
 }
 
-template <bool BF16, int TBN, bool BATCH = false>
+template <bool BF16, int TBN, bool BATCH = false, int EPI_NB = 2>
 cudaError_t launch_tc(const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& ty,
                       const Params& p, int grid, cudaStream_t st) {
+  using C = TcCfg<TBN, EPI_NB>;
   static std::once_flag once[64];
   static cudaError_t attr_err[64];
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess || dev < 0 || dev >= 64) return e != cudaSuccess ? e : cudaErrorInvalidDevice;
   std::call_once(once[dev], [&] {
-    attr_err[dev] = cudaFuncSetAttribute(gemm_w8a8_tc_kernel<BF16, TBN, BATCH>,
+    attr_err[dev] = cudaFuncSetAttribute(gemm_w8a8_tc_kernel<BF16, TBN, BATCH, EPI_NB>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)TcCfg<TBN>::SMEM);
+                                         (int)C::SMEM);
   });
   if (attr_err[dev] != cudaSuccess) return attr_err[dev];
-  return launch_pdl(gemm_w8a8_tc_kernel<BF16, TBN, BATCH>, dim3(grid), dim3(THREADS),
-                    TcCfg<TBN>::SMEM, st, ta, tb, ty, p);
+  return launch_pdl(gemm_w8a8_tc_kernel<BF16, TBN, BATCH, EPI_NB>, dim3(grid), dim3(THREADS),
+                    C::SMEM, st, ta, tb, ty, p);
 }
 
 // Tile width for the large-M kernel: the per-tile time grows with the width,
