@@ -198,7 +198,9 @@ class Layer:
 
     def step(self, ev=None, upto=5):
         """The first `upto` of the five calls (all five: one step); ev = (start,
-        end) events recorded around them, or None."""
+        end) events recorded around them, or None.  (Running the weight
+        column peaks on a second stream beside the calibration was measured
+        no faster: whichever kernel starts first fills the SMs.)"""
         sq, L = self.sq, self.lin
         if ev is not None:
             ev[0].record()

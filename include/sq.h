@@ -145,6 +145,28 @@ sq_status sq_smooth_scales(const float* amax_x, const void* w, sq_dtype wt,
                            sq_stream stream);
 
 /*
+ * sq_weight_colmax and sq_smooth_scales_peaks -- sq_smooth_scales in two
+ * steps, for callers that keep the weight peaks (an alpha search, a model
+ * whose weights do not change) or compute them concurrently with the
+ * calibration (they do not depend on it):
+ *
+ *   sq_weight_colmax:        amax_w[k] = max_n |W[n,k]|   (w [N,K] type wt;
+ *                            amax_w [K] fp32 out, overwritten)
+ *   sq_smooth_scales_peaks:  s, inv_s (and act_delta_static) from amax_x and
+ *                            amax_w exactly as sq_smooth_scales computes them
+ *                            (amax_w is floored at 1e-7 there, not here)
+ *
+ * Arguments and errors as sq_smooth_scales; the two steps give the same
+ * bits as the one call.
+ */
+sq_status sq_weight_colmax(const void* w, sq_dtype wt, int64_t N, int64_t K,
+                           float* amax_w, sq_stream stream);
+sq_status sq_smooth_scales_peaks(const float* amax_x, const float* amax_w,
+                                 int64_t K, float alpha, float* s,
+                                 float* inv_s, float* act_delta_static,
+                                 sq_stream stream);
+
+/*
  * sq_fuse_weights_q8 -- offline fold of s ([embedded] §二; [review] §5.1
  * eq. (3), §5.5):
  *

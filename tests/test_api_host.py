@@ -160,6 +160,19 @@ def test_bmm_checks(lib):
     assert L.sq_bmm_w8a8(A, A, 0, 4, 4, 16, A2, 1, A2, 1, A2, 1, None, None) == lib.SQ_OK
 
 
+def test_weight_peaks_and_scales_checks(lib):
+    L = lib.lib
+    assert L.sq_weight_colmax(A, 1, 4, 24, A2, None) == lib.SQ_ERR_SHAPE
+    assert L.sq_weight_colmax(A, 1, 4, 16, None, None) == lib.SQ_ERR_INVALID_ARG
+    assert L.sq_weight_colmax(A, 5, 4, 16, A2, None) == lib.SQ_ERR_DTYPE
+    assert L.sq_weight_colmax(MIS, 1, 4, 16, A2, None) == lib.SQ_ERR_ALIGN
+    assert L.sq_smooth_scales_peaks(A, A, 16, 1.5, A2, A2, None, None) == lib.SQ_ERR_INVALID_ARG
+    assert L.sq_smooth_scales_peaks(A, None, 16, 0.5, A2, A2, None, None) == \
+        lib.SQ_ERR_INVALID_ARG
+    assert L.sq_smooth_scales_peaks(A, A, 20, 0.5, A2, A2, None, None) == lib.SQ_ERR_SHAPE
+    assert L.sq_smooth_scales_peaks(A, A, 16, 0.5, A2, A2, MIS, None) == lib.SQ_ERR_ALIGN
+
+
 def test_gemm_bias_checks(lib):
     L = lib.lib
     assert L.sq_gemm_w8a8_bias(A, A, 4, 4, 16, A2, 1, A2, MIS, A2, 1, None, None, 0, None) == \

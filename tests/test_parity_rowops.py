@@ -252,3 +252,26 @@ def test_fuse_weights_ring_reuse(sq, orc, N, K):
     sq.sq_sync_status()
     assert_bits_equal(host(ws), ws_want, "w_scale")
     assert_bits_equal(host(wq), wq_want, "wq")
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+@pytest.mark.parametrize("N,K", [(1, 16), (300, 1040), (12288, 4096), (77, 20480)])
+@pytest.mark.parametrize("alpha", [0.5, 0.8, 0.0, 1.0])
+def test_weight_peaks_then_scales(sq, orc, dtype, N, K, alpha):
+    """sq_weight_colmax + sq_smooth_scales_peaks (the weight peaks computed on
+    their own, e.g. concurrently with the calibration) give the weight peaks
+    of the oracle and the same bits as the one-call sq_smooth_scales,
+    including the static step."""
+    w = _x(N + K, N, K, dtype)
+    amax_x = np.abs(_x(K, 64, K, "f32")).max(axis=0).astype(np.float32)
+    f32 = dict(dtype=torch.float32, device="cuda")
+    amax_w = torch.empty(K, **f32)
+    sq.sq_weight_colmax(dev(w), amax_w)
+    s1, i1, d1 = torch.empty(K, **f32), torch.empty(K, **f32), torch.empty(1, **f32)
+    sq.sq_smooth_scales_peaks(dev(amax_x), amax_w, alpha, s1, i1, d1)
+    s2, i2, d2 = torch.empty(K, **f32), torch.empty(K, **f32), torch.empty(1, **f32)
+    sq.sq_smooth_scales(dev(amax_x), dev(w), alpha, s2, i2, d2)
+    sq.sq_sync_status()
+    assert_bits_equal(host(amax_w), orc.weight_colmax(w), "amax_w")
+    for a, b, what in ((s1, s2, "s"), (i1, i2, "inv_s"), (d1, d2, "delta_A")):
+        assert_bits_equal(host(a), host(b), what)

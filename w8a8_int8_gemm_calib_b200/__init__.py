@@ -28,6 +28,7 @@ __all__ = [
     "sq_sync_status", "sq_selftest_bounded_wait", "SQError", "Workspace",
     "sq_calib_absmax_rms", "sq_rms_smooth_quant_act", "sq_fold_into_producer",
     "sq_alpha_sweep_workspace_bytes", "sq_alpha_sweep", "sq_bmm_w8a8",
+    "sq_weight_colmax", "sq_smooth_scales_peaks",
 ]
 
 
@@ -75,6 +76,23 @@ def sq_smooth_scales(amax_x, w, alpha, s, inv_s, act_delta_static=None, stream=N
     check(lib.sq_smooth_scales(_ptr(amax_x), _ptr(w), _dt(w), N, K, float(alpha), _ptr(s),
                                _ptr(inv_s), _ptr(act_delta_static), _stream(stream)),
           "sq_smooth_scales")
+    return s, inv_s
+
+
+def sq_weight_colmax(w, amax_w, stream=None):
+    """amax_w[k] = max_n |W[n,k]| (the weight half of eq. (4)'s peaks)."""
+    N, K = w.shape
+    check(lib.sq_weight_colmax(_ptr(w), _dt(w), N, K, _ptr(amax_w), _stream(stream)),
+          "sq_weight_colmax")
+    return amax_w
+
+
+def sq_smooth_scales_peaks(amax_x, amax_w, alpha, s, inv_s, act_delta_static=None, stream=None):
+    """eq. (4) from both sets of peaks: s, 1/s (and the static step)."""
+    K = amax_x.numel()
+    check(lib.sq_smooth_scales_peaks(_ptr(amax_x), _ptr(amax_w), K, float(alpha), _ptr(s),
+                                     _ptr(inv_s), _ptr(act_delta_static), _stream(stream)),
+          "sq_smooth_scales_peaks")
     return s, inv_s
 
 

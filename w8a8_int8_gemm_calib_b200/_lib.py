@@ -37,6 +37,7 @@ EXPORTS = [
     "sq_selftest_bounded_wait", "sq_gemm_w8a8_noalloc", "sq_gemm_w8a8_bias",
     "sq_calib_absmax_rms", "sq_rms_smooth_quant_act", "sq_fold_into_producer",
     "sq_alpha_sweep_workspace_bytes", "sq_alpha_sweep", "sq_bmm_w8a8",
+    "sq_weight_colmax", "sq_smooth_scales_peaks",
 ]
 
 
@@ -57,6 +58,8 @@ def _load() -> ctypes.CDLL:
     L.sq_calib_absmax.argtypes = [p, i, i64, i64, p, p, f, p, p]
     L.sq_calib_absmax_rms.argtypes = [p, i, i64, i64, p, f, p, p]
     L.sq_fold_into_producer.argtypes = [p, i64, p, p, p]
+    L.sq_weight_colmax.argtypes = [p, i, i64, i64, p, p]
+    L.sq_smooth_scales_peaks.argtypes = [p, p, i64, f, p, p, p, p]
     L.sq_bmm_w8a8.argtypes = [p, p, i64, i64, i64, i64, p, i, p, i, p, i, p, p]
     L.sq_alpha_sweep_workspace_bytes.argtypes = [i64, i64, i64]
     L.sq_alpha_sweep_workspace_bytes.restype = sz
@@ -80,7 +83,7 @@ def _load() -> ctypes.CDLL:
                "sq_ln_smooth_quant_act", "sq_gemm_w8a8", "sq_sync_status",
                "sq_selftest_bounded_wait", "sq_gemm_w8a8_noalloc", "sq_gemm_w8a8_bias",
                "sq_calib_absmax_rms", "sq_rms_smooth_quant_act", "sq_fold_into_producer",
-               "sq_alpha_sweep", "sq_bmm_w8a8"):
+               "sq_alpha_sweep", "sq_bmm_w8a8", "sq_weight_colmax", "sq_smooth_scales_peaks"):
         getattr(L, fn).restype = st
     return L
 

@@ -126,7 +126,40 @@ sq_status sq_smooth_scales(const float* amax_x, const void* w, sq_dtype wt, int6
   // s first holds the weight column peaks (running max from 0)
   cudaError_t e = cudaMemsetAsync(s, 0, (size_t)K * sizeof(float), st);
   if (e == cudaSuccess && N > 0) e = launch_colmax(w, wt, N, K, s, st);
-  if (e == cudaSuccess) e = launch_scales(amax_x, K, alpha, s, inv_s, act_delta_static, st);
+  if (e == cudaSuccess) e = launch_scales(amax_x, s, K, alpha, s, inv_s, act_delta_static, st);
+  return e == cudaSuccess ? SQ_OK : cuda_fail(e, fn);
+}
+
+sq_status sq_weight_colmax(const void* w, sq_dtype wt, int64_t N, int64_t K, float* amax_w,
+                           sq_stream stream) {
+  const char* fn = "sq_weight_colmax";
+  g_last_error[0] = 0;
+  SQ_TRY(check_dtype(wt, fn));
+  if (N < 0) return fail(SQ_ERR_SHAPE, "%s: N=%lld < 0", fn, (long long)N);
+  SQ_TRY(check_k(K, fn));
+  SQ_REQ(amax_w, fn);
+  if (N > 0) SQ_REQ(w, fn);
+  cudaStream_t st = (cudaStream_t)stream;
+  cudaError_t e = cudaMemsetAsync(amax_w, 0, (size_t)K * sizeof(float), st);
+  if (e == cudaSuccess && N > 0) e = launch_colmax(w, wt, N, K, amax_w, st);
+  return e == cudaSuccess ? SQ_OK : cuda_fail(e, fn);
+}
+
+sq_status sq_smooth_scales_peaks(const float* amax_x, const float* amax_w, int64_t K, float alpha,
+                                 float* s, float* inv_s, float* act_delta_static,
+                                 sq_stream stream) {
+  const char* fn = "sq_smooth_scales_peaks";
+  g_last_error[0] = 0;
+  SQ_TRY(check_k(K, fn));
+  if (!(alpha >= 0.0f && alpha <= 1.0f))
+    return fail(SQ_ERR_INVALID_ARG, "%s: alpha=%g must lie in [0, 1]", fn, (double)alpha);
+  SQ_REQ(amax_x, fn);
+  SQ_REQ(amax_w, fn);
+  SQ_REQ(s, fn);
+  SQ_REQ(inv_s, fn);
+  SQ_OPT(act_delta_static, fn);
+  cudaError_t e = launch_scales(amax_x, amax_w, K, alpha, s, inv_s, act_delta_static,
+                                (cudaStream_t)stream);
   return e == cudaSuccess ? SQ_OK : cuda_fail(e, fn);
 }
 
@@ -452,9 +485,8 @@ sq_status sq_alpha_sweep(const float* amax_x, const void* w, sq_dtype wt, int64_
   cudaError_t e = cudaMemsetAsync(wmax, 0, 4 * (size_t)K, st);
   if (e == cudaSuccess) e = launch_colmax(w, wt, N, K, wmax, st);
   for (int i = 0; e == cudaSuccess && i < n_alpha; ++i) {
-    // eq. (4) (and the static step); scales_kernel reads the peaks from s
-    e = cudaMemcpyAsync(s, wmax, 4 * (size_t)K, cudaMemcpyDeviceToDevice, st);
-    if (e == cudaSuccess) e = launch_scales(amax_x, K, alphas[i], s, inv_s, stat ? dA : nullptr, st);
+    // eq. (4) (and the static step) from the two sets of peaks
+    e = launch_scales(amax_x, wmax, K, alphas[i], s, inv_s, stat ? dA : nullptr, st);
     // the fold: W * s -> wq, w_scale; gamma / s, beta / s
     RowArgs f{};
     f.x = w; f.T = N; f.K = K; f.mul = s; f.scale = ws; f.q = wq;

@@ -518,7 +518,7 @@ cudaError_t launch_row(const RowArgs& a, sq_dtype xt, RowMode mode, cudaStream_t
 constexpr int kScaleThreads = 256;
 
 __global__ void __launch_bounds__(kScaleThreads)
-scales_kernel(const float* __restrict__ amax_x, int64_t K, float alpha,
+scales_kernel(const float* __restrict__ amax_x, const float* amax_w, int64_t K, float alpha,
               float* s, float* __restrict__ inv_s, unsigned int* __restrict__ delta_out) {
   __shared__ float wmax[kScaleThreads / 32];
   pdl_launch_dependents();
@@ -528,7 +528,7 @@ scales_kernel(const float* __restrict__ amax_x, int64_t K, float alpha,
   for (int64_t k = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; k < K;
        k += (int64_t)gridDim.x * blockDim.x) {
     const float a = amax_x[k];
-    const float bw = fmaxf(s[k], 1e-7f);  // s holds the weight column peak on entry
+    const float bw = fmaxf(amax_w[k], 1e-7f);  // amax_w may be s itself (read before written)
     const double ad = (double)a, bd = (double)bw;
     double sd;
     if (alpha == 0.5f)
@@ -558,16 +558,16 @@ scales_kernel(const float* __restrict__ amax_x, int64_t K, float alpha,
   }
 }
 
-cudaError_t launch_scales(const float* amax_x, int64_t K, float alpha, float* s, float* inv_s,
-                          float* delta_out, cudaStream_t st) {
+cudaError_t launch_scales(const float* amax_x, const float* amax_w, int64_t K, float alpha,
+                          float* s, float* inv_s, float* delta_out, cudaStream_t st) {
   if (delta_out) {
     cudaError_t e = cudaMemsetAsync(delta_out, 0, sizeof(float), st);
     if (e != cudaSuccess) return e;
   }
   int64_t blocks = (K + kScaleThreads - 1) / kScaleThreads;
   if (blocks > 4 * (int64_t)sm_count()) blocks = 4 * (int64_t)sm_count();
-  return launch_pdl(scales_kernel, dim3((unsigned)blocks), dim3(kScaleThreads), 0, st, amax_x, K,
-                    alpha, s, inv_s, (unsigned int*)delta_out);
+  return launch_pdl(scales_kernel, dim3((unsigned)blocks), dim3(kScaleThreads), 0, st, amax_x,
+                    amax_w, K, alpha, s, inv_s, (unsigned int*)delta_out);
 }
 
 // ============================================================ per-tensor step

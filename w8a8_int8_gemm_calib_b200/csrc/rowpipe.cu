@@ -361,6 +361,12 @@ __global__ void __launch_bounds__(kThreads, NB) rowpipe_kernel(const Pipe P) {
     const int q = tid / ST, j = tid % ST;
     const int v = j >> 5, lane = j & 31;
     const float kf = (float)K;
+    // x / K for a power-of-two K is x * (1/K) exactly (both are the correctly
+    // rounded value of the same exact quotient): a multiply instead of a
+    // division subroutine
+    const bool k_pow2 = (K & (K - 1)) == 0;
+    const float kinv = 1.0f / kf;
+    auto divk = [&](float v) { return k_pow2 ? __fmul_rn(v, kinv) : __fdiv_rn(v, kf); };
     constexpr int NC = (MODE == ROW_COLMAX && CM > 0) ? CM * 8 : 1;
     float cmax[NC];
 #pragma unroll
@@ -507,7 +513,7 @@ __global__ void __launch_bounds__(kThreads, NB) rowpipe_kernel(const Pipe P) {
               p[m % G] = __fadd_rn(p[m % G], x[e].y);
             }
           });
-          mu = __fdiv_rn(slot_sum(p, 0), kf);
+          mu = divk(slot_sum(p, 0));
         }
         negmu2 = make_float2(-mu, -mu);
 #pragma unroll
@@ -520,7 +526,7 @@ __global__ void __launch_bounds__(kThreads, NB) rowpipe_kernel(const Pipe P) {
             p[m % G] = __fmaf_rn(x[e].y, x[e].y, p[m % G]);
           }
         });
-        const float rstd = __fdiv_rn(1.0f, __fsqrt_rn(__fadd_rn(__fdiv_rn(slot_sum(p, 1), kf), a.eps)));
+        const float rstd = __fdiv_rn(1.0f, __fsqrt_rn(__fadd_rn(divk(slot_sum(p, 1)), a.eps)));
         rstd2 = make_float2(rstd, rstd);
       }
       constexpr int kLvlIn = LN ? 1 : 0;  // level the y pass starts from

@@ -53,10 +53,10 @@ bool rowpipe_fits(int64_t K, sq_dtype xt, RowMode mode, bool ln);
 cudaError_t launch_rowpipe(const RowArgs& a, sq_dtype xt, RowMode mode,
                            cudaStream_t st);
 
-// s / inv_s from amax_x and the weight column peaks held (as fp32) in s.
-cudaError_t launch_scales(const float* amax_x, int64_t K, float alpha,
-                          float* s, float* inv_s, float* delta_out,
-                          cudaStream_t st);
+// s / inv_s (and the static step) from amax_x and the weight column peaks
+// amax_w (which may be s itself).
+cudaError_t launch_scales(const float* amax_x, const float* amax_w, int64_t K, float alpha,
+                          float* s, float* inv_s, float* delta_out, cudaStream_t st);
 
 // act_scale[0] = Delta(act_scale[0]) = max(peak, 1e-7) / 127 (one thread).
 cudaError_t launch_peak_to_delta(float* act_scale, cudaStream_t st);
