@@ -62,6 +62,30 @@ def test_bmm(sq, orc, B, M, N, K, out, per_token, per_channel):
     assert_bits_equal(y, y_want, "y")
 
 
+@pytest.mark.parametrize("B,M,N,K", [(3, 130, 200, 240), (3, 130, 200, 512),
+                                     (3, 130, 200, 528), (2, 1024, 2048, 64)])
+@pytest.mark.parametrize("out", ["f32", "bf16"])
+def test_bmm_short_k_epilogue(sq, orc, B, M, N, K, out):
+    """Head-sized K: three epilogue warps per accumulator quarter up to four
+    k-blocks (K = 528 is back on one), with the largest accumulators the
+    codes allow beside random rows.  130 x 200 per batch picks the
+    128-column tile (four chunks over three warps), 1024 x 2048 the
+    256-column one."""
+    r = np.random.default_rng(K + M)
+    xq = r.integers(-128, 128, (B, M, K)).astype(np.int8)
+    wq = r.integers(-128, 128, (B, N, K)).astype(np.int8)
+    xq[:, :2] = -128
+    wq[:, :2] = -128
+    wq[1, 5] = 127
+    act = r.uniform(1e-3, 0.1, B * M).astype(np.float32)
+    ws = r.uniform(1e-4, 1e-2, B).astype(np.float32)
+    y_want, acc_want = orc.bmm_w8a8(xq, wq, act, ws, True, False, out_bf16=(out == "bf16"))
+    y, acc = _run(sq, xq, wq, act, ws, True, False, out)
+    assert acc[0, 0, 0] == K * 16384 and acc[1, 0, 5] == -K * 16256
+    assert_bits_equal(acc, acc_want, "acc")
+    assert_bits_equal(y, y_want, "y")
+
+
 def test_bmm_attention_sizes_match_per_batch_gemm(sq):
     """OPT-6.7B-shaped attention (32 heads, 2048 tokens, head dimension 128):
     one batched launch equals 32 separate GEMM calls, bit for bit, for the

@@ -84,6 +84,29 @@ def test_gemm_extremes(sq, orc):
     assert_bits_equal(y, y_want, "y")
 
 
+@pytest.mark.parametrize("M,N,K", [(200, 264, 240), (200, 264, 512), (200, 264, 528),
+                                   (2048, 2048, 128)])
+def test_gemm_short_k_epilogue(sq, orc, M, N, K):
+    """Short K (at most four 128-byte k-blocks) runs the epilogue on three
+    warps per accumulator quarter, each taking every third 32-column chunk;
+    K = 528 is the first width back on one warp per quarter.  The largest
+    accumulators the codes allow (-128 x -128 x K) sit beside random rows.
+    2048 x 2048 picks the 256-column tile, the others the 192-column one."""
+    r = np.random.default_rng(K + N)
+    xq = r.integers(-128, 128, (M, K)).astype(np.int8)
+    wq = r.integers(-128, 128, (N, K)).astype(np.int8)
+    xq[:3] = -128
+    wq[:2] = -128
+    wq[2] = 127
+    act = r.uniform(1e-3, 0.1, M).astype(np.float32)
+    ws = r.uniform(1e-4, 1e-2, N).astype(np.float32)
+    y_want, acc_want = orc.gemm_w8a8(xq, wq, act, ws, out_bf16=True)
+    y, acc = _run(sq, xq, wq, act, ws, True, "bf16", workspace=sq.Workspace())
+    assert acc[0, 0] == K * 16384 and acc[0, 2] == -K * 16256
+    assert_bits_equal(acc, acc_want, "acc")
+    assert_bits_equal(y, y_want, "y")
+
+
 def test_gemm_without_acc_dump(sq, orc):
     M, N, K = 300, 520, 1024
     xq, wq, act, ws = _operands(M, N, K, 5)

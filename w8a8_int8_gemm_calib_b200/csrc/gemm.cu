@@ -15,7 +15,8 @@
 // K steps, a 4-stage TMA ring, and two TMEM accumulators (2 x 256 columns) so
 // the epilogue of one tile overlaps the main loop of the next.  Warp roles:
 // warp 0 issues TMA loads, warp 1 issues the MMAs (one elected thread), warps
-// 2-5 drain TMEM, dequantize and store.  Every mbarrier wait is bounded.
+// 2-5 drain TMEM, dequantize and store (warps 2-13 when K is short and the
+// epilogue sets the pace).  Every mbarrier wait is bounded.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 #include <cuda_bf16.h>
@@ -38,7 +39,7 @@ constexpr int BM = 128;     // token rows per tile (MMA M)
 constexpr int BK = 128;     // bytes of K per stage = one 128B swizzle row
 constexpr int UK = 32;      // K per tcgen05.mma kind::i8
 constexpr int A_BYTES = BM * BK;
-constexpr int THREADS = 192;
+constexpr int THREADS = 192;  // small-M kernel: TMA, MMA and 4 epilogue warps
 constexpr int GROUP_M = 16;  // tile raster: 16 row blocks share each column sweep
 constexpr uint64_t kWaitNs = 4000000000ull;   // 4 s: far above any pipeline step
 constexpr uint64_t kDrainNs = 1000000000ull;  // waits for copies already in flight
@@ -50,14 +51,19 @@ constexpr int EPI_BUF = 32 * 64;
 // the host picks the one that fills the last wave of SMs best.  EPI_NB
 // output staging buffers per epilogue warp (EPI_NB - 1 TMA stores in flight
 // per warp; deeper staging was measured not to speed up output-bound
-// shapes, whose epilogue is latency-bound instead).
-template <int TBN, int EPI_NB = 2>
+// shapes).  EPI_W epilogue warps, 4 or 12: with 12, three warps share each
+// 32-lane quarter of the accumulator and take every third 32-column chunk,
+// for short K, where the epilogue and not the main loop sets the tile time
+// and one warp per quarter leaves it latency-bound.
+template <int TBN, int EPI_NB = 2, int EPI_W = 4>
 struct TcCfg {
+  static_assert(EPI_W == 4 || EPI_W == 12, "one or three warps per accumulator quarter");
+  static constexpr int THREADS = 64 + 32 * EPI_W;  // TMA warp, MMA warp, epilogue
   static constexpr int B_BYTES = TBN * BK;
   static constexpr int STAGE = A_BYTES + B_BYTES;
-  static constexpr int EPI_BYTES = 4 * EPI_NB * EPI_BUF;
-  // as many stages as fit: with 2 staging buffers 4 at 256 columns, 5 at
-  // 192, 6 at 128
+  static constexpr int EPI_BYTES = EPI_W * EPI_NB * EPI_BUF;
+  // as many stages as fit: with 4 epilogue warps of 2 staging buffers, 4 at
+  // 256 columns, 5 at 192, 6 at 128
   static constexpr int STAGES = (224 * 1024 - 2048 - EPI_BYTES) / STAGE;
   static constexpr uint32_t TMEM_COLS = 2 * TBN <= 256 ? 256 : 512;  // power of two
   static constexpr size_t SMEM = 1024 + (size_t)STAGES * STAGE + EPI_BYTES + 256;
@@ -188,11 +194,11 @@ __device__ __forceinline__ void store_chunk(const Params& p, size_t yrow, int co
   }
 }
 
-template <bool BF16, int TBN, bool BATCH, int EPI_NB>
-__global__ void __launch_bounds__(THREADS, 1)
+template <bool BF16, int TBN, bool BATCH, int EPI_NB, int EPI_W>
+__global__ void __launch_bounds__(TcCfg<TBN, EPI_NB, EPI_W>::THREADS, 1)
 gemm_w8a8_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                     const __grid_constant__ CUtensorMap tmY, const Params p) {
-  using C = TcCfg<TBN, EPI_NB>;
+  using C = TcCfg<TBN, EPI_NB, EPI_W>;
   constexpr int STAGES = C::STAGES;
   constexpr int B_BYTES = C::B_BYTES;
   constexpr int STAGE_BYTES = C::STAGE;
@@ -223,7 +229,7 @@ gemm_w8a8_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
     }
     for (int b = 0; b < 2; ++b) {
       tc::mbar_init(tfull_bar(b), 1);
-      tc::mbar_init(tempty_bar(b), 4);  // one arrival per epilogue warp
+      tc::mbar_init(tempty_bar(b), EPI_W);  // one arrival per epilogue warp
     }
     tc::mbar_init(drain_bar, 1);
     *abort_flag = 0;
@@ -323,6 +329,7 @@ gemm_w8a8_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
   } else {
     // ------------------------------------------------------------ epilogue
     const int quarter = warp & 3;  // this warp may read TMEM lanes 32*quarter..+31
+    const int chunk0 = (warp - 2) >> 2;  // first of this warp's 32-column chunks
     uint8_t* ebuf = sEpi + (warp - 2) * EPI_NB * EPI_BUF;
     uint32_t nstore = 0;  // TMA stores issued by this warp (selects the buffer)
     uint32_t abuf = 0, aphase = 0;
@@ -340,7 +347,7 @@ gemm_w8a8_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
                                    : __ldg(p.act_scale + b);
       const uint32_t taddr = tmem_base + abuf * BN + ((uint32_t)(quarter * 32) << 16);
 #pragma unroll 1
-      for (int c = 0; c < BN / 32; ++c) {
+      for (int c = chunk0; c < BN / 32; c += EPI_W / 4) {
         uint32_t r[32];
         tc::tmem_ld32(taddr + c * 32, r);
         tc::tmem_ld_wait();
@@ -794,23 +801,23 @@ bool make_tmap_out3(CUtensorMap* m, void* base, uint64_t cols, uint64_t rows, ui
   return r == CUDA_SUCCESS;
 }
 
-template <bool BF16, int TBN, bool BATCH = false, int EPI_NB = 2>
+template <bool BF16, int TBN, bool BATCH = false, int EPI_NB = 2, int EPI_W = 4>
 cudaError_t launch_tc(const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& ty,
                       const Params& p, int grid, cudaStream_t st) {
-  using C = TcCfg<TBN, EPI_NB>;
+  using C = TcCfg<TBN, EPI_NB, EPI_W>;
   static std::once_flag once[64];
   static cudaError_t attr_err[64];
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess || dev < 0 || dev >= 64) return e != cudaSuccess ? e : cudaErrorInvalidDevice;
   std::call_once(once[dev], [&] {
-    attr_err[dev] = cudaFuncSetAttribute(gemm_w8a8_tc_kernel<BF16, TBN, BATCH, EPI_NB>,
+    attr_err[dev] = cudaFuncSetAttribute(gemm_w8a8_tc_kernel<BF16, TBN, BATCH, EPI_NB, EPI_W>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)C::SMEM);
   });
   if (attr_err[dev] != cudaSuccess) return attr_err[dev];
-  return launch_pdl(gemm_w8a8_tc_kernel<BF16, TBN, BATCH, EPI_NB>, dim3(grid), dim3(THREADS),
-                    C::SMEM, st, ta, tb, ty, p);
+  return launch_pdl(gemm_w8a8_tc_kernel<BF16, TBN, BATCH, EPI_NB, EPI_W>, dim3(grid),
+                    dim3(C::THREADS), C::SMEM, st, ta, tb, ty, p);
 }
 
 // Tile width for the large-M kernel: the per-tile time grows with the width,
@@ -830,6 +837,33 @@ int pick_tile_n(int64_t M, int64_t N, int sms, int64_t batch = 1, bool narrow = 
   return best;
 }
 
+
+// The large-M kernel for a tile width, output type and epilogue width (the
+// 128-column tiles are only picked for batched calls).  Short K (at most
+// four k-blocks) takes 12 epilogue warps: there a tile's main loop is a few
+// MMAs and the epilogue sets the pace.
+template <bool BATCH>
+cudaError_t launch_tiles(const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& ty,
+                         const Params& p, int grid, int tbn, bool bf16, cudaStream_t st) {
+  if (p.nk <= 4) {
+    if (tbn == 256) return bf16 ? launch_tc<true, 256, BATCH, 2, 12>(ta, tb, ty, p, grid, st)
+                                : launch_tc<false, 256, BATCH, 2, 12>(ta, tb, ty, p, grid, st);
+    if (tbn == 192) return bf16 ? launch_tc<true, 192, BATCH, 2, 12>(ta, tb, ty, p, grid, st)
+                                : launch_tc<false, 192, BATCH, 2, 12>(ta, tb, ty, p, grid, st);
+    if constexpr (BATCH)
+      return bf16 ? launch_tc<true, 128, BATCH, 2, 12>(ta, tb, ty, p, grid, st)
+                  : launch_tc<false, 128, BATCH, 2, 12>(ta, tb, ty, p, grid, st);
+  } else {
+    if (tbn == 256) return bf16 ? launch_tc<true, 256, BATCH>(ta, tb, ty, p, grid, st)
+                                : launch_tc<false, 256, BATCH>(ta, tb, ty, p, grid, st);
+    if (tbn == 192) return bf16 ? launch_tc<true, 192, BATCH>(ta, tb, ty, p, grid, st)
+                                : launch_tc<false, 192, BATCH>(ta, tb, ty, p, grid, st);
+    if constexpr (BATCH)
+      return bf16 ? launch_tc<true, 128, BATCH>(ta, tb, ty, p, grid, st)
+                  : launch_tc<false, 128, BATCH>(ta, tb, ty, p, grid, st);
+  }
+  return cudaErrorInvalidValue;
+}
 
 constexpr int64_t kSmallMaxM = 128;
 
@@ -986,10 +1020,7 @@ sq_status launch_gemm(const GemmArgs& a, cudaStream_t st) {
                 make_tmap_out(&ty, a.y, (uint64_t)a.N, (uint64_t)a.M, bf16);
   int grid = sm_count();
   if (grid > p.num_tiles) grid = p.num_tiles;
-  cudaError_t e = tbn == 256 ? (bf16 ? launch_tc<true, 256>(ta, tb, ty, p, grid, st)
-                                     : launch_tc<false, 256>(ta, tb, ty, p, grid, st))
-                              : (bf16 ? launch_tc<true, 192>(ta, tb, ty, p, grid, st)
-                                      : launch_tc<false, 192>(ta, tb, ty, p, grid, st));
+  const cudaError_t e = launch_tiles<false>(ta, tb, ty, p, grid, tbn, bf16, st);
   if (e != cudaSuccess) return fail(SQ_ERR_CUDA, "sq_gemm_w8a8: %s", cudaGetErrorString(e));
   return SQ_OK;
 }
@@ -1025,13 +1056,7 @@ sq_status launch_bmm(const BmmArgs& a, cudaStream_t st) {
                 make_tmap_out3(&ty, a.y, (uint64_t)a.N, (uint64_t)a.M, (uint64_t)a.batch, bf16);
   int grid = sms;
   if (grid > p.num_tiles) grid = p.num_tiles;
-  cudaError_t e;
-  if (tbn == 256) e = bf16 ? launch_tc<true, 256, true>(ta, tb, ty, p, grid, st)
-                           : launch_tc<false, 256, true>(ta, tb, ty, p, grid, st);
-  else if (tbn == 192) e = bf16 ? launch_tc<true, 192, true>(ta, tb, ty, p, grid, st)
-                                : launch_tc<false, 192, true>(ta, tb, ty, p, grid, st);
-  else e = bf16 ? launch_tc<true, 128, true>(ta, tb, ty, p, grid, st)
-                : launch_tc<false, 128, true>(ta, tb, ty, p, grid, st);
+  const cudaError_t e = launch_tiles<true>(ta, tb, ty, p, grid, tbn, bf16, st);
   if (e != cudaSuccess) return fail(SQ_ERR_CUDA, "sq_bmm_w8a8: %s", cudaGetErrorString(e));
   return SQ_OK;
 }
