@@ -586,8 +586,8 @@ cudaError_t launch_peak_to_delta(float* act_scale, cudaStream_t st) {
 // ============================================================ output error
 // sum (y - r)^2 and sum r^2 in fp64, deterministic: each thread accumulates
 // a grid-stride share, warps and blocks reduce, each block writes its two
-// partial sums to its own slot, and one thread adds the slots in block
-// order.
+// partial sums to its own slot, and one block adds the slots in a fixed
+// order (a strided share per thread, then a halving tree).
 constexpr int kErrThreads = 256;
 
 int output_error_blocks(int64_t n) {
@@ -638,15 +638,32 @@ output_error_kernel(const float* __restrict__ y, const float* __restrict__ r, in
   }
 }
 
-__global__ void output_error_final_kernel(const double* part, int nblocks, double* err) {
+// One block of kErrThreads: the slots are read in parallel (a single thread
+// walking them would wait out one memory latency after another).
+__global__ void __launch_bounds__(kErrThreads)
+output_error_final_kernel(const double* part, int nblocks, double* err) {
+  __shared__ double s[2][kErrThreads];
   pdl_launch_dependents();
   pdl_wait();
-  if (threadIdx.x == 0) {
-    double num = 0.0, den = 0.0;
-    for (int i = 0; i < nblocks; ++i) {
-      num += part[2 * i];
-      den += part[2 * i + 1];
+  const int t = threadIdx.x;
+  double num = 0.0, den = 0.0;
+  for (int i = t; i < nblocks; i += kErrThreads) {
+    num += part[2 * i];
+    den += part[2 * i + 1];
+  }
+  s[0][t] = num;
+  s[1][t] = den;
+  __syncthreads();
+  for (int h = kErrThreads / 2; h > 0; h >>= 1) {
+    if (t < h) {
+      s[0][t] += s[0][t + h];
+      s[1][t] += s[1][t + h];
     }
+    __syncthreads();
+  }
+  if (t == 0) {
+    num = s[0][0];
+    den = s[1][0];
     *err = den > 0.0 ? sqrt(num / den) : (num > 0.0 ? (double)INFINITY : 0.0);
   }
 }
@@ -657,7 +674,7 @@ cudaError_t launch_output_error(const float* y, const float* y_ref, int64_t n, d
   cudaError_t e = launch_pdl(output_error_kernel, dim3((unsigned)blocks), dim3(kErrThreads), 0,
                              st, y, y_ref, n, scratch);
   if (e != cudaSuccess) return e;
-  return launch_pdl(output_error_final_kernel, dim3(1), dim3(32), 0, st,
+  return launch_pdl(output_error_final_kernel, dim3(1), dim3(kErrThreads), 0, st,
                     (const double*)scratch, blocks, err);
 }
 
