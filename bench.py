@@ -437,7 +437,8 @@ def run_small_m(sq, torch, dev, flush, reps=20):
     ws = torch.rand(N, device=dev, generator=g) * 1e-3 + 1e-5
     hbm = load_peaks()[0].get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"])
     out = {"workload": "175b_fc1_decode: fc1 12288->49152, per-token, bf16 out",
-           "kernel": "gemm_w8a8 weight-streaming path (tcgen05 kind::i8, stream-K)",
+           "kernel": "gemm_w8a8 (tcgen05 kind::i8): stream-K weight streaming up to 8 tokens, "
+                     "the persistent 128-row-tile kernel beyond (its 256 tiles fill the SMs)",
            "hbm_peak_gbs": hbm}
     for M in (1, 8, 32, 128):
         xq = torch.randint(-127, 128, (M, K), dtype=torch.int8, device=dev, generator=g)
@@ -464,7 +465,8 @@ def run_small_m(sq, torch, dev, flush, reps=20):
         nbytes = M * K + N * K + M * N * 2 + 4 * N + 4 * M
         gbs = nbytes / (ms * 1e-3) / 1e9
         out[f"M{M}"] = {"us": round(ms * 1e3, 2), "gbs": round(gbs, 1),
-                        "hbm_frac": round(gbs / hbm, 3), "bytes": int(nbytes)}
+                        "hbm_frac": round(gbs / hbm, 3), "bytes": int(nbytes),
+                        "path": "stream-K" if sq.sq_gemm_workspace_bytes(M, N, K) else "tiles"}
         del graph
     return out
 

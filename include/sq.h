@@ -255,11 +255,13 @@ sq_status sq_rms_smooth_quant_act(const void* x, sq_dtype xt, int64_t T,
 
 /*
  * sq_gemm_workspace_bytes -- device scratch sq_gemm_w8a8 needs for this
- * shape on the current device (0 when it needs none).  Problems with
- * M <= 128 tokens take the weight-streaming path, which splits the K loop of
- * a weight tile across SMs and reduces the exact INT32 partial tiles in the
- * workspace: 256 bytes per 128 output channels (rounded up to 256) plus
- * 2 * M * 128 * 4 bytes per SM used.
+ * shape on the current device (0 when it needs none).  Problems of up to 8
+ * tokens, and of up to 128 tokens whose output is too narrow for 128-row
+ * tiles to give every SM one (N / 192 or N / 256 below the SM count), take
+ * the stream-K weight-streaming path.  It splits the K loop of a weight tile
+ * across SMs and reduces the exact INT32 partial tiles in the workspace:
+ * 256 bytes per 128 output channels (rounded up to 256) plus
+ * 2 * M * 128 * 4 bytes per SM used.  Every other shape needs none.
  */
 size_t sq_gemm_workspace_bytes(int64_t M, int64_t N, int64_t K);
 
@@ -316,14 +318,14 @@ sq_status sq_gemm_w8a8_bias(const int8_t* xq, const int8_t* wq, int64_t M,
  * step receives only its inputs and outputs.  This entry point takes the
  * same arguments as sq_gemm_w8a8 minus the workspace and allocates nothing
  * (no cudaMalloc/cudaFree, no allocating library routine): the scratch the
- * M <= 128 path needs lives in a fixed array of 8 MiB (8,388,608 bytes) of
+ * stream-K path needs lives in a fixed array of 8 MiB (8,388,608 bytes) of
  * device memory that the library reserves on every GPU that loads it, held
  * until the process exits.
  *
  *   - Shapes whose sq_gemm_workspace_bytes(M,N,K) exceeds 8 MiB are refused
  *     with SQ_ERR_WORKSPACE before anything is launched (at 148 SMs that is
- *     roughly M > 52 tokens on the M <= 128 path); M > 128 needs no scratch
- *     and is always served.
+ *     roughly M > 52 tokens on the stream-K path); shapes off that path need
+ *     no scratch and are always served.
  *   - The first call on a device looks up the array's device address with
  *     cudaGetSymbolAddress, so make that first call before any stream capture
  *     begins on that device.

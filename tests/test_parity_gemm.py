@@ -126,13 +126,17 @@ def test_gemm_is_deterministic(sq):
 
 
 # ---------------------------------------------------------------- small M
-# M <= 128 takes the weight-streaming kernel: tokens padded to 8/16/32/64/128
-# as the MMA N dimension, (tile, k-block) units split evenly over the SMs,
-# partial tiles summed exactly by the last CTA to arrive.
+# Up to 8 tokens, and up to 128 on outputs too narrow for the large-M tiles
+# to fill the SMs, take the stream-K weight-streaming kernel: tokens padded to
+# 8/16/32/64/128 as the MMA N dimension, (tile, k-block) units split evenly
+# over the SMs, partial tiles summed exactly by the last CTA to arrive.  The
+# wide outputs below (49152 and 57344 columns at 9 to 128 tokens) run the
+# large-M kernel with a single, mostly padded, 128-row block.
 SMALL_SHAPES = [
     (1, 130, 16), (2, 1000, 12288), (8, 4096, 2064), (9, 300, 4096), (16, 2048, 1040),
     (17, 777, 8192), (32, 1024, 6144), (33, 260, 144), (64, 3000, 2048), (100, 1536, 4096),
-    (128, 512, 12288), (128, 49152, 256), (5, 128, 20480),
+    (128, 512, 12288), (128, 49152, 256), (5, 128, 20480), (16, 49152, 512),
+    (12, 57344, 384), (8, 49152, 384),
 ]
 
 
@@ -159,6 +163,19 @@ def test_gemm_small_m_workspace_reuse(sq, orc):
         y, acc = _run(sq, xq, wq, act, ws, True, "bf16", workspace=wsbuf)
         assert_bits_equal(acc, acc_want, "acc reuse")
         assert_bits_equal(y, y_want, "y reuse")
+
+
+def test_gemm_decode_path_choice(sq):
+    """Which decode shapes need the stream-K scratch: up to 8 tokens always;
+    9 to 128 tokens only while the large-M tiles across N would not give
+    every SM one; more than 128 never."""
+    sms = torch.cuda.get_device_properties(0).multi_processor_count
+    assert sq.sq_gemm_workspace_bytes(8, 49152, 12288) > 0
+    assert sq.sq_gemm_workspace_bytes(16, 49152, 12288) == 0  # 256 tiles of 192
+    assert sq.sq_gemm_workspace_bytes(128, 49152, 12288) == 0
+    assert sq.sq_gemm_workspace_bytes(128, 12288, 12288) > 0  # 64 tiles
+    assert sq.sq_gemm_workspace_bytes(16, 192 * (sms - 1), 4096) > 0
+    assert sq.sq_gemm_workspace_bytes(129, 512, 4096) == 0
 
 
 def test_gemm_small_m_rejects_short_workspace(sq):

@@ -75,8 +75,10 @@ def test_noalloc_matches_workspace_entry_point(sq, M, N, K, out):
 
 def test_noalloc_refuses_shapes_beyond_its_scratch(sq):
     """A shape whose scratch exceeds the 8 MiB array is refused before any
-    launch, with a message that names the sizes."""
-    M, N, K = 128, 49152, 12288
+    launch, with a message that names the sizes (128 tokens on a 12288-wide
+    output: 64 large-M tiles would not fill the SMs, so it stays on the
+    stream-K path and its scratch)."""
+    M, N, K = 128, 12288, 12288
     assert sq.sq_gemm_workspace_bytes(M, N, K) > STATIC_SCRATCH_BYTES
     xq, wq, act, ws = _inputs(M, N, 256, 7)[0], None, None, None
     xq = torch.zeros((M, K), dtype=torch.int8, device="cuda")
