@@ -193,8 +193,9 @@ class Layer:
         self.y = torch.empty((M, N), dtype=io, device=dev)
         self.workspace = sq.Workspace(dev)
         # this library's kernels per step: calibration peak; column peak +
-        # eq. (4) factors; weight fold (+ LayerNorm fold); quantizer; GEMM
-        self.kernels_per_step = 7 if lin.ln else 6
+        # eq. (4) factors; weight fold (which also divides gamma and beta by
+        # s); quantizer; GEMM
+        self.kernels_per_step = 6
 
     def step(self, ev=None, upto=5):
         """The first `upto` of the five calls (all five: one step); ev = (start,
@@ -316,7 +317,7 @@ def run_ours(args):
             layer.step(ev, upto)
         return g, ev
 
-    # the timed graph: one whole step (five calls, seven kernels), event
+    # the timed graph: one whole step (five calls, six kernels), event
     # nodes only at its two ends
     graph, ev_step = capture(5)
     for _ in range(max(3, args.warmup)):

@@ -183,17 +183,20 @@ sq_status sq_fuse_weights_q8(const void* w, sq_dtype wt, int64_t N, int64_t K, c
   }
   cudaStream_t st = (cudaStream_t)stream;
   cudaError_t e = cudaSuccess;
+  const bool fold_g = gamma && gamma_out, fold_b = beta && beta_out;
   if (N > 0) {
     // W_hat = W * s, then per-row (output channel) dynamic INT8: the same
-    // row quantizer as the activations, with s as the column multiplier
+    // row quantizer as the activations, with s as the column multiplier.
+    // The same launch divides gamma and beta by s (no kernel of its own).
     RowArgs a{};
     a.x = w; a.T = N; a.K = K; a.mul = s; a.scale = w_scale; a.q = wq;
+    a.fold_g = gamma; a.fold_g_out = fold_g ? gamma_out : nullptr;
+    a.fold_b = beta; a.fold_b_out = fold_b ? beta_out : nullptr;
     e = launch_row(a, wt, ROW_DYNAMIC, st);
-  }
-  const bool fold_g = gamma && gamma_out, fold_b = beta && beta_out;
-  if (e == cudaSuccess && (fold_g || fold_b))
+  } else if (fold_g || fold_b) {
     e = launch_fold_ln(gamma, beta, s, K, fold_g ? gamma_out : nullptr,
                        fold_b ? beta_out : nullptr, st);
+  }
   return e == cudaSuccess ? SQ_OK : cuda_fail(e, fn);
 }
 
@@ -487,12 +490,14 @@ sq_status sq_alpha_sweep(const float* amax_x, const void* w, sq_dtype wt, int64_
   for (int i = 0; e == cudaSuccess && i < n_alpha; ++i) {
     // eq. (4) (and the static step) from the two sets of peaks
     e = launch_scales(amax_x, wmax, K, alphas[i], s, inv_s, stat ? dA : nullptr, st);
-    // the fold: W * s -> wq, w_scale; gamma / s, beta / s
+    // the fold: W * s -> wq, w_scale; gamma / s, beta / s in the same launch
     RowArgs f{};
     f.x = w; f.T = N; f.K = K; f.mul = s; f.scale = ws; f.q = wq;
+    if (ln_gamma) {
+      f.fold_g = ln_gamma; f.fold_g_out = g2;
+      f.fold_b = ln_beta; f.fold_b_out = ln_beta ? b2 : nullptr;
+    }
     if (e == cudaSuccess) e = launch_row(f, wt, ROW_DYNAMIC, st);
-    if (e == cudaSuccess && ln_gamma)
-      e = launch_fold_ln(ln_gamma, ln_beta, s, K, g2, ln_beta ? b2 : nullptr, st);
     // the quantizer
     RowArgs q{};
     q.x = x; q.T = M; q.K = K; q.eps = ln_eps; q.scale = act; q.q = xq;

@@ -210,6 +210,9 @@ row_kernel(RowArgs a) {
   extern __shared__ unsigned int colmax_s[];  // ROW_COLMAX: per-CTA column peaks [K]
   pdl_launch_dependents();
   pdl_wait();
+  if constexpr (!LN)
+    fold_columns(a.mul, a.fold_g, a.fold_b, a.fold_g_out, a.fold_b_out, a.K, threadIdx.x,
+                 blockDim.x);
 
   uint32_t dyn_smem;
   asm("mov.u32 %0, %%dynamic_smem_size;" : "=r"(dyn_smem));

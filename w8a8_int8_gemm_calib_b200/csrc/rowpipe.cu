@@ -356,6 +356,8 @@ __global__ void __launch_bounds__(kThreads, NB) rowpipe_kernel(const Pipe P) {
   } else {
     // ------------------------------------------------------------ consumers
     stage_params<LN>(a, pg, pb, MODE == ROW_COLMAX ? colmax_s : nullptr, (int)K, tid);
+    if constexpr (!LN)
+      fold_columns(a.mul, a.fold_g, a.fold_b, a.fold_g_out, a.fold_b_out, K, tid, kConsumers);
     asm volatile("bar.sync 9, %0;" ::"r"(kConsumers) : "memory");  // consumers only
 
     const int q = tid / ST, j = tid % ST;

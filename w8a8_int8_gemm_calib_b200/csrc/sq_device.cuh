@@ -81,6 +81,20 @@ __device__ __forceinline__ uint32_t pack4(int a, int b, int c, int d) {
   return __byte_perm(lo, hi, 0x5410);
 }
 
+// g_out = g / s and b_out = b / s over columns [0, K) (either output may be
+// NULL), this CTA's share with nt threads: the LayerNorm fold that rides
+// along with the weight fold, one IEEE fp32 division per element.
+__device__ __forceinline__ void fold_columns(const float* s, const float* g, const float* b,
+                                             float* g_out, float* b_out, int64_t K, int t,
+                                             int nt) {
+  if (!g_out && !b_out) return;
+  for (int64_t k = (int64_t)blockIdx.x * nt + t; k < K; k += (int64_t)gridDim.x * nt) {
+    const float sk = s[k];
+    if (g_out) g_out[k] = __fdiv_rn(g[k], sk);
+    if (b_out) b_out[k] = __fdiv_rn(b[k], sk);
+  }
+}
+
 // Bounded-wait clock: nanoseconds from the global timer.
 __device__ __forceinline__ uint64_t global_ns() {
   uint64_t t;

@@ -42,6 +42,13 @@ struct RowArgs {
   unsigned long long* n_clipped;  // may be NULL
   float* colmax;       // ROW_COLMAX: running max [K] (fp32 bits, atomic max)
   float* peak;         // ROW_PEAK: running peak [1] (fp32 bits, atomic max)
+  // With mul (the weight fold): also fold_g_out = fold_g / mul and
+  // fold_b_out = fold_b / mul over the K columns, shared out among the
+  // launch's CTAs (each output NULL to skip it)
+  const float* fold_g;
+  const float* fold_b;
+  float* fold_g_out;
+  float* fold_b_out;
 };
 
 cudaError_t launch_row(const RowArgs& a, sq_dtype xt, RowMode mode,
