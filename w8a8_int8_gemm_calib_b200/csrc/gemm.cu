@@ -506,8 +506,8 @@ __device__ __forceinline__ void small_store(const SmallParams& p, int n, int t0,
 __device__ __forceinline__ void epi_bar() {
   asm volatile("bar.sync 1, 128;" ::: "memory");
 }
-// AND of v over the 128 epilogue threads (also a barrier among them), so
-// that all four epilogue warps take the same branch
+// AND of v over the 128 epilogue threads of the small-M kernel (also a
+// barrier among them), so that its four epilogue warps take the same branch
 __device__ __forceinline__ bool epi_and(bool v) {
   uint32_t r;
   asm volatile(

@@ -705,7 +705,9 @@ cudaError_t launch_fold_producer(const float* s, int64_t K, float* w_scale, floa
 }
 
 // ============================================================ LayerNorm fold
-// gamma' = gamma / s, beta' = beta / s ([embedded] §二), fp32 division.
+// gamma' = gamma / s, beta' = beta / s ([embedded] §二), fp32 division.  The
+// weight fold's row kernel does this itself; this kernel serves calls with
+// no weight rows.
 __global__ void fold_ln_kernel(const float* __restrict__ gamma, const float* __restrict__ beta,
                                const float* __restrict__ s, int64_t K,
                                float* __restrict__ gamma_out, float* __restrict__ beta_out) {
