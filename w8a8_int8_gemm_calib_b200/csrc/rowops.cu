@@ -573,6 +573,24 @@ cudaError_t launch_scales(const float* amax_x, const float* amax_w, int64_t K, f
                     amax_w, K, alpha, s, inv_s, (unsigned int*)delta_out);
 }
 
+// ============================================================ zero fill
+__global__ void __launch_bounds__(256) zero_kernel(uint32_t* p, int64_t n) {
+  pdl_launch_dependents();
+  pdl_wait();
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n;
+       i += (int64_t)gridDim.x * blockDim.x)
+    p[i] = 0u;
+}
+
+cudaError_t launch_zero(void* p, size_t bytes, cudaStream_t st) {
+  if (bytes % 4 != 0) return cudaErrorInvalidValue;
+  const int64_t n = (int64_t)(bytes / 4);
+  if (n == 0) return cudaSuccess;
+  int64_t blocks = (n + 255) / 256;
+  if (blocks > 4 * (int64_t)sm_count()) blocks = 4 * (int64_t)sm_count();
+  return launch_pdl(zero_kernel, dim3((unsigned)blocks), dim3(256), 0, st, (uint32_t*)p, n);
+}
+
 // ============================================================ per-tensor step
 // The second step of per-tensor dynamic quantization: the peak folded into
 // act_scale[0] by the ROW_PEAK pass becomes Delta = max(peak, 1e-7) / 127.

@@ -9,6 +9,14 @@
 
 namespace sq {
 
+// Zero `bytes` (a multiple of 4) at p with a kernel launched like every
+// other one of this library (programmatic dependent launch), so that the
+// kernel after it can overlap its launch, which a memset node prevents.
+// Measured faster only where the next kernel is a short pass (the
+// per-tensor step's reset); ahead of the weight column peaks a memset
+// measured faster, so those keep it.
+cudaError_t launch_zero(void* p, size_t bytes, cudaStream_t st);
+
 // Device address of the per-device status word (a static __device__
 // variable in status.cu), looked up once per device.  NULL on failure.
 unsigned int* status_word();
