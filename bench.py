@@ -541,9 +541,10 @@ def time_call(torch, call, flush, reps=20):
 
 def run_alpha_sweep(sq, torch, layer, lin, flush, alphas=(0.0, 0.25, 0.5, 0.75, 1.0)):
     """alpha chosen by the layer's output error (NEXT-2): the whole smoothed
-    layer at five alphas on the step's tokens (eq. (4), fold, quantizer,
-    GEMM in fp32, fp64 error), against the unquantized layer in fp32 (the
-    reference is computed once with torch, outside the timing)."""
+    layer at five alphas on the step's tokens (eq. (4), fold, quantizer, and
+    the GEMM with the fp64 error sums in its epilogue), against the
+    unquantized layer in fp32 (the reference is computed once with torch,
+    outside the timing)."""
     import torch.nn.functional as F
 
     xf = layer.x.float()

@@ -5,6 +5,8 @@ compared with the oracle's same chain.  The layer outputs are bit-exact for
 alpha in {0, 0.5, 1}, so the errors agree to the fp64 summation order; for
 other alpha the factors may differ by one fp32 ulp (neither fp64 pow is
 correctly rounded), so the errors agree to 1e-3 relative."""
+import dataclasses
+
 import numpy as np
 import pytest
 
@@ -25,8 +27,10 @@ def sq():
     return m
 
 
-def _case(dtype, ln, T=64, T_cal=256, N=256):
+def _case(dtype, ln, T=64, T_cal=256, N=256, K=None):
     lin = synth.workloads()["tiny_k1024"].linears[0]
+    if K is not None:
+        lin = dataclasses.replace(lin, K=K)
     d = synth.make_linear_inputs(lin, T=T, T_cal=T_cal, N=N)
     x, x_cal, w = d["x"], d["x_cal"], d["w"]
     if dtype == "bf16":
@@ -84,3 +88,26 @@ def test_alpha_sweep_larger_bf16_layer(sq, orc):
         assert abs(e_got - e_want) <= 1e-9 * e_want
     assert np.array_equal(host(again)[::-1], got)  # reuse, any order: deterministic sums
     assert got[1] < got[0] and got[1] < got[2]
+
+
+@pytest.mark.parametrize("T,N,K", [(300, 264, 1024), (200, 520, 256)])
+@pytest.mark.parametrize("gran,dtype,ln", [("token", "bf16", True), ("static", "f32", False),
+                                           ("tensor", "bf16", False)])
+def test_alpha_sweep_error_in_gemm_epilogue(sq, orc, T, N, K, gran, dtype, ln):
+    """More than 128 tokens: the GEMM folds the error sums into its epilogue
+    (one fp64 pair per each of its 12 epilogue warps) and never writes y.
+    Ragged rows and columns, a long and a short K; errors against the
+    oracle's same chain, and bit-identical on a second run."""
+    x, x_cal, w, g, b = _case(dtype, ln, T=T, T_cal=256, N=N, K=K)
+    amax = orc.calib_absmax(x_cal, g, b)
+    y_ref = _ref(orc, x, w, g, b)
+    alphas = [0.0, 0.5, 1.0]
+    want = [orc.alpha_error(amax, w, x, y_ref, a, g, b, gran=gran) for a in alphas]
+    kw = dict(per_token=gran == "token", per_tensor_dynamic=gran == "tensor")
+    err = sq.sq_alpha_sweep(dev(amax), dev(w), dev(x), dev(y_ref), alphas, dev(g), dev(b), **kw)
+    again = sq.sq_alpha_sweep(dev(amax), dev(w), dev(x), dev(y_ref), alphas, dev(g), dev(b), **kw)
+    sq.sq_sync_status()
+    got = host(err)
+    for a, e_got, e_want in zip(alphas, got, want):
+        assert abs(e_got - e_want) <= 1e-9 * e_want, (a, e_got, e_want)
+    assert np.array_equal(host(again), got)

@@ -2,6 +2,8 @@
 // kernel launchers.  Nothing is enqueued when a check fails.
 #include <cuda_runtime.h>
 #include <math.h>
+
+#include <algorithm>
 #include <stdarg.h>
 #include <stdio.h>
 #include <string.h>
@@ -400,8 +402,10 @@ sq_status sq_gemm_w8a8_noalloc(const int8_t* xq, const int8_t* wq, int64_t M, in
 namespace {
 // Workspace of sq_alpha_sweep, carved in this order (each piece 256-byte
 // aligned): wmax, s, inv_s, Delta_A [K|K|K|4] fp32; gamma', beta' [K|K];
-// w_scale [N]; act_scale [M]; wq [N,K]; xq [M,K]; y [M,N] fp32; the error
-// reduction's per-block fp64 sums; then the GEMM's own workspace.
+// w_scale [N]; act_scale [M]; wq [N,K]; xq [M,K]; y [M,N] fp32 (used only
+// when the GEMM cannot fold the error into its epilogue); the error
+// reduction's fp64 sums (per block, or per epilogue warp); then the GEMM's
+// own workspace.
 struct SweepLayout {
   size_t wmax, s, inv_s, dA, g2, b2, ws, act, wq, xq, y, sums, gemm, total;
 };
@@ -420,7 +424,8 @@ SweepLayout sweep_layout(int64_t M, int64_t N, int64_t K) {
   L.wq = o; o += al((size_t)N * (size_t)K);
   L.xq = o; o += al((size_t)M * (size_t)K);
   L.y = o; o += al(4 * (size_t)M * (size_t)N);
-  L.sums = o; o += al(output_error_scratch_bytes());
+  const size_t warp_sums = 2 * sizeof(double) * (size_t)gemm_err_max_slots();
+  L.sums = o; o += al(std::max(output_error_scratch_bytes(), warp_sums));
   L.gemm = o; o += al(gemm_workspace_bytes(M, N, K));
   L.total = o;
   return L;
@@ -512,16 +517,23 @@ sq_status sq_alpha_sweep(const float* amax_x, const void* w, sq_dtype wt, int64_
     if (e == cudaSuccess && stat)
       e = cudaMemcpyAsync(act, dA, sizeof(float), cudaMemcpyDeviceToDevice, st);
     if (e == cudaSuccess) e = run_quant(q, xt, gran, st);
-    // the GEMM in fp32, then the error against y_ref
+    // the GEMM in fp32 and the error against y_ref: folded into the GEMM's
+    // epilogue where the large-M kernel serves the shape (y never written),
+    // else y, then a pass over y and y_ref
     GemmArgs g{};
     g.xq = xq; g.wq = wq; g.M = M; g.N = N; g.K = K; g.act_scale = act;
     g.act_per_token = gran == SQ_ACT_PER_TOKEN_DYNAMIC ? 1 : 0; g.w_scale = ws; g.y = y;
     g.yt = SQ_F32; g.workspace = base + L.gemm; g.workspace_bytes = L.total - L.gemm;
-    if (e == cudaSuccess) {
+    if (e == cudaSuccess && gemm_err_ok(M, N)) {
+      int nslots = 0;
+      const sq_status gs = launch_gemm_err(g, y_ref, sums, &nslots, st);
+      if (gs != SQ_OK) return gs;
+      e = launch_output_error_final(sums, nslots, err + i, st);
+    } else if (e == cudaSuccess) {
       const sq_status gs = launch_gemm(g, st);
       if (gs != SQ_OK) return gs;
+      e = launch_output_error(y, y_ref, M * N, sums, err + i, st);
     }
-    if (e == cudaSuccess) e = launch_output_error(y, y_ref, M * N, sums, err + i, st);
   }
   return e == cudaSuccess ? SQ_OK : cuda_fail(e, fn);
 }

@@ -689,14 +689,19 @@ output_error_final_kernel(const double* part, int nblocks, double* err) {
   }
 }
 
+cudaError_t launch_output_error_final(const double* part, int nslots, double* err,
+                                      cudaStream_t st) {
+  return launch_pdl(output_error_final_kernel, dim3(1), dim3(kErrThreads), 0, st, part, nslots,
+                    err);
+}
+
 cudaError_t launch_output_error(const float* y, const float* y_ref, int64_t n, double* scratch,
                                 double* err, cudaStream_t st) {
   const int blocks = output_error_blocks(n);
   cudaError_t e = launch_pdl(output_error_kernel, dim3((unsigned)blocks), dim3(kErrThreads), 0,
                              st, y, y_ref, n, scratch);
   if (e != cudaSuccess) return e;
-  return launch_pdl(output_error_final_kernel, dim3(1), dim3(kErrThreads), 0, st,
-                    (const double*)scratch, blocks, err);
+  return launch_output_error_final(scratch, blocks, err, st);
 }
 
 // ============================================================ producer fold

@@ -86,6 +86,9 @@ cudaError_t launch_fold_producer(const float* s, int64_t K, float* w_scale, floa
 size_t output_error_scratch_bytes();
 cudaError_t launch_output_error(const float* y, const float* y_ref, int64_t n, double* scratch,
                                 double* err, cudaStream_t st);
+// The last step alone: *err from nslots (sum (y - r)^2, sum r^2) pairs.
+cudaError_t launch_output_error_final(const double* part, int nslots, double* err,
+                                      cudaStream_t st);
 
 cudaError_t launch_fold_ln(const float* gamma, const float* beta,
                            const float* s, int64_t K, float* gamma_out,
@@ -126,6 +129,15 @@ sq_status launch_bmm(const BmmArgs& a, cudaStream_t st);
 
 size_t gemm_workspace_bytes(int64_t M, int64_t N, int64_t K);
 sq_status launch_gemm(const GemmArgs& a, cudaStream_t st);
+
+// The GEMM in error mode (fp32 y, shapes the large-M kernel serves:
+// gemm_err_ok): y is not written; each epilogue warp leaves its
+// (sum (y - y_ref)^2, sum y_ref^2) in fp64 in part[2*i], part[2*i+1], and
+// *nslots (at most gemm_err_max_slots()) says how many pairs were written.
+bool gemm_err_ok(int64_t M, int64_t N);
+int gemm_err_max_slots();
+sq_status launch_gemm_err(const GemmArgs& a, const float* y_ref, double* part, int* nslots,
+                          cudaStream_t st);
 
 // sq_gemm_w8a8_noalloc: the same GEMM with its scratch in a static device
 // array of kNoallocScratchBytes (gemm.cu).
