@@ -218,3 +218,20 @@ def test_binding_fails_loudly_without_library(tmp_path, monkeypatch):
     monkeypatch.setattr(os.path, "exists", lambda p: False if p.endswith(".so") else True)
     with pytest.raises(ImportError):
         spec.loader.exec_module(mod)
+
+
+def test_gemm_decode_routing_on_the_host(lib):
+    """Which GEMM shapes take the stream-K path (and so need scratch) is
+    decided on the host; without a device the SM count is taken as 148.
+    Up to 8 tokens always stream-K; 9-128 tokens only while the 128-row
+    tiles across N would not give every SM one; more than 128 never.  The
+    scratch size follows the header's formula."""
+    f = lib.lib.sq_gemm_workspace_bytes
+    sms = 148
+    assert f(8, 49152, 12288) > 0
+    assert f(16, 49152, 12288) == 0 and f(128, 49152, 12288) == 0  # 256 tiles of 192
+    assert f(128, 12288, 12288) > 0                                  # 64 tiles
+    assert f(16, 192 * (sms - 1), 4096) > 0                          # one tile short of the SMs
+    assert f(129, 512, 4096) == 0
+    # 1000 channels: 8 tile counters (256 bytes) + 148 SMs x 2 slots x 1 token x 128 x 4
+    assert f(1, 1000, 12288) == 256 + sms * 2 * 1 * 128 * 4
