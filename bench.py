@@ -52,8 +52,13 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # DRAM bytes (read + write) of one launch of the dominant kernel, from the ncu
 # capture summarised in profiles/ (null when the kernel has changed since)
 GEMM_DRAM_TRAFFIC = {
-    "opt6.7b_qkv_t2048": (75.33e6, "profiles/gemm_w8a8_tc_opt6.7b_qkv_t2048.md: "
-                          "dram__bytes_read.sum 58.82 MB + dram__bytes_write.sum 16.51 MB"),
+    # the kernel was rebuilt after this capture (template parameters for the
+    # short-K and error-mode epilogues; its 4-warp path's loads and stores are
+    # the same), so the counters are given as context, not claimed for it
+    "opt6.7b_qkv_t2048": (None, "not re-captured for this build; last capture "
+                          "(profiles/gemm_w8a8_tc_opt6.7b_qkv_t2048.md, earlier build of the "
+                          "same main loop): dram__bytes_read.sum 58.82 MB + dram__bytes_write.sum "
+                          "16.51 MB = 75.33 MB per launch"),
 }
 
 
