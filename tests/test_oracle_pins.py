@@ -511,6 +511,118 @@ def test_rmsnorm_exact_closed_form(orc):
     assert not np.array_equal(orc.layernorm_row(x, g, None, eps=0.0), y)
 
 
+# Rows whose fp32 mean depends on the order of the canonical reduction: two
+# elements of +-2^24 and two ones.  Under the library's order the pair that
+# is summed first decides whether a one is lost to rounding (2^24 + 1 is a
+# tie and rounds to the even 2^24; -2^24 + 1 is exact).
+#
+# Row A (the cross-group combination): 2^24 at k = 0 (slot 0, group 0),
+# -2^24 at k = 256 (slot 32, group 1), 1 at k = 512 (group 2) and k = 768
+# (group 3).  Each group's butterfly only adds zeros to its one element, so
+# (r0, r1, r2, r3) = (2^24, -2^24, 1, 1) and (r0 + r2) + (r1 + r3) =
+# 2^24 + (-2^24 + 1) = 1.  Left to right, or (r0 + r1) + (r2 + r3), gives 2.
+#
+# Row B (the butterfly inside a group): 2^24 at k = 0 (slot 0), -2^24 at
+# k = 8 (slot 1), 1 at k = 128 (slot 16) and k = 136 (slot 17).  The first
+# butterfly round (xor 16) pairs slot 0 with 16 and slot 1 with 17: 2^24 and
+# -2^24 + 1; the last round (xor 1) adds those: 1.  A butterfly starting at
+# xor 1, or a sequential sum, gives 0 + 2 = 2.
+#
+# Either way mu = 1/1024 = 2^-10 exactly.  Variance pass: (+-2^24 - mu)
+# rounds to +-2^24, whose square 2^48 absorbs every other term of its slot
+# and group (each < 2^24, half an ulp of 2^48); the two 2^48 meet in the
+# final sum, so var = 2^49 / 1024 = 2^39 in both rows.
+def _order_rows():
+    K = 1024
+    a = np.zeros(K, np.float32)
+    a[0], a[256], a[512], a[768] = 2.0 ** 24, -(2.0 ** 24), 1.0, 1.0
+    b = np.zeros(K, np.float32)
+    b[0], b[8], b[128], b[136] = 2.0 ** 24, -(2.0 ** 24), 1.0, 1.0
+    return a, b
+
+
+def _ln_by_hand(x, mu, var, eps=np.float32(0.0)):
+    """y = ((x - mu) * rstd) * 1 + 0 from given moments, each step one fp32
+    rounding (numpy float32 arithmetic is IEEE round-to-nearest)."""
+    rstd = np.float32(1.0) / np.sqrt(np.float32(var) + eps)
+    return ((x - np.float32(mu)) * rstd).astype(np.float32)
+
+
+def test_layernorm_canonical_order_rows(orc):
+    """The fixed LayerNorm reduction order (128 slots, xor-16-first butterfly,
+    groups as (r0 + r2) + (r1 + r3)) on two hand-built rows whose fp32 mean
+    is 2^-10 under that order and 2^-9 under the plausible others (see the
+    comment above): y equals the hand-derived values bit for bit and differs
+    from the alternative mean's."""
+    g = np.ones(1024, np.float32)
+    for x in _order_rows():
+        y = orc.layernorm_row(x, g, None, eps=0.0)
+        want = _ln_by_hand(x, 2.0 ** -10, 2.0 ** 39)
+        assert np.array_equal(y.view(np.uint32), want.view(np.uint32))
+        alt = _ln_by_hand(x, 2.0 ** -9, 2.0 ** 39)
+        assert not np.array_equal(y, alt)
+
+
+def test_quant_act_rms_exact_rows(orc):
+    """The RMSNorm quantizer pinned by hand.  Rows of +-2 with eps = 0: the
+    mean of squares is exactly 4 in any order, rstd = 1/2, so y = +-gamma'.
+    Per token, the row peak 4 gives Delta = 4/127 and 1/Delta = 31.75 exactly,
+    so gamma' = 4, 1, 0.5, 2, 3, 0.25, 1.5, 0.75 code to 127, 32, 16 (15.875),
+    64 (63.5, tie to even), 95 (95.25), 8 (7.9375), 48 (47.625), 24 (23.8125).
+    Static step 1/32: 4 -> 128 saturates to 127 (counted), the others to 32,
+    16, 64, 96, 8, 48, 24.  Per-tensor dynamic over both rows: peak 4 again,
+    so the per-token codes.  The rows' mean is 1, not 0: a LayerNorm in place
+    of the RMSNorm would shift and rescale y and change the codes."""
+    gp = np.array([4, 1, 0.5, 2, 3, 0.25, 1.5, 0.75] * 2, np.float32)
+    sign = np.array([[1, -1, 1, 1, -1, 1, 1, 1, 1, -1, 1, 1, 1, 1, -1, 1],
+                     [-1, 1, 1, 1, 1, -1, 1, 1, 1, 1, -1, 1, 1, 1, 1, -1]], np.float32)
+    x = (2.0 * sign).astype(np.float32)
+    mag_tok = np.array([127, 32, 16, 64, 95, 8, 48, 24] * 2)
+    mag_st = np.array([127, 32, 16, 64, 96, 8, 48, 24] * 2)
+    xq, act, ncl = orc.quant_act_rms(x, gp, eps=0.0, per_token=True)
+    assert np.array_equal(act, np.full(2, np.float32(4.0) / np.float32(127.0)))
+    assert np.array_equal(xq, (sign * mag_tok).astype(np.int8)) and ncl == 0
+    xq, _, ncl = orc.quant_act_rms(x, gp, eps=0.0, per_token=False,
+                                   static_delta=np.float32(1.0 / 32))
+    assert np.array_equal(xq, (sign * mag_st).astype(np.int8)) and ncl == 4
+    xq, act, _ = orc.quant_act_rms(x, gp, eps=0.0, per_tensor_dynamic=True)
+    assert act[0] == np.float32(4.0) / np.float32(127.0)
+    assert np.array_equal(xq, (sign * mag_tok).astype(np.int8))
+    xq_ln, _, _ = orc.quant_act(x, gp, None, 0.0, per_token=True)
+    assert not np.array_equal(xq_ln, (sign * mag_tok).astype(np.int8))
+
+
+def test_quant_act_rms_through_rmsnorm_row(orc):
+    """The RMSNorm quantizer equals the separately pinned RMSNorm row
+    (orc.rmsnorm_row) followed by the textbook quantizer written out here in
+    fp32 numpy -- Delta = max(peak, 1e-7)/127, codes rne(y * (1/Delta))
+    clamped to +-127 -- on outlier-structured rows, per token, static and per
+    tensor dynamic."""
+    lin = synth.workloads()["tiny_k1024"].linears[0]
+    d = synth.make_linear_inputs(lin, T=12, T_cal=16, N=8)
+    g = (1 + 0.1 * np.random.default_rng(15).standard_normal(1024)).astype(np.float32)
+    y = np.stack([orc.rmsnorm_row(row, g) for row in d["x"]])
+
+    def q(yv, dl):
+        inv = np.float32(1.0) / np.float32(dl)
+        return np.clip(np.rint(yv * inv), -127, 127).astype(np.int8)
+
+    def dlt(peak):
+        return np.float32(max(np.float32(peak), np.float32(1e-7))) / np.float32(127.0)
+
+    xq, act, _ = orc.quant_act_rms(d["x"], g, per_token=True)
+    for t in range(y.shape[0]):
+        assert act[t] == dlt(np.abs(y[t]).max())
+        assert np.array_equal(xq[t], q(y[t], act[t]))
+    ds = np.float32(0.02)
+    xq, _, ncl = orc.quant_act_rms(d["x"], g, per_token=False, static_delta=ds)
+    assert np.array_equal(xq, q(y, ds))
+    assert ncl == int(np.sum(np.abs(np.rint(y * (np.float32(1) / ds))) > 127))
+    xq, act, _ = orc.quant_act_rms(d["x"], g, per_tensor_dynamic=True)
+    assert act[0] == dlt(np.abs(y).max())
+    assert np.array_equal(xq, q(y, act[0]))
+
+
 def test_rmsnorm_fold_alpha_one(orc):
     """Calibration through the RMSNorm, alpha = 1 (s = the peaks), the fold
     gamma' = gamma / s: the smoothed calibration peaks are 1 within 2 ulp

@@ -176,6 +176,114 @@ def test_quant_act_edge_values(sq, orc):
         assert int(host(ncl)[0]) == ncl_want
 
 
+def _with_non_finite(x, seed):
+    """Rows with NaN among finite values (row 0: one NaN; row 1: several
+    NaN and a +inf; row 2: all NaN; row 3: NaN beside the row's largest
+    element), the rest of the rows untouched."""
+    x = np.array(x, copy=True)
+    r = np.random.default_rng(seed)
+    K = x.shape[1]
+    nan = np.float32(np.nan) if x.dtype == np.float32 else synth.bf16_bits(np.float32(np.nan))[0]
+    inf = np.float32(np.inf) if x.dtype == np.float32 else synth.bf16_bits(np.float32(np.inf))[0]
+    x[0, r.integers(0, K)] = nan
+    x[1, r.integers(0, K, 5)] = nan
+    x[1, r.integers(0, K)] = inf
+    x[2, :] = nan
+    mag = np.abs(x[3].astype(np.float32)) if x.dtype == np.float32 else np.abs(
+        (x[3].astype(np.uint32) << 16).view(np.float32))
+    k = int(np.argmax(mag))
+    x[3, (k + 1) % K] = nan
+    return x
+
+
+NAN_SHAPES = [(6, 64), (5, 1040), (7, 4096), (4, 20480)]
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+@pytest.mark.parametrize("mode", ["ln", "inv_s", "plain"])
+@pytest.mark.parametrize("gran", ["token", "static", "tensor"])
+@pytest.mark.parametrize("T,K", NAN_SHAPES)
+def test_quant_act_nan_rows(sq, orc, dtype, mode, gran, T, K):
+    """NaN (and +inf) in per-token, static and per-tensor-dynamic rows, with
+    a LayerNorm, a 1/s multiplier or neither: NaN codes to 0, the peaks skip
+    NaN, a LayerNorm row with a NaN is NaN throughout (all codes 0, the
+    floored step); codes, steps and saturation counts bit-exact."""
+    x = _with_non_finite(_x(41, T, K, dtype), T * K)
+    r = np.random.default_rng(K)
+    g = b = inv = None
+    if mode == "ln":
+        g, b = _ln(41, K)
+    elif mode == "inv_s":
+        inv = r.uniform(0.02, 2.0, K).astype(np.float32)
+    dstatic = np.float32(0.05)
+    kw = dict(per_token=(gran == "token"), static_delta=dstatic,
+              per_tensor_dynamic=(gran == "tensor"))
+    xq_want, act_want, ncl_want = orc.quant_act(x, g, b, 1e-5, inv, **kw)
+    xq = torch.empty((T, K), dtype=torch.int8, device="cuda")
+    if gran == "token":
+        act = torch.empty(T, dtype=torch.float32, device="cuda")
+    else:
+        act = torch.tensor([dstatic], dtype=torch.float32, device="cuda")
+    ncl = torch.zeros(1, dtype=torch.int64, device="cuda")
+    sq.sq_ln_smooth_quant_act(dev(x), xq, act, dev(g), dev(b), 1e-5, dev(inv),
+                              per_token=(gran == "token"), n_clipped=ncl,
+                              per_tensor_dynamic=(gran == "tensor"))
+    sq.sq_sync_status()
+    if gran != "static":
+        assert_bits_equal(host(act), act_want, "act_scale (NaN rows)")
+    assert_bits_equal(host(xq), xq_want, "xq (NaN rows)")
+    assert int(host(ncl)[0]) == ncl_want
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+@pytest.mark.parametrize("ln", [False, True])
+@pytest.mark.parametrize("T,K", [(40, 1040), (9, 4096), (300, 8192)])
+def test_calib_absmax_nan_rows(sq, orc, dtype, ln, T, K):
+    """Calibration peaks skip NaN (raw column strips and LayerNorm rows)."""
+    x = _with_non_finite(_x(43, T, K, dtype), T + K)
+    g, b = _ln(43, K) if ln else (None, None)
+    want = orc.calib_absmax(x, g, b, 1e-5)
+    amax = torch.zeros(K, dtype=torch.float32, device="cuda")
+    sq.sq_calib_absmax(dev(x), amax, dev(g), dev(b), 1e-5)
+    assert_bits_equal(host(amax), want, "amax (NaN rows)")
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+def test_layernorm_order_rows(sq, orc, dtype):
+    """The two hand-built rows whose fp32 mean depends on the canonical
+    LayerNorm reduction order (the oracle is pinned on them by hand), with
+    seeded rows beside them: calibration peak and per-token / static codes
+    bit-exact against the oracle, eps = 0 and 1e-5."""
+    K = 1024
+    ra = np.zeros(K, np.float32)
+    ra[0], ra[256], ra[512], ra[768] = 2.0 ** 24, -(2.0 ** 24), 1.0, 1.0
+    rb = np.zeros(K, np.float32)
+    rb[0], rb[8], rb[128], rb[136] = 2.0 ** 24, -(2.0 ** 24), 1.0, 1.0
+    x = np.concatenate([ra[None], rb[None], _x(45, 6, K, "f32")]).astype(np.float32)
+    if dtype == "bf16":
+        x = synth.bf16_bits(x)
+    g = np.ones(K, np.float32)
+    gs, bs = _ln(45, K)
+    for eps in (0.0, 1e-5):
+        for gg, bb in ((g, None), (gs, bs)):
+            want = orc.calib_absmax(x, gg, bb, eps)
+            amax = torch.zeros(K, dtype=torch.float32, device="cuda")
+            sq.sq_calib_absmax(dev(x), amax, dev(gg), dev(bb), eps)
+            assert_bits_equal(host(amax), want, "amax (order rows)")
+            for per_token in (True, False):
+                dstatic = np.float32(1e-4)
+                xq_want, act_want, _ = orc.quant_act(x, gg, bb, eps, per_token=per_token,
+                                                     static_delta=dstatic)
+                xq = torch.empty((x.shape[0], K), dtype=torch.int8, device="cuda")
+                act = (torch.empty(x.shape[0], dtype=torch.float32, device="cuda") if per_token
+                       else torch.tensor([dstatic], device="cuda"))
+                sq.sq_ln_smooth_quant_act(dev(x), xq, act, dev(gg), dev(bb), eps,
+                                          per_token=per_token)
+                if per_token:
+                    assert_bits_equal(host(act), act_want, "act (order rows)")
+                assert_bits_equal(host(xq), xq_want, "xq (order rows)")
+
+
 def test_runs_are_deterministic(sq):
     """Two runs of the LN calibration and the quantizer give identical bits
     (a race in the reductions would show up here)."""
