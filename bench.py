@@ -10,6 +10,9 @@ tcgen05 GEMM with the dequantizing epilogue.
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
                     [--impl reference]
 
+The default workload is the large prefill (calibration peaks over 65536 x
+8192 bf16 tokens, then the 8192 -> 28672 linear at 16384 tokens, static
+per-tensor activations), the largest single-GPU configuration.
 `value` is whole-job throughput in TOPS = 2*M*N*K per step (all ranks) over
 the device time of the timed steps, max over ranks.  Each step is one replay
 of a CUDA graph of the five calls, timed on the device by event nodes at the
@@ -19,14 +22,23 @@ adds to the step.  Before every timed replay L2 is flushed outside the timed
 events: a 256 MiB buffer is written, then another 256 MiB buffer is read, so
 that the timed work finds neither its data nor the flush's dirty lines in
 L2.  Inputs are resident in HBM.
+`runtime_forward` times what serving pays per batch (the quantizer and the
+GEMM) on its own.  `int8_peak` measures the denominator of the GEMM's
+roofline on this GPU: the tcgen05 kind::i8 issue rate with no memory traffic
+(sq_probe_mma_i8) and cuBLAS's INT8 GEMM at 8192^3 (torch._int_mm).
 `e2e` is the same metric through the public Python API with pinned host
 buffers: every step copies its inputs host->device and its output back.
-`--impl reference` times the CPU oracle (tests-only code) on bounded samples
-of the same workload, each step extrapolated linearly to the full workload.
+`--impl reference` times the CPU oracle (tests-only code) on one host core,
+on bounded samples of the same workload, each step extrapolated linearly to
+the full workload.
+`--profile-call NAME` only runs the named call of the step `--steps` times
+after the warm-up steps (for an ncu capture of one kernel) and prints no
+line; `--tokens T` shrinks the runtime token count for such a capture.
 """
 from __future__ import annotations
 
 import argparse
+import dataclasses
 import json
 import os
 import statistics
@@ -43,23 +55,17 @@ sys.path.insert(0, ROOT)
 import synth  # noqa: E402
 
 METRIC = "W8A8 smoothed-linear TOPS & % INT8 peak; small-M HBM GB/s (1×B200)"
-DEFAULT_WORKLOAD = "opt6.7b_qkv_t2048"
+DEFAULT_WORKLOAD = "large_prefill_k8192"
+SECONDARY_WORKLOAD = "opt6.7b_qkv_t2048"
 FLUSH_BYTES = 256 << 20
-# INT8 dense peak = measured bf16 dense peak x the nominal int8:bf16 ratio
-# (4.5 POPS : 2.25 PFLOP/s = 2).
+# nominal ratio of dense int8 to dense bf16 tensor throughput (4.5 : 2.25)
 INT8_PER_BF16 = 2.0
+VENDOR_INT8_TOPS = 4500.0  # dense, NVIDIA's figure for B200
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
-# DRAM bytes (read + write) of one launch of the dominant kernel, from the ncu
-# capture summarised in profiles/ (null when the kernel has changed since)
-GEMM_DRAM_TRAFFIC = {
-    # the kernel was rebuilt after this capture (template parameters for the
-    # short-K and error-mode epilogues; its 4-warp path's loads and stores are
-    # the same), so the counters are given as context, not claimed for it
-    "opt6.7b_qkv_t2048": (None, "not re-captured for this build; last capture "
-                          "(profiles/gemm_w8a8_tc_opt6.7b_qkv_t2048.md, earlier build of the "
-                          "same main loop): dram__bytes_read.sum 58.82 MB + dram__bytes_write.sum "
-                          "16.51 MB = 75.33 MB per launch"),
-}
+CALLS = ["calib_absmax", "smooth_scales", "fuse_weights_q8", "ln_smooth_quant_act", "gemm_w8a8"]
+# DRAM bytes (read + write) of one launch of the step's GEMM, from an ncu
+# capture of the current kernel (None until one exists for the workload)
+GEMM_DRAM_TRAFFIC = {}
 
 
 def load_peaks():
@@ -83,14 +89,22 @@ def parse():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-small-m", action="store_true",
                     help="skip the decode-shaped (small-M) GEMM measurement")
+    ap.add_argument("--no-extras", action="store_true",
+                    help="skip the secondary workload, the HBM rows and the next rows")
+    ap.add_argument("--profile-call", default=None, choices=CALLS + ["int8_probe"],
+                    help="run only this call (after the warm-up steps) --steps times; no line")
+    ap.add_argument("--tokens", type=int, default=None,
+                    help="runtime tokens of the workload's linear (profiling of smaller cases)")
     return ap.parse_args()
 
 
-def pick_linear(args):
-    wl = synth.workloads()[args.workload]
+def pick_linear(args, workload=None):
+    wl = synth.workloads()[workload or args.workload]
     lin = wl.linears[0]
-    if args.linear:
+    if args.linear and workload is None:
         lin = next(l for l in wl.linears if l.name == args.linear)
+    if args.tokens and workload is None:
+        lin = dataclasses.replace(lin, T=int(args.tokens))
     return wl, lin
 
 
@@ -145,7 +159,7 @@ class ClockSampler:
                         self.reasons.add(name)
             except Exception:  # noqa: BLE001
                 pass
-            time.sleep(0.02)
+            time.sleep(0.005)
 
     def __enter__(self):
         if self._ok:
@@ -194,7 +208,9 @@ class Layer:
         self.g2 = torch.empty(K, dtype=f32, device=dev) if lin.ln else None
         self.b2 = torch.empty(K, dtype=f32, device=dev) if lin.ln else None
         self.xq = torch.empty((M, K), dtype=torch.int8, device=dev)
-        self.act = torch.empty(M if lin.per_token else 1, dtype=f32, device=dev)
+        # per-token steps are written by the quantizer; a static step is the
+        # one the smoothing call derives (dA), read by the quantizer and GEMM
+        self.act = torch.empty(M, dtype=f32, device=dev) if lin.per_token else self.dA
         self.y = torch.empty((M, N), dtype=io, device=dev)
         self.workspace = sq.Workspace(dev)
         # this library's kernels per step: calibration peak; column peak +
@@ -202,37 +218,40 @@ class Layer:
         # s); quantizer; GEMM
         self.kernels_per_step = 6
 
-    def step(self, ev=None, upto=5):
-        """The first `upto` of the five calls (all five: one step); ev = (start,
-        end) events recorded around them, or None.  (Running the weight
-        column peaks on a second stream beside the calibration was measured
-        no faster: whichever kernel starts first fills the SMs.)"""
+    def step(self, ev=None, upto=5, start=1):
+        """Calls start..upto of the five (1..5: one step); ev = (start, end)
+        events recorded around them, or None.  (Running the weight column
+        peaks on a second stream beside the calibration was measured no
+        faster: whichever kernel starts first fills the SMs.)"""
         sq, L = self.sq, self.lin
         if ev is not None:
             ev[0].record()
-        self.amax.zero_()
-        sq.sq_calib_absmax(self.x_cal, self.amax, self.gamma, self.beta, 1e-5)
-        if upto >= 2:
+        if start <= 1 <= upto:
+            self.amax.zero_()
+            sq.sq_calib_absmax(self.x_cal, self.amax, self.gamma, self.beta, 1e-5)
+        if start <= 2 <= upto:
             sq.sq_smooth_scales(self.amax, self.w, L.alpha, self.s, self.inv_s,
                                 None if L.per_token else self.dA)
-        if upto >= 3:
+        if start <= 3 <= upto:
             sq.sq_fuse_weights_q8(self.w, self.s, self.wq, self.ws, self.gamma, self.beta,
                                   self.g2, self.b2)
-        act = self.act
-        if upto >= 4:
-            if not L.per_token:
-                act.copy_(self.dA)
+        if start <= 4 <= upto:
             if L.ln:
-                sq.sq_ln_smooth_quant_act(self.x, self.xq, act, self.g2, self.b2, 1e-5,
+                sq.sq_ln_smooth_quant_act(self.x, self.xq, self.act, self.g2, self.b2, 1e-5,
                                           per_token=L.per_token)
             else:
-                sq.sq_ln_smooth_quant_act(self.x, self.xq, act, inv_s=self.inv_s,
+                sq.sq_ln_smooth_quant_act(self.x, self.xq, self.act, inv_s=self.inv_s,
                                           per_token=L.per_token)
-        if upto >= 5:
-            sq.sq_gemm_w8a8(self.xq, self.wq, act, self.ws, self.y, per_token=L.per_token,
+        if start <= 5 <= upto:
+            sq.sq_gemm_w8a8(self.xq, self.wq, self.act, self.ws, self.y, per_token=L.per_token,
                             workspace=self.workspace)
         if ev is not None:
             ev[1].record()
+
+    def call(self, name):
+        """One of the five calls on its own (inputs from an earlier step)."""
+        j = CALLS.index(name) + 1
+        self.step(upto=j, start=j)
 
 
 class L2Flush:
@@ -280,6 +299,145 @@ def algorithmic_bytes(lin):
     }
 
 
+def time_step_graphs(torch, layer, flush, K, clocks=None, prefixes=True):
+    """Step times (ms) of K replays of the whole step's graph, each after an
+    L2 flush, device events at the graph's two ends; then (prefixes) the
+    mean time of graphs of the first 1..4 calls, so that a call's time is
+    what it adds to the step."""
+
+    def capture(upto, start=1):
+        ev = (torch.cuda.Event(enable_timing=True, external=True),
+              torch.cuda.Event(enable_timing=True, external=True))
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            layer.step(ev, upto, start)
+        return g, ev
+
+    def replay(g, ev, n):
+        t = []
+        for i in range(n):
+            flush(i)  # evicts the previous replay's data from L2
+            g.replay()
+            torch.cuda.synchronize()
+            t.append(ev[0].elapsed_time(ev[1]))
+        return t
+
+    graph, ev_step = capture(5)
+    for _ in range(3):
+        graph.replay()
+    torch.cuda.synchronize()
+    if clocks is not None:
+        with clocks:
+            step_ms = replay(graph, ev_step, K)
+    else:
+        step_ms = replay(graph, ev_step, K)
+    del graph
+    if not prefixes:
+        return step_ms, None
+    prefix_ms = {0: 0.0, 5: statistics.mean(step_ms)}
+    for upto in range(1, 5):
+        g, ev = capture(upto)
+        g.replay()
+        prefix_ms[upto] = statistics.mean(replay(g, ev, K))
+        del g
+    per = {n: prefix_ms[j + 1] - prefix_ms[j] for j, n in enumerate(CALLS)}
+    return step_ms, per
+
+
+def kernel_table(lin, per, hbm, int8_peak):
+    ops = 2.0 * lin.T * lin.N * lin.K
+    ab = algorithmic_bytes(lin)
+    kernels = {}
+    for n in CALLS:
+        ms = per[n]
+        k = {"ms": round(ms, 5), "bytes": int(ab[n]),
+             "gbs": round(ab[n] / (ms * 1e-3) / 1e9, 1),
+             "hbm_frac": round(ab[n] / (ms * 1e-3) / 1e9 / hbm, 3)}
+        if n == "gemm_w8a8":
+            tops = ops / (ms * 1e-3) / 1e12
+            k["tops"] = round(tops, 1)
+            k["int8_frac"] = round(tops / int8_peak, 3)
+            k["int8_frac_vendor"] = round(tops / VENDOR_INT8_TOPS, 3)
+        kernels[n] = k
+    return kernels
+
+
+def measure_int8_peak(sq, torch, dev, clocks_cls):
+    """The dense INT8 tensor-core ceiling of this GPU, measured two ways:
+    (1) the tcgen05.mma kind::i8 issue rate with the operands in shared
+    memory and no other work (sq_probe_mma_i8, one CTA per SM), in bursts of
+    about 2 ms with idle gaps -- the way the step's GEMM runs in the timed
+    region -- and, for context, back to back for ~30 ms launches, where the
+    power cap lowers the clock; (2) cuBLAS's INT8 GEMM (torch._int_mm) at
+    8192^3.  Best of several launches each, CUDA events on the launching
+    stream, NVML clock sampled during each.  The larger of the burst probe
+    and cuBLAS is the roofline's peak."""
+    sms = torch.cuda.get_device_properties(dev).multi_processor_count
+
+    def ev_time(fn, reps, warm, gap_s=0.0):
+        for _ in range(warm):
+            fn()
+        torch.cuda.synchronize()
+        best = None
+        for _ in range(reps):
+            if gap_s:
+                time.sleep(gap_s)
+            e0 = torch.cuda.Event(enable_timing=True)
+            e1 = torch.cuda.Event(enable_timing=True)
+            e0.record()
+            fn()
+            e1.record()
+            torch.cuda.synchronize()
+            t = e0.elapsed_time(e1)
+            best = t if best is None else min(best, t)
+        return best
+
+    out = {}
+    for name, kblocks, reps, gap in (("tcgen05_i8_probe", 8000, 10, 0.05),
+                                     ("tcgen05_i8_probe_sustained", 100_000, 5, 0.0)):
+        clocks = clocks_cls(torch.cuda.current_device())
+        with clocks:
+            ms = ev_time(lambda: sq.sq_probe_mma_i8(kblocks, sms), reps, 2, gap)
+        st = sq.sq_sync_status()
+        tops = 8388608.0 * kblocks * sms / (ms * 1e-3) / 1e12
+        out[name] = {"tops": round(tops, 1), "ms": round(ms, 3), "ctas": sms,
+                     "kblocks_per_cta": kblocks, "idle_gap_s": gap,
+                     "mma": "128x256x32 kind::i8, one accumulator, operands in smem",
+                     "clocks": clocks.summary(), "status": st}
+    probe_tops = out["tcgen05_i8_probe"]["tops"]
+    n = 8192
+    g = torch.Generator(device=dev).manual_seed(5)
+    a = torch.randint(-127, 128, (n, n), dtype=torch.int8, device=dev, generator=g)
+    b = torch.randint(-127, 128, (n, n), dtype=torch.int8, device=dev, generator=g)
+    try:
+        ms2 = ev_time(lambda: torch._int_mm(a, b.t()), 10, 3)
+        cub = 2.0 * n ** 3 / (ms2 * 1e-3) / 1e12
+        out["cublas_int8_gemm_8192"] = {"tops": round(cub, 1), "ms": round(ms2, 3),
+                                        "call": "torch._int_mm (cuBLASLt), int32 out"}
+    except Exception as e:  # noqa: BLE001 - reported, the probe still stands
+        cub = 0.0
+        out["cublas_int8_gemm_8192"] = {"error": str(e)[:200]}
+    del a, b
+    out["peak_tops"] = round(max(probe_tops, cub), 1)
+    out["peak_from"] = "tcgen05_i8_probe" if probe_tops >= cub else "cublas_int8_gemm_8192"
+    out["vendor_dense_tops"] = VENDOR_INT8_TOPS
+    return out
+
+
+def profile_only(args, sq, torch, layer, flush):
+    """--profile-call: the named call alone, --steps times, nothing printed."""
+    for _ in range(max(1, args.warmup)):
+        layer.step()
+    torch.cuda.synchronize()
+    for i in range(args.steps):
+        if args.profile_call == "int8_probe":
+            sq.sq_probe_mma_i8(2000, torch.cuda.get_device_properties(0).multi_processor_count)
+        else:
+            layer.call(args.profile_call)
+    torch.cuda.synchronize()
+    sq.sq_sync_status()
+
+
 def run_ours(args):
     import torch
     import torch.distributed as dist
@@ -302,99 +460,70 @@ def run_ours(args):
     d = synth.make_linear_inputs(lin)
     layer = Layer(sq, torch, lin, d, dev)
     flush = L2Flush(torch, dev)
+    if args.profile_call:
+        profile_only(args, sq, torch, layer, flush)
+        return
 
     def barrier():
         if world > 1:
             dist.barrier()
         torch.cuda.synchronize()
 
-    for _ in range(max(3, args.warmup)):
+    warm = max(3, args.warmup)
+    for _ in range(warm):
         layer.step()
     sq.sq_sync_status()
-    names = ["calib_absmax", "smooth_scales", "fuse_weights_q8", "ln_smooth_quant_act",
-             "gemm_w8a8"]
 
-    def capture(upto):
-        ev = (torch.cuda.Event(enable_timing=True, external=True),
-              torch.cuda.Event(enable_timing=True, external=True))
-        g = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(g):
-            layer.step(ev, upto)
-        return g, ev
-
-    # the timed graph: one whole step (five calls, six kernels), event
-    # nodes only at its two ends
-    graph, ev_step = capture(5)
-    for _ in range(max(3, args.warmup)):
-        graph.replay()
-    barrier()
-
+    # the timed region: K replays of the step's graph (five calls, six
+    # kernels), event nodes only at its two ends
     K = args.steps
-    step_ms = []
     clocks = ClockSampler(torch.cuda.current_device())
-    with clocks:
-        barrier()
-        for i in range(K):
-            flush(i)  # evicts the previous step's data from L2
-            graph.replay()
-            torch.cuda.synchronize()
-            step_ms.append(ev_step[0].elapsed_time(ev_step[1]))
-        barrier()
+    barrier()
+    step_ms, per = time_step_graphs(torch, layer, flush, K, clocks)
+    barrier()
     sq.sq_sync_status()
     total_ms = max_over_ranks(float(sum(step_ms)), world, dev)
     ops = 2.0 * lin.T * lin.N * lin.K
     value = throughput_tops(ops, K, world, total_ms)
 
-    # per-call breakdown (after the timed region): graphs of the first 1..4
-    # calls, timed like the step; a call's time is what it adds to the step
-    prefix_ms = {5: statistics.mean(step_ms)}
-    for upto in range(1, 5):
-        g, ev = capture(upto)
-        g.replay()
-        t = []
-        for i in range(K):
-            flush(i)
-            g.replay()
-            torch.cuda.synchronize()
-            t.append(ev[0].elapsed_time(ev[1]))
-        prefix_ms[upto] = statistics.mean(t)
-        del g
-    prefix_ms[0] = 0.0
-    per = {n: prefix_ms[j + 1] - prefix_ms[j] for j, n in enumerate(names)}
-    sq.sq_sync_status()
+    peaks, peak_kind = load_peaks()
+    hbm = peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"])
+    bf16_peak = peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"])
+    int8 = measure_int8_peak(sq, torch, dev, ClockSampler)
+    int8_peak = int8["peak_tops"]
+    kernels = kernel_table(lin, per, hbm, int8_peak)
+    gemm_tops = kernels["gemm_w8a8"]["tops"]
+
+    # what serving pays per batch: the quantizer and the GEMM alone
+    fwd_ms = time_graph_calls(torch, lambda: layer.step(upto=5, start=4), flush, K)
+    runtime_forward = {
+        "calls": "sq_ln_smooth_quant_act + sq_gemm_w8a8 (the offline steps excluded)",
+        "us": round(fwd_ms * 1e3, 2), "tops": round(ops / (fwd_ms * 1e-3) / 1e12, 1),
+        "int8_frac": round(ops / (fwd_ms * 1e-3) / 1e12 / int8_peak, 3)}
 
     # ---- e2e through the public API with pinned host buffers
     e2e = run_e2e(sq, torch, layer, lin, d, dev, args.e2e_steps, world, barrier)
     small_m = None if args.no_small_m else run_small_m(sq, torch, dev, flush)
-    next_rows = {"o2_per_tensor_dynamic_quant": run_o2(sq, torch, layer, lin, flush),
-                 "gemm_bias_epilogue": run_gemm_bias(sq, torch, layer, lin, flush),
-                 "rmsnorm_quant_per_token": run_rms_quant(sq, torch, layer, lin, flush),
-                 "alpha_sweep": run_alpha_sweep(sq, torch, layer, lin, flush),
-                 "attention_bmm": run_attention_bmm(sq, torch, layer.x.device, flush)}
+    extras = {}
+    if not args.no_extras:
+        extras["secondary_workloads"] = {
+            SECONDARY_WORKLOAD: run_secondary(args, sq, torch, dev, flush, hbm, int8_peak)}
+        extras["hbm_rows"] = run_hbm_rows(sq, torch, dev, flush, hbm)
+        extras["next_rows"] = {
+            "o2_per_tensor_dynamic_quant": run_o2(sq, torch, layer, lin, flush),
+            "gemm_bias_epilogue": run_gemm_bias(sq, torch, layer, lin, flush, int8_peak),
+            "rmsnorm_quant_per_token": run_rms_quant(sq, torch, layer, lin, flush),
+            "alpha_sweep": run_alpha_sweep(sq, torch, layer, lin, flush),
+            "attention_bmm": run_attention_bmm(sq, torch, layer.x.device, flush, int8_peak)}
 
-    peaks, peak_kind = load_peaks()
-    bf16_peak = peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"])
-    int8_peak = bf16_peak * INT8_PER_BF16
-    gemm_ms = per["gemm_w8a8"]
-    gemm_tops = ops / (gemm_ms * 1e-3) / 1e12
-    ab = algorithmic_bytes(lin)
-    hbm = peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"])
-    kernels = {}
-    for n in names:
-        ms = per[n]
-        k = {"ms": round(ms, 5), "gbs": round(ab[n] / (ms * 1e-3) / 1e9, 1),
-             "hbm_frac": round(ab[n] / (ms * 1e-3) / 1e9 / hbm, 3)}
-        if n == "gemm_w8a8":
-            k["tops"] = round(gemm_tops, 1)
-            k["int8_frac"] = round(gemm_tops / int8_peak, 3)
-        kernels[n] = k
+    traffic = GEMM_DRAM_TRAFFIC.get(wl.name, (None, None))
     line = {
         "metric": METRIC,
         "value": round(value, 2),
         "unit": "TOPS",
         "n_gpus": world,
         "steps": K,
-        "warmup": max(3, args.warmup),
+        "warmup": warm,
         "ms_per_step": round(total_ms / K, 5),
         "higher_is_better": True,
         "scaling": "weak",
@@ -404,19 +533,24 @@ def run_ours(args):
         "config": config_of(wl, lin, world),
         "roofline": {
             "bound": "tensor",
-            "kernel": "gemm_w8a8 (tcgen05.mma kind::i8)",
+            "kernel": "gemm_w8a8 (tcgen05.mma kind::i8), its share of the step",
             "achieved": round(gemm_tops, 1),
-            "peak": round(int8_peak, 1),
+            "peak": int8_peak,
             "unit": "TFLOP/s",
             "frac": round(gemm_tops / int8_peak, 4),
-            "traffic": GEMM_DRAM_TRAFFIC.get(wl.name, (None, None))[0],
-            "traffic_source": GEMM_DRAM_TRAFFIC.get(wl.name, (None, None))[1],
-            "peak_note": f"int8 dense = {peak_kind} bf16 burst {bf16_peak} TFLOP/s x 2 "
-                         "(nominal int8:bf16 ratio); 'TFLOP/s' here counts int8 ops",
+            "frac_vendor": round(gemm_tops / VENDOR_INT8_TOPS, 4),
+            "frac_bf16x2": round(gemm_tops / (bf16_peak * INT8_PER_BF16), 4),
+            "traffic": traffic[0],
+            "traffic_source": traffic[1],
+            "peak_note": f"int8 ops; peak measured live on this GPU ({int8['peak_from']}); "
+                         f"frac_vendor against the dense {VENDOR_INT8_TOPS:.0f} TOPS spec; "
+                         f"frac_bf16x2 against the {peak_kind} bf16 burst {bf16_peak} TFLOP/s x 2",
         },
+        "int8_peak": int8,
         "kernels": kernels,
+        "runtime_forward": runtime_forward,
         "small_m_decode": small_m,
-        "next_rows": next_rows,
+        **extras,
         "e2e": e2e,
         "gpu_launches": layer.kernels_per_step * K,
         "clocks": clocks.summary(),
@@ -428,6 +562,81 @@ def run_ours(args):
         dist.destroy_process_group()
     if rank == 0:
         print(json.dumps(line), flush=True)
+
+
+def time_graph_calls(torch, fn, flush, reps):
+    """Mean device time (ms) of fn captured as one CUDA graph, replayed reps
+    times, each replay after an L2 flush, device events at its two ends."""
+    e0 = torch.cuda.Event(enable_timing=True, external=True)
+    e1 = torch.cuda.Event(enable_timing=True, external=True)
+    fn()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        e0.record()
+        fn()
+        e1.record()
+    graph.replay()
+    t = []
+    for i in range(reps):
+        flush(i)
+        graph.replay()
+        torch.cuda.synchronize()
+        t.append(e0.elapsed_time(e1))
+    del graph
+    return statistics.mean(t)
+
+
+def run_secondary(args, sq, torch, dev, flush, hbm, int8_peak):
+    """The OPT-6.7B-shaped QKV step (LayerNorm, per-token) timed like the
+    headline step: whole-step TOPS and the per-call breakdown."""
+    _, lin = pick_linear(args, SECONDARY_WORKLOAD)
+    d = synth.make_linear_inputs(lin)
+    layer = Layer(sq, torch, lin, d, dev)
+    for _ in range(3):
+        layer.step()
+    step_ms, per = time_step_graphs(torch, layer, flush, max(args.steps, 20))
+    sq.sq_sync_status()
+    ms = statistics.mean(step_ms)
+    ops = 2.0 * lin.T * lin.N * lin.K
+    fwd_ms = time_graph_calls(torch, lambda: layer.step(upto=5, start=4), flush, 20)
+    out = {"config": config_of(synth.workloads()[SECONDARY_WORKLOAD], lin, 1),
+           "ms_per_step": round(ms, 5), "tops": round(ops / (ms * 1e-3) / 1e12, 1),
+           "kernels": kernel_table(lin, per, hbm, int8_peak),
+           "runtime_forward": {"us": round(fwd_ms * 1e3, 2),
+                               "tops": round(ops / (fwd_ms * 1e-3) / 1e12, 1)}}
+    del layer
+    return out
+
+
+def run_hbm_rows(sq, torch, dev, flush, hbm):
+    """HBM-bound steps at sizes where they are HBM-bound (inputs far larger
+    than L2): the 13B fc2 input quantizer (4096 x 20480 bf16, per-token,
+    x * 1/s) and its raw calibration peak, each one graph replay after an
+    L2 flush."""
+    lin = next(l for l in synth.workloads()["13b_layer_t4096"].linears if l.name == "fc2_a0.5")
+    K, T = lin.K, lin.T
+    out_ch = synth.outlier_pattern(lin.seed, K, lin.outlier_frac, tag=f"k{K}")
+    x = torch.from_numpy(synth.bf16_bits(synth.activations(
+        lin.seed, "bench/fc2_x", T, K, out_ch, relu=True)).view(np.int16)).view(torch.bfloat16).to(dev)
+    g = torch.Generator(device=dev).manual_seed(17)
+    inv_s = torch.rand(K, device=dev, generator=g) * 1.9 + 0.02
+    xq = torch.empty((T, K), dtype=torch.int8, device=dev)
+    act = torch.empty(T, dtype=torch.float32, device=dev)
+    amax = torch.zeros(K, dtype=torch.float32, device=dev)
+    res = {}
+    ms = time_graph_calls(torch, lambda: sq.sq_ln_smooth_quant_act(x, xq, act, inv_s=inv_s,
+                                                                   per_token=True), flush, 20)
+    nb = T * K * 2 + T * K + 4 * T + 4 * K
+    res["13b_fc2_quant_per_token"] = {"shape": f"{T}x{K} bf16, x * 1/s", "us": round(ms * 1e3, 2),
+                                      "bytes": nb, "gbs": round(nb / (ms * 1e-3) / 1e9, 1),
+                                      "hbm_frac": round(nb / (ms * 1e-3) / 1e9 / hbm, 3)}
+    ms = time_graph_calls(torch, lambda: sq.sq_calib_absmax(x, amax), flush, 20)
+    nb = T * K * 2 + 4 * K
+    res["13b_fc2_calib_absmax"] = {"shape": f"{T}x{K} bf16, raw", "us": round(ms * 1e3, 2),
+                                   "bytes": nb, "gbs": round(nb / (ms * 1e-3) / 1e9, 1),
+                                   "hbm_frac": round(nb / (ms * 1e-3) / 1e9 / hbm, 3)}
+    sq.sq_sync_status()
+    return res
 
 
 def run_small_m(sq, torch, dev, flush, reps=20):
@@ -572,13 +781,11 @@ def run_alpha_sweep(sq, torch, layer, lin, flush, alphas=(0.0, 0.25, 0.5, 0.75, 
             "rel_error": [round(e, 6) for e in err], "us_per_alpha": round(ms * 1e3 / len(alphas), 1)}
 
 
-def run_attention_bmm(sq, torch, dev, flush, heads=32, tokens=2048, head_dim=128):
+def run_attention_bmm(sq, torch, dev, flush, int8_peak, heads=32, tokens=2048, head_dim=128):
     """Attention's INT8 matmuls (NEXT-4) at OPT-6.7B shapes, one batched
     launch over the heads each: scores = Q K^T (per-token Q steps, one K step
     per head) and P V (V^T as the K-major operand), bf16 out."""
     g = torch.Generator(device=dev).manual_seed(11)
-    peaks, _ = load_peaks()
-    int8_peak = peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]) * INT8_PER_BF16
     out = {}
     for name, (M, N, K) in (("scores_qk", (tokens, tokens, head_dim)),
                             ("pv", (tokens, head_dim, tokens))):
@@ -614,7 +821,7 @@ def run_rms_quant(sq, torch, layer, lin, flush):
             "hbm_frac": round(gbs / hbm, 3), "bytes": int(nbytes)}
 
 
-def run_gemm_bias(sq, torch, layer, lin, flush, reps=20):
+def run_gemm_bias(sq, torch, layer, lin, flush, int8_peak, reps=20):
     """The step's GEMM with the bias epilogue (y = dequantized acc + bias[n]),
     timed like the decode GEMM: one CUDA-graph replay per call after an L2
     flush, device events around it."""
@@ -644,8 +851,6 @@ def run_gemm_bias(sq, torch, layer, lin, flush, reps=20):
     sq.sq_sync_status()
     del graph
     ms = statistics.mean(times)
-    peaks, _ = load_peaks()
-    int8_peak = peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]) * INT8_PER_BF16
     tops = 2.0 * M * N * K / (ms * 1e-3) / 1e12
     return {"shape": f"{M}x{N}x{K}", "us": round(ms * 1e3, 2), "tops": round(tops, 1),
             "int8_frac": round(tops / int8_peak, 3),
@@ -697,15 +902,44 @@ def run_e2e(sq, torch, layer, lin, d, dev, steps, world, barrier):
 
 
 # ---------------------------------------------------------------- CPU oracle
-def oracle_step_sample(lin, d, frac_tokens, gemm_rows, frac_w):
-    """Time the oracle on a bounded sample of each step and extrapolate each
-    step linearly in the sampled dimension.  Returns (seconds_full, sample)."""
+def host_record():
+    """The host the oracle runs on: CPU model, logical CPUs, and the core
+    the timing thread is pinned to."""
+    model = "unknown"
+    try:
+        with open("/proc/cpuinfo") as f:
+            for ln in f:
+                if ln.startswith("model name"):
+                    model = ln.split(":", 1)[1].strip()
+                    break
+    except OSError:
+        pass
+    return {"cpu_model": model, "nproc": os.cpu_count()}
+
+
+class PinnedToOneCore:
+    """Pins the calling thread to one allowed core (the highest-numbered,
+    away from the usual interrupt and driver cores) for the oracle timing,
+    and restores the previous affinity afterwards."""
+
+    def __enter__(self):
+        self.prev = os.sched_getaffinity(0)
+        self.core = max(self.prev)
+        os.sched_setaffinity(0, {self.core})
+        return self
+
+    def __exit__(self, *a):
+        os.sched_setaffinity(0, self.prev)
+
+
+def oracle_step_sample(lin, d, Tc, Tq, Nw, R):
+    """Time the oracle on a bounded sample of each step -- the first Tc
+    calibration tokens, Nw weight rows, Tq runtime tokens and an R x Nw x K
+    GEMM of `d` -- and extrapolate each step linearly in the sampled
+    dimension to lin's full sizes.  Returns (seconds_full, parts, sample)."""
     import oracle
 
     oracle.build()
-    Tc = max(1, int(lin.T_cal * frac_tokens))
-    Tq = max(1, int(lin.T * frac_tokens))
-    Nw = max(1, int(lin.N * frac_w))
     t = {}
     t0 = time.perf_counter()
     amax = oracle.calib_absmax(d["x_cal"][:Tc], d["gamma"], d["beta"], 1e-5)
@@ -728,27 +962,37 @@ def oracle_step_sample(lin, d, frac_tokens, gemm_rows, frac_w):
         xq, act, _ = oracle.quant_act(d["x"][:Tq], inv_s=inv_s, per_token=lin.per_token,
                                       static_delta=dA)
     t["quant"] = (time.perf_counter() - t0) * lin.T / Tq
-    R = max(1, min(gemm_rows, Tq))
+    R = max(1, min(R, Tq))
     t0 = time.perf_counter()
     oracle.gemm_w8a8(xq[:R], wq, act[:R] if lin.per_token else act, ws,
                      per_token=lin.per_token, out_bf16=(lin.dtype == "bf16"))
     t["gemm"] = (time.perf_counter() - t0) * (lin.T / R) * (lin.N / Nw)
-    sample = (f"oracle (single-threaded C) on {Tc}/{lin.T_cal} calibration tokens, "
-              f"{Nw}/{lin.N} weight rows, {Tq}/{lin.T} runtime tokens and a {R}x{Nw}x{lin.K} "
-              f"GEMM; each step extrapolated linearly to the full workload")
+    sample = (f"oracle (single-threaded C, one pinned core) on {Tc}/{lin.T_cal} calibration "
+              f"tokens, {Nw}/{lin.N} weight rows, {Tq}/{lin.T} runtime tokens and a "
+              f"{R}x{Nw}x{lin.K} GEMM; each step extrapolated linearly to the full workload")
     return sum(t.values()), t, sample
 
 
 def cpu_baseline(lin, d):
     # the offline steps and the quantizer on every token and weight row, and
-    # a quarter of the GEMM's token rows: about 10 s of one host core (the
-    # GEMM dominates; the rest is extrapolated from it linearly)
-    secs, parts, sample = oracle_step_sample(lin, d, 1, lin.T // 4, 1)
+    # 48 of the GEMM's token rows (one host core, about 15 s; the GEMM is
+    # extrapolated from them linearly)
+    with PinnedToOneCore() as pin:
+        t0 = time.perf_counter()
+        secs, parts, sample = oracle_step_sample(lin, d, lin.T_cal, lin.T, lin.N, 48)
+        timed = time.perf_counter() - t0
     ops = 2.0 * lin.T * lin.N * lin.K
     return {"value": round(ops / secs / 1e12, 6), "unit": "TOPS", "cores": 1,
-            "kind": "oracle", "sample": sample,
+            "kind": "oracle", "sample": sample, "extrapolated": True,
             "seconds_per_step_extrapolated": round(secs, 2),
+            "seconds_timed": round(timed, 2), "pinned_core": pin.core, **host_record(),
             "parts_s": {k: round(v, 3) for k, v in parts.items()}}
+
+
+# the reference arm's sample: 1/16 of the tokens, 1/8 of the weight rows and
+# a 2-row GEMM of the workload, drawn with the workload's own recipe (about
+# half a second of one host core per step at the large prefill)
+REF_FRAC_TOKENS, REF_FRAC_W, REF_GEMM_ROWS = 16, 8, 2
 
 
 def run_reference(args):
@@ -757,18 +1001,23 @@ def run_reference(args):
     if rank != 0:
         return
     wl, lin = pick_linear(args)
-    d = synth.make_linear_inputs(lin)
-    # each step: the oracle on a bounded sample of the step (about 20 ms of
-    # one core), extrapolated to the full workload; exactly `steps` of them
-    # after at least 3 warm-up samples
+    Tc = max(1, lin.T_cal // REF_FRAC_TOKENS)
+    Tq = max(1, lin.T // REF_FRAC_TOKENS)
+    Nw = max(1, lin.N // REF_FRAC_W)
+    d = synth.make_linear_inputs(lin, T=Tq, T_cal=Tc, N=Nw)
+    # each step: the oracle on the bounded sample, extrapolated to the full
+    # workload; exactly `steps` of them after at least 3 warm-up samples
     warm = max(3, args.warmup)
-    for _ in range(warm):
-        oracle_step_sample(lin, d, 1 / 64, 2, 1 / 16)
-    secs_all = []
+    secs_all, timed_all = [], []
     sample = ""
-    for _ in range(max(1, args.steps)):
-        secs, _, sample = oracle_step_sample(lin, d, 1 / 64, 2, 1 / 16)
-        secs_all.append(secs)
+    with PinnedToOneCore() as pin:
+        for _ in range(warm):
+            oracle_step_sample(lin, d, Tc, Tq, Nw, REF_GEMM_ROWS)
+        for _ in range(max(1, args.steps)):
+            t0 = time.perf_counter()
+            secs, _, sample = oracle_step_sample(lin, d, Tc, Tq, Nw, REF_GEMM_ROWS)
+            timed_all.append(time.perf_counter() - t0)
+            secs_all.append(secs)
     ops = 2.0 * lin.T * lin.N * lin.K
     total = sum(secs_all)
     value = ops * len(secs_all) / total / 1e12
@@ -776,11 +1025,14 @@ def run_reference(args):
         "metric": METRIC, "value": round(value, 6), "unit": "TOPS", "impl": "reference",
         "n_gpus": world, "steps": len(secs_all), "warmup": warm,
         "ms_per_step": round(total / len(secs_all) * 1e3, 3),
+        "ms_per_step_is": "extrapolated from the timed sample to the full workload",
+        "sample_ms_per_step": round(sum(timed_all) / len(timed_all) * 1e3, 3),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "int8",
         "data": "synthetic (seeded outlier-structured activations, random-init weights)",
         "config": config_of(wl, lin, world),
         "cpu_baseline": {"value": round(value, 6), "unit": "TOPS", "cores": 1, "kind": "oracle",
-                         "sample": sample},
+                         "sample": sample, "extrapolated": True, "pinned_core": pin.core,
+                         **host_record()},
         "e2e": {"value": round(value, 6), "unit": "TOPS", "h2d_bytes_per_step": 0,
                 "d2h_bytes_per_step": 0},
     }

@@ -422,6 +422,20 @@ const char* sq_last_error(void);
  */
 sq_status sq_selftest_bounded_wait(int64_t limit_ns, sq_stream stream);
 
+/*
+ * sq_probe_mma_i8 -- measurement support (no counterpart on the pages): the
+ * INT8 tensor-core rate of this GPU, the ceiling the large-M GEMM is compared
+ * with.  Launches `grid` CTAs (one per SM when grid <= the SM count; each
+ * takes more shared memory than two CTAs could share) that each issue
+ * kblocks x 4 tcgen05.mma kind::i8 steps of 128 x 256 x 32 back to back into
+ * one INT32 TMEM accumulator, from operand tiles in shared memory, with no
+ * global-memory traffic.  The work is 8,388,608 * kblocks * grid int8 ops
+ * (2 per multiply-add); the caller times the launch on `stream`.
+ * kblocks in [1, 2^30], grid in [1, 65535], else SQ_ERR_INVALID_ARG; the
+ * final wait is bounded (SQ_ERR_TIMEOUT through sq_sync_status).
+ */
+sq_status sq_probe_mma_i8(int64_t kblocks, int grid, sq_stream stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -28,7 +28,7 @@ __all__ = [
     "sq_sync_status", "sq_selftest_bounded_wait", "SQError", "Workspace",
     "sq_calib_absmax_rms", "sq_rms_smooth_quant_act", "sq_fold_into_producer",
     "sq_alpha_sweep_workspace_bytes", "sq_alpha_sweep", "sq_bmm_w8a8",
-    "sq_weight_colmax", "sq_smooth_scales_peaks",
+    "sq_weight_colmax", "sq_smooth_scales_peaks", "sq_probe_mma_i8",
 ]
 
 
@@ -239,3 +239,11 @@ def sq_sync_status(stream=None):
 def sq_selftest_bounded_wait(limit_ns: int, stream=None):
     check(lib.sq_selftest_bounded_wait(int(limit_ns), _stream(stream)),
           "sq_selftest_bounded_wait")
+
+
+def sq_probe_mma_i8(kblocks: int, grid: int, stream=None):
+    """Launch the INT8 tensor-core rate probe: grid CTAs, each issuing
+    kblocks x 4 tcgen05.mma kind::i8 steps of 128 x 256 x 32 (8,388,608 ops
+    per k-block).  Returns the op count; the caller times the launch."""
+    check(lib.sq_probe_mma_i8(int(kblocks), int(grid), _stream(stream)), "sq_probe_mma_i8")
+    return 8388608 * int(kblocks) * int(grid)

@@ -578,4 +578,14 @@ sq_status sq_selftest_bounded_wait(int64_t limit_ns, sq_stream stream) {
   return e == cudaSuccess ? SQ_OK : cuda_fail(e, "sq_selftest_bounded_wait");
 }
 
+sq_status sq_probe_mma_i8(int64_t kblocks, int grid, sq_stream stream) {
+  g_last_error[0] = 0;
+  if (kblocks < 1 || kblocks > ((int64_t)1 << 30))
+    return fail(SQ_ERR_INVALID_ARG, "sq_probe_mma_i8: kblocks must be in [1, 2^30]");
+  if (grid < 1 || grid > 65535)
+    return fail(SQ_ERR_INVALID_ARG, "sq_probe_mma_i8: grid must be in [1, 65535]");
+  cudaError_t e = launch_mma_probe(kblocks, grid, (cudaStream_t)stream);
+  return e == cudaSuccess ? SQ_OK : cuda_fail(e, "sq_probe_mma_i8");
+}
+
 }  // extern "C"

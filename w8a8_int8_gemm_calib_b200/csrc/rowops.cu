@@ -34,6 +34,17 @@ namespace sq {
 // (valid because every value is >= 0).
 constexpr int kColWarps = 8;
 
+__device__ __forceinline__ float warp_sum_butterfly(float p) {
+#pragma unroll
+  for (int o = 16; o >= 1; o >>= 1) p = __fadd_rn(p, __shfl_xor_sync(0xffffffffu, p, o));
+  return p;
+}
+__device__ __forceinline__ float warp_max(float p) {
+#pragma unroll
+  for (int o = 16; o >= 1; o >>= 1) p = fmaxf(p, __shfl_xor_sync(0xffffffffu, p, o));
+  return p;
+}
+
 template <typename T>
 __global__ void __launch_bounds__(kColWarps * 32)
 colmax_kernel(const T* __restrict__ x, int64_t T_, int64_t K, int64_t rows_per_slab,
@@ -87,6 +98,36 @@ colmax_kernel(const T* __restrict__ x, int64_t T_, int64_t K, int64_t rows_per_s
   if (k < K) atomicMax(out + k, __float_as_uint(v));
 }
 
+// Slabs of rows per column strip so that the grid is one wave of resident
+// CTAs (per_sm of them on every SM): a second, partial wave would leave a
+// few CTAs streaming alone at the end, far below the HBM rate (65536 x 8192
+// bf16 peaks: 262 us with 768 CTAs on 740 slots).
+int64_t strip_rows(int64_t T, int64_t strips, int per_sm) {
+  const int64_t target = (int64_t)sm_count() * per_sm;
+  int64_t slabs = target / strips;
+  if (slabs < 1) slabs = 1;
+  const int64_t min_rows = 8 * kColWarps;  // at least one unrolled step
+  const int64_t maxslabs = (T + min_rows - 1) / min_rows;
+  if (slabs > maxslabs) slabs = maxslabs;
+  if (slabs > 65535) slabs = 65535;
+  if (slabs < 1) slabs = 1;
+  return (T + slabs - 1) / slabs;
+}
+
+// Resident CTAs per SM of a kernel at kColWarps warps (queried once per
+// device and instantiation).
+template <typename Kern>
+int strip_occupancy(Kern kern, std::once_flag* once, int* occ) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 1;
+  std::call_once(once[dev], [&] {
+    int n = 0;
+    cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, kern, kColWarps * 32, 0);
+    occ[dev] = n < 1 ? 1 : n;
+  });
+  return occ[dev];
+}
+
 // Column strips stream the rows with plain 16-byte loads and no
 // synchronisation at all; measured faster here than staging whole rows
 // through the shared-memory ring, where every row waits for all the warps
@@ -97,34 +138,110 @@ cudaError_t launch_colmax(const void* x, sq_dtype xt, int64_t T, int64_t K, floa
   const int64_t strips = (K + 255) / 256;
   static std::once_flag once[2][64];
   static int occ[2][64];
-  int dev = 0;
-  cudaError_t de = cudaGetDevice(&dev);
-  if (de != cudaSuccess || dev < 0 || dev >= 64) return de != cudaSuccess ? de : cudaErrorInvalidDevice;
-  const int ti = xt == SQ_BF16 ? 0 : 1;
-  std::call_once(once[ti][dev], [&] {
-    int n = 0;
-    if (xt == SQ_BF16)
-      cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, colmax_kernel<uint16_t>, kColWarps * 32, 0);
-    else
-      cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, colmax_kernel<float>, kColWarps * 32, 0);
-    occ[ti][dev] = n < 1 ? 1 : n;
-  });
-  const int per_sm = occ[ti][dev];
-  const int64_t target = (int64_t)sm_count() * per_sm;  // one wave of CTAs
-  int64_t slabs = (target + strips - 1) / strips;
-  const int64_t min_rows = 8 * kColWarps;               // at least one unrolled step
-  int64_t maxslabs = (T + min_rows - 1) / min_rows;
-  if (slabs > maxslabs) slabs = maxslabs;
-  if (slabs < 1) slabs = 1;
-  if (slabs > 65535) slabs = 65535;
-  const int64_t rows = (T + slabs - 1) / slabs;
-  slabs = (T + rows - 1) / rows;
-  dim3 grid((unsigned)strips, (unsigned)slabs);
+  const int per_sm = xt == SQ_BF16 ? strip_occupancy(colmax_kernel<uint16_t>, once[0], occ[0])
+                                   : strip_occupancy(colmax_kernel<float>, once[1], occ[1]);
+  const int64_t rows = strip_rows(T, strips, per_sm);
+  dim3 grid((unsigned)strips, (unsigned)((T + rows - 1) / rows));
   if (xt == SQ_BF16)
     return launch_pdl(colmax_kernel<uint16_t>, grid, dim3(kColWarps * 32), 0, st,
                       (const uint16_t*)x, T, K, rows, (unsigned int*)out);
   return launch_pdl(colmax_kernel<float>, grid, dim3(kColWarps * 32), 0, st, (const float*)x, T,
                     K, rows, (unsigned int*)out);
+}
+
+// ============================================================ strip quantizer
+// The activation quantizer when no LayerNorm precedes and the step is one
+// number for the whole call: y = x * m[k] (or x) and Q(y; Delta) are
+// independent per element, so the call is a plain stream -- the column-strip
+// layout of colmax_kernel (a warp per 256 columns and 8 rows, several rows
+// in flight per thread), each lane's 8 multipliers in registers, 8 codes
+// stored per lane per row.  PEAK: no codes; the peak of |y| over the call
+// (NaN skipped) is folded into *peak with one atomic max per warp (the first
+// pass of per-tensor dynamic quantization).
+template <typename T, bool PEAK>
+__global__ void __launch_bounds__(kColWarps * 32)
+strip_quant_kernel(const T* __restrict__ x, int64_t T_, int64_t K, int64_t rows_per_slab,
+                   const float* __restrict__ mul, const float* scale, int8_t* __restrict__ q,
+                   unsigned long long* n_clipped, unsigned int* peak) {
+  pdl_launch_dependents();
+  pdl_wait();
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int64_t nchunk = K >> 3;
+  const int64_t chunk = (int64_t)blockIdx.x * 32 + lane;
+  const bool live = chunk < nchunk;
+  const int64_t r0 = (int64_t)blockIdx.y * rows_per_slab;
+  const int64_t r1 = min(T_, r0 + rows_per_slab);
+  float m8[8];
+#pragma unroll
+  for (int e = 0; e < 8; ++e) m8[e] = 1.0f;
+  if (live && mul) load8(mul + chunk * 8, m8);
+  const float inv = PEAK ? 0.0f : __fdiv_rn(1.0f, __ldg(scale));
+  const bool count = n_clipped != nullptr;
+  unsigned clipped = 0;
+  float pk = 0.0f;
+  auto work = [&](const Raw8<T>& raw, int64_t r) {
+    float v[8];
+    unpack(raw, v);
+    if (mul) {
+#pragma unroll
+      for (int e = 0; e < 8; ++e) v[e] = __fmul_rn(v[e], m8[e]);
+    }
+    if constexpr (PEAK) {
+#pragma unroll
+      for (int e = 0; e < 8; ++e) pk = fmaxf(pk, fabsf(v[e]));
+    } else {
+      uint32_t b[8];
+#pragma unroll
+      for (int e = 0; e < 8; ++e) b[e] = qbits(v[e], inv, count, clipped);
+      store_codes(q + r * K + chunk * 8, b);
+    }
+  };
+  if (live) {
+    const T* base = x + chunk * 8;
+    constexpr int U = sizeof(T) == 2 ? 8 : 4;  // 128 B in flight per thread
+    int64_t r = r0 + warp;
+    for (; r + (U - 1) * kColWarps < r1; r += U * kColWarps) {
+      Raw8<T> raw[U];
+#pragma unroll
+      for (int u = 0; u < U; ++u) load_raw(base + (r + u * kColWarps) * K, raw[u]);
+#pragma unroll
+      for (int u = 0; u < U; ++u) work(raw[u], r + u * kColWarps);
+    }
+    for (; r < r1; r += kColWarps) {
+      Raw8<T> raw;
+      load_raw(base + r * K, raw);
+      work(raw, r);
+    }
+  }
+  if constexpr (PEAK) {
+    pk = warp_max(pk);
+    if (lane == 0) atomicMax(peak, __float_as_uint(pk));
+  } else if (count) {
+#pragma unroll
+    for (int o = 16; o >= 1; o >>= 1) clipped += __shfl_xor_sync(0xffffffffu, clipped, o);
+    if (lane == 0 && clipped) atomicAdd(n_clipped, (unsigned long long)clipped);
+  }
+}
+
+template <typename T, bool PEAK>
+cudaError_t launch_strip_quant_t(const RowArgs& a, cudaStream_t st) {
+  static std::once_flag once[64];
+  static int occ[64];
+  const int per_sm = strip_occupancy(strip_quant_kernel<T, PEAK>, once, occ);
+  const int64_t strips = (a.K + 255) / 256;
+  const int64_t rows = strip_rows(a.T, strips, per_sm);
+  dim3 grid((unsigned)strips, (unsigned)((a.T + rows - 1) / rows));
+  return launch_pdl(strip_quant_kernel<T, PEAK>, grid, dim3(kColWarps * 32), 0, st,
+                    (const T*)a.x, a.T, a.K, rows, a.mul, (const float*)a.scale, a.q,
+                    a.n_clipped, reinterpret_cast<unsigned int*>(a.peak));
+}
+
+cudaError_t launch_strip_quant(const RowArgs& a, sq_dtype xt, RowMode mode, cudaStream_t st) {
+  if (mode == ROW_PEAK)
+    return xt == SQ_BF16 ? launch_strip_quant_t<uint16_t, true>(a, st)
+                         : launch_strip_quant_t<float, true>(a, st);
+  return xt == SQ_BF16 ? launch_strip_quant_t<uint16_t, false>(a, st)
+                       : launch_strip_quant_t<float, false>(a, st);
 }
 
 // ============================================================ row kernel
@@ -153,16 +270,6 @@ __device__ __forceinline__ void slice_bar(int slice) {
   asm volatile("bar.sync %0, %1;" ::"r"(slice + 1), "r"(kSliceThreads) : "memory");
 }
 
-__device__ __forceinline__ float warp_sum_butterfly(float p) {
-#pragma unroll
-  for (int o = 16; o >= 1; o >>= 1) p = __fadd_rn(p, __shfl_xor_sync(0xffffffffu, p, o));
-  return p;
-}
-__device__ __forceinline__ float warp_max(float p) {
-#pragma unroll
-  for (int o = 16; o >= 1; o >>= 1) p = fmaxf(p, __shfl_xor_sync(0xffffffffu, p, o));
-  return p;
-}
 
 // Calls f(i, c, v[8]) for every chunk the thread owns, in increasing c.
 template <int MAXC, typename T, typename F>
@@ -349,8 +456,8 @@ row_kernel(RowArgs a) {
           if constexpr (MAXC > 0) {
             cmax[i * 8 + e] = fmaxf(cmax[i * 8 + e], y);
           } else {
-            if (use_smem) atomicMax(&colmax_s[c * 8 + e], __float_as_uint(y));
-            else atomicMax((unsigned int*)a.colmax + c * 8 + e, __float_as_uint(y));
+            if (use_smem) atomicMax(&colmax_s[c * 8 + e], peak_bits(y));
+            else atomicMax((unsigned int*)a.colmax + c * 8 + e, peak_bits(y));
           }
         }
       });
@@ -505,6 +612,10 @@ static cudaError_t dispatch_mode(const RowArgs& a, RowMode mode, cudaStream_t st
 }
 
 cudaError_t launch_row(const RowArgs& a, sq_dtype xt, RowMode mode, cudaStream_t st) {
+  // no LayerNorm and one step for the whole call: a plain element stream
+  const bool folds = a.fold_g_out || a.fold_b_out;
+  if (!a.g && !folds && (mode == ROW_STATIC || mode == ROW_PEAK))
+    return launch_strip_quant(a, xt, mode, st);
   if (rowpipe_fits(a.K, xt, mode, a.g != nullptr))
     return launch_rowpipe(a, xt, mode, st);
   if (xt == SQ_BF16) return dispatch_mode<uint16_t>(a, mode, st);

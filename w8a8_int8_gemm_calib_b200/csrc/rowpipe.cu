@@ -48,7 +48,6 @@ constexpr size_t kSmemBudget2 = 112 * 1024;  // two CTAs per SM (228 KB per SM)
 constexpr uint32_t kCopyPiece = 32768;
 constexpr uint64_t kWaitNs = 2000000000ull;
 constexpr uint64_t kDrainNs = 1000000000ull;
-constexpr float kRoundMagic = 12582912.0f;  // 1.5 * 2^23
 constexpr int kSrcSmem = 0, kSrcRaw = 1, kSrcF32 = 2;
 
 struct Pipe {
@@ -177,28 +176,6 @@ __device__ __forceinline__ float warp_maxabs_nan(float v) {
   float r;
   asm volatile("redux.sync.max.abs.NaN.f32 %0, %1, 0xffffffff;" : "=f"(r) : "f"(v));
   return r;
-}
-
-// Q(y; Delta) given inv = 1/Delta, as the fp32 whose low byte is the code:
-// general form (any y: NaN -> 0, saturation counted and clamped).
-__device__ __forceinline__ uint32_t qbits(float y, float inv, bool count, unsigned& clipped) {
-  float r = __fmul_rn(y, inv);
-  if (count) clipped += fabsf(r) >= 127.5f;  // rounds outside [-127, 127]
-  r = (r != r) ? 0.0f : r;
-  r = fminf(fmaxf(r, -127.0f), 127.0f);
-  return __float_as_uint(__fadd_rn(r, kRoundMagic));
-}
-
-__device__ __forceinline__ uint32_t pack4u(uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
-  const uint32_t lo = __byte_perm(a, b, 0x0040);
-  const uint32_t hi = __byte_perm(c, d, 0x0040);
-  return __byte_perm(lo, hi, 0x5410);
-}
-__device__ __forceinline__ void store_codes(int8_t* dst, const uint32_t (&b)[8]) {
-  uint2 pk;
-  pk.x = pack4u(b[0], b[1], b[2], b[3]);
-  pk.y = pack4u(b[4], b[5], b[6], b[7]);
-  *reinterpret_cast<uint2*>(dst) = pk;
 }
 
 // Producer (one thread): streams rows r0 .. r0+R-1 of P.a.x into the ring,
@@ -542,8 +519,8 @@ __global__ void __launch_bounds__(kThreads, NB) rowpipe_kernel(const Pipe P) {
               cmax[m * 8 + 2 * e] = fmaxf(cmax[m * 8 + 2 * e], fabsf(x[e].x));
               cmax[m * 8 + 2 * e + 1] = fmaxf(cmax[m * 8 + 2 * e + 1], fabsf(x[e].y));
             } else {
-              atomicMax(&colmax_s[c * 8 + 2 * e], __float_as_uint(fabsf(x[e].x)));
-              atomicMax(&colmax_s[c * 8 + 2 * e + 1], __float_as_uint(fabsf(x[e].y)));
+              atomicMax(&colmax_s[c * 8 + 2 * e], peak_bits(fabsf(x[e].x)));
+              atomicMax(&colmax_s[c * 8 + 2 * e + 1], peak_bits(fabsf(x[e].y)));
             }
           }
         });

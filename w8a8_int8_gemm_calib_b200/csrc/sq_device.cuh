@@ -59,6 +59,42 @@ __device__ __forceinline__ void unpack(const Raw8<uint16_t>& r, float (&v)[8]) {
   v[6] = bf16lo(r.a.w); v[7] = bf16hi(r.a.w);
 }
 
+// Q(y; Delta) given inv = 1/Delta, as the fp32 whose low byte is the code:
+// r = y * inv is clamped to [-127, 127] (NaN -> 0) and 1.5 * 2^23 is added;
+// the fp32 addition rounds r to the nearest integer, ties to even, and the
+// low byte of the sum's bit pattern is the two's-complement code (the
+// constant's low byte is zero).  This equals round-half-even then clamp,
+// without the quarter-rate float-to-int conversion.  count: values that
+// round outside [-127, 127] are counted in `clipped`.
+constexpr float kRoundMagic = 12582912.0f;  // 1.5 * 2^23
+__device__ __forceinline__ uint32_t qbits(float y, float inv, bool count, unsigned& clipped) {
+  float r = __fmul_rn(y, inv);
+  if (count) clipped += fabsf(r) >= 127.5f;  // rounds outside [-127, 127]
+  r = (r != r) ? 0.0f : r;
+  r = fminf(fmaxf(r, -127.0f), 127.0f);
+  return __float_as_uint(__fadd_rn(r, kRoundMagic));
+}
+
+// Low bytes of four qbits results, packed little-endian.
+__device__ __forceinline__ uint32_t pack4u(uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
+  const uint32_t lo = __byte_perm(a, b, 0x0040);
+  const uint32_t hi = __byte_perm(c, d, 0x0040);
+  return __byte_perm(lo, hi, 0x5410);
+}
+__device__ __forceinline__ void store_codes(int8_t* dst, const uint32_t (&b)[8]) {
+  uint2 pk;
+  pk.x = pack4u(b[0], b[1], b[2], b[3]);
+  pk.y = pack4u(b[4], b[5], b[6], b[7]);
+  *reinterpret_cast<uint2*>(dst) = pk;
+}
+
+// The fp32 bit pattern of a magnitude |y| for an unsigned atomic max (the
+// order of the patterns of non-negative floats is their numeric order); a
+// NaN gives 0, so that column peaks skip NaN as fmaxf does.
+__device__ __forceinline__ unsigned int peak_bits(float a) {
+  return a != a ? 0u : __float_as_uint(a);
+}
+
 // 8 consecutive fp32 parameters (gamma, beta, multipliers), L1-cached.
 __device__ __forceinline__ void load8(const float* p, float (&v)[8]) {
   float4 a = __ldg(reinterpret_cast<const float4*>(p));

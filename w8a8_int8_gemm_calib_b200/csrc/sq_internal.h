@@ -147,4 +147,7 @@ sq_status launch_gemm_noalloc(GemmArgs a, cudaStream_t st);
 // ---------------------------------------------------------------- self test
 cudaError_t launch_wait_selftest(int64_t limit_ns, cudaStream_t st);
 
+// ---------------------------------------------------------------- measurement
+cudaError_t launch_mma_probe(int64_t kblocks, int grid, cudaStream_t st);
+
 }  // namespace sq
