@@ -107,6 +107,35 @@ def test_gemm_short_k_epilogue(sq, orc, M, N, K):
     assert_bits_equal(y, y_want, "y")
 
 
+# Shapes on the CTA-pair kernel (more than 128 tokens, more than four
+# k-blocks): 256-row tiles shared by two CTAs, each CTA holding 128 rows of A
+# and half the tile's rows of B.  Tokens within one pair tile (the odd CTA's
+# rows partly or wholly past M), ragged rows and columns, odd N (direct
+# stores), both tile widths (192 when every tile fits in one wave, 256 for
+# 2048 x 4096), and more tiles than pairs (the persistent loop wraps).
+PAIR_SHAPES = [(129, 257, 1040), (200, 300, 640), (256, 256, 1024), (257, 200, 2048),
+               (1000, 777, 640), (2048, 4096, 1024), (4100, 1000, 640)]
+
+
+@pytest.mark.parametrize("M,N,K", PAIR_SHAPES)
+@pytest.mark.parametrize("out", ["f32", "bf16"])
+def test_gemm_cta_pair_shapes(sq, orc, M, N, K, out):
+    xq, wq, act, ws = _operands(M, N, K, M * 13 + N * 5 + K)
+    rows = None
+    if M * N * K > 1 << 31:  # sampled rows (every column) for the large ones
+        r = np.random.default_rng(M + K)
+        rows = np.unique(np.concatenate([
+            [0, 1, 127, 128, 255, 256, M // 2, M - 2, M - 1],
+            r.integers(0, M, 24)]).clip(0, M - 1)).astype(np.int64)
+    y_want, acc_want = orc.gemm_w8a8(xq, wq, act, ws, per_token=True, rows=rows,
+                                     out_bf16=(out == "bf16"))
+    y, acc = _run(sq, xq, wq, act, ws, True, out, workspace=sq.Workspace())
+    if rows is not None:
+        y, acc = y[rows], acc[rows]
+    assert_bits_equal(acc, acc_want, "acc")
+    assert_bits_equal(y, y_want, "y")
+
+
 def test_gemm_without_acc_dump(sq, orc):
     M, N, K = 300, 520, 1024
     xq, wq, act, ws = _operands(M, N, K, 5)

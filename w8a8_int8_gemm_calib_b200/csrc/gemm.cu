@@ -43,6 +43,7 @@ constexpr int THREADS = 192;  // small-M kernel: TMA, MMA and 4 epilogue warps
 constexpr int GROUP_M = 16;  // tile raster: 16 row blocks share each column sweep
 constexpr uint64_t kWaitNs = 4000000000ull;   // 4 s: far above any pipeline step
 constexpr uint64_t kDrainNs = 1000000000ull;  // waits for copies already in flight
+constexpr uint64_t kPairGraceNs = 2000000ull;   // after a time-out: the peer's copies land
 // Output staging for the TMA-store epilogue: per epilogue warp, buffers of
 // 32 rows x 64 bytes (32 bf16 or 16 fp32 columns), 64-byte swizzled.
 constexpr int EPI_BUF = 32 * 64;
@@ -55,11 +56,15 @@ constexpr int EPI_BUF = 32 * 64;
 // 32-lane quarter of the accumulator and take every third 32-column chunk,
 // for short K, where the epilogue and not the main loop sets the tile time
 // and one warp per quarter leaves it latency-bound.
-template <int TBN, int EPI_NB = 2, int EPI_W = 4>
+template <int TBN, int EPI_NB = 2, int EPI_W = 4, bool PAIR = false>
 struct TcCfg {
   static_assert(EPI_W == 4 || EPI_W == 12, "one or three warps per accumulator quarter");
   static constexpr int THREADS = 64 + 32 * EPI_W;  // TMA warp, MMA warp, epilogue
-  static constexpr int B_BYTES = TBN * BK;
+  // a CTA pair's tile is 256 x TBN: each CTA holds 128 rows of A and TBN/2
+  // rows of B per stage
+  static constexpr int TILE_M = PAIR ? 2 * BM : BM;
+  static constexpr int B_ROWS = PAIR ? TBN / 2 : TBN;
+  static constexpr int B_BYTES = B_ROWS * BK;
   static constexpr int STAGE = A_BYTES + B_BYTES;
   static constexpr int EPI_BYTES = EPI_W * EPI_NB * EPI_BUF;
   // as many stages as fit: with 4 epilogue warps of 2 staging buffers, 4 at
@@ -90,11 +95,12 @@ struct Params {
   double* err_part;
 };
 
-__device__ __forceinline__ void tile_coords(int tile, int m_tiles, int n_tiles, int& mb, int& nb) {
-  const int per_group = GROUP_M * n_tiles;
+__device__ __forceinline__ void tile_coords(int tile, int m_tiles, int n_tiles, int& mb, int& nb,
+                                            int group_m = GROUP_M) {
+  const int per_group = group_m * n_tiles;
   const int group = tile / per_group;
-  const int first = group * GROUP_M;
-  const int gm = min(m_tiles - first, GROUP_M);
+  const int first = group * group_m;
+  const int gm = min(m_tiles - first, group_m);
   const int r = tile - group * per_group;
   mb = first + r % gm;
   nb = r / gm;
@@ -198,11 +204,25 @@ __device__ __forceinline__ void store_chunk(const Params& p, size_t yrow, int co
   }
 }
 
-template <bool BF16, int TBN, bool BATCH, int EPI_NB, int EPI_W, bool ERR>
-__global__ void __launch_bounds__(TcCfg<TBN, EPI_NB, EPI_W>::THREADS, 1)
+// PAIR: a cluster of two CTAs (an even and an odd one, on two SMs) shares
+// each 256 x TBN tile through tcgen05 .cta_group::2 -- every CTA loads 128
+// rows of A and TBN/2 rows of B per k-block into its own shared memory, the
+// even CTA issues the MMAs for both, and each CTA drains its own 128 rows of
+// the accumulator.  Per SM that moves (16 + TBN/16) KB per k-block from L2
+// instead of (16 + TBN/8) KB, for the same multiply-adds.  Both CTAs walk
+// the same tile sequence; the odd CTA's loads complete on the even CTA's
+// stage barriers, the even CTA's commits arrive on both CTAs' barriers, and
+// both CTAs' epilogue warps release the accumulator on the even CTA's
+// barrier.  No load is multicast.
+template <bool BF16, int TBN, bool BATCH, int EPI_NB, int EPI_W, bool ERR, bool PAIR = false>
+__global__ void __launch_bounds__(TcCfg<TBN, EPI_NB, EPI_W, PAIR>::THREADS, 1)
 gemm_w8a8_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                     const __grid_constant__ CUtensorMap tmY, const Params p) {
-  using C = TcCfg<TBN, EPI_NB, EPI_W>;
+  static_assert(!PAIR || (!BATCH && !ERR), "CTA pairs serve the plain GEMM");
+  using C = TcCfg<TBN, EPI_NB, EPI_W, PAIR>;
+  constexpr int TILE_M = C::TILE_M;
+  constexpr int B_ROWS = C::B_ROWS;
+  constexpr int GROUP = PAIR ? GROUP_M / 2 : GROUP_M;  // same 2048-row bands
   constexpr int STAGES = C::STAGES;
   constexpr int B_BYTES = C::B_BYTES;
   constexpr int STAGE_BYTES = C::STAGE;
@@ -225,6 +245,12 @@ gemm_w8a8_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
   auto tfull_bar = [&](int b) { return tc::smem_u32(bars + 2 * STAGES + b); };
   auto tempty_bar = [&](int b) { return tc::smem_u32(bars + 2 * STAGES + 2 + b); };
   const uint32_t drain_bar = tc::smem_u32(bars + 2 * STAGES + 4);
+  // the CTA's place in its pair (0, the even CTA, issues the MMAs), and the
+  // persistent loop's unit: one tile per CTA, or per pair
+  const uint32_t rank = PAIR ? tc::cluster_ctarank() : 0u;
+  const bool leader = rank == 0;
+  const int unit0 = PAIR ? (int)(blockIdx.x >> 1) : (int)blockIdx.x;
+  const int units = PAIR ? (int)(gridDim.x >> 1) : (int)gridDim.x;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
@@ -233,7 +259,8 @@ gemm_w8a8_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
     }
     for (int b = 0; b < 2; ++b) {
       tc::mbar_init(tfull_bar(b), 1);
-      tc::mbar_init(tempty_bar(b), EPI_W);  // one arrival per epilogue warp
+      // one arrival per epilogue warp (of both CTAs of a pair)
+      tc::mbar_init(tempty_bar(b), PAIR ? 2 * EPI_W : EPI_W);
     }
     tc::mbar_init(drain_bar, 1);
     *abort_flag = 0;
@@ -242,11 +269,17 @@ gemm_w8a8_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
     tc::tma_prefetch_desc(&tmB);
   }
   if (warp == 1) {
-    tc::tmem_alloc(tc::smem_u32(tmem_slot), TMEM_COLS);
-    tc::tmem_relinquish();
+    if constexpr (PAIR) {
+      tc::tmem_alloc_pair(tc::smem_u32(tmem_slot), TMEM_COLS);
+      tc::tmem_relinquish_pair();
+    } else {
+      tc::tmem_alloc(tc::smem_u32(tmem_slot), TMEM_COLS);
+      tc::tmem_relinquish();
+    }
   }
   tc::tc_fence_before();
-  __syncthreads();
+  if constexpr (PAIR) tc::cluster_sync();  // the peer's barriers are initialised
+  else __syncthreads();
   tc::tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
   pdl_wait();  // the prologue above touches no global memory
@@ -256,14 +289,28 @@ gemm_w8a8_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
     if (tc::elect_one()) {
       uint32_t stage = 0, phase = 0, issued = 0, issued_par = 0;
       bool ok = true;
-      for (int tile = blockIdx.x; ok && tile < p.num_tiles; tile += gridDim.x) {
+      for (int tile = unit0; ok && tile < p.num_tiles; tile += units) {
         int mb, nb;
         const int b = BATCH ? tile / p.tiles_per_batch : 0;
-        tile_coords(tile - b * p.tiles_per_batch, p.m_tiles, p.n_tiles, mb, nb);
+        tile_coords(tile - b * p.tiles_per_batch, p.m_tiles, p.n_tiles, mb, nb, GROUP);
         for (int kb = 0; kb < p.nk; ++kb) {
           if (!tc::mbar_wait(empty_bar(stage), phase ^ 1u, abort_flag, kWaitNs, p.status)) {
             ok = false;
             break;
+          }
+          if constexpr (PAIR) {
+            // both CTAs' bytes complete on the even CTA's barrier, which
+            // alone expects them
+            const uint32_t fb = tc::mapa_shared(full_bar(stage), 0);
+            if (leader) tc::mbar_arrive_expect_tx(full_bar(stage), 2 * STAGE_BYTES);
+            tc::tma_load_2d_pair(tc::smem_u32(sA + stage * A_BYTES), &tmA, kb * BK,
+                                 mb * TILE_M + (int)rank * BM, fb);
+            tc::tma_load_2d_pair(tc::smem_u32(sB + stage * B_BYTES), &tmB, kb * BK,
+                                 nb * BN + (int)rank * B_ROWS, fb);
+            issued |= 1u << stage;
+            issued_par = (issued_par & ~(1u << stage)) | (phase << stage);
+            if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+            continue;
           }
           tc::mbar_arrive_expect_tx(full_bar(stage), STAGE_BYTES);
           if constexpr (BATCH) {
@@ -285,19 +332,27 @@ gemm_w8a8_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
       if (!ok) {
         // let every load already issued land before the CTA exits
         int never = 0;
-        for (int s = 0; s < STAGES; ++s)
-          if (issued & (1u << s))
-            tc::mbar_wait(full_bar(s), (issued_par >> s) & 1u, &never, kDrainNs, p.status);
+        if (leader)
+          for (int s = 0; s < STAGES; ++s)
+            if (issued & (1u << s))
+              tc::mbar_wait(full_bar(s), (issued_par >> s) & 1u, &never, kDrainNs, p.status);
+        if constexpr (PAIR) {
+          // the odd CTA's copies complete on the even CTA's barriers, which
+          // it cannot wait on: a fixed grace period lets them land
+          const uint64_t t0 = global_ns();
+          while (global_ns() - t0 < kPairGraceNs) {
+          }
+        }
       }
     }
     __syncwarp();
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
-    if (tc::elect_one()) {
-      constexpr uint32_t idesc = tc::idesc_i8(BM, BN);
+    if (leader && tc::elect_one()) {
+      constexpr uint32_t idesc = tc::idesc_i8(TILE_M, BN);
       uint32_t stage = 0, phase = 0, abuf = 0, aphase = 0;
       bool ok = true;
-      for (int tile = blockIdx.x; ok && tile < p.num_tiles; tile += gridDim.x) {
+      for (int tile = unit0; ok && tile < p.num_tiles; tile += units) {
         if (!tc::mbar_wait(tempty_bar(abuf), aphase ^ 1u, abort_flag, kWaitNs, p.status)) {
           ok = false;
           break;
@@ -313,19 +368,27 @@ gemm_w8a8_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
           const uint32_t a0 = tc::smem_u32(sA + stage * A_BYTES);
           const uint32_t b0 = tc::smem_u32(sB + stage * B_BYTES);
 #pragma unroll
-          for (int k = 0; k < BK / UK; ++k)
-            tc::mma_i8(d, tc::desc_k_sw128(a0 + k * UK), tc::desc_k_sw128(b0 + k * UK), idesc,
-                       (kb | k) != 0);
-          tc::mma_commit(empty_bar(stage));
+          for (int k = 0; k < BK / UK; ++k) {
+            if constexpr (PAIR)
+              tc::mma_i8_pair(d, tc::desc_k_sw128(a0 + k * UK), tc::desc_k_sw128(b0 + k * UK),
+                              idesc, (kb | k) != 0);
+            else
+              tc::mma_i8(d, tc::desc_k_sw128(a0 + k * UK), tc::desc_k_sw128(b0 + k * UK), idesc,
+                         (kb | k) != 0);
+          }
+          if constexpr (PAIR) tc::mma_commit_pair(empty_bar(stage), 0x3);
+          else tc::mma_commit(empty_bar(stage));
           if (++stage == STAGES) { stage = 0; phase ^= 1u; }
         }
         if (!ok) break;
-        tc::mma_commit(tfull_bar(abuf));
+        if constexpr (PAIR) tc::mma_commit_pair(tfull_bar(abuf), 0x3);
+        else tc::mma_commit(tfull_bar(abuf));
         abuf ^= 1u;
         if (abuf == 0) aphase ^= 1u;
       }
       // every MMA issued so far must finish before TMEM is released
-      tc::mma_commit(drain_bar);
+      if constexpr (PAIR) tc::mma_commit_pair(drain_bar, 0x1);
+      else tc::mma_commit(drain_bar);
       int never = 0;
       tc::mbar_wait(drain_bar, 0, &never, kDrainNs, p.status);
     }
@@ -338,13 +401,13 @@ gemm_w8a8_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
     uint32_t nstore = 0;  // TMA stores issued by this warp (selects the buffer)
     double e_num = 0.0, e_den = 0.0;  // error mode: this lane's sums
     uint32_t abuf = 0, aphase = 0;
-    for (int tile = blockIdx.x; tile < p.num_tiles; tile += gridDim.x) {
+    for (int tile = unit0; tile < p.num_tiles; tile += units) {
       int mb, nb;
       const int b = BATCH ? tile / p.tiles_per_batch : 0;
-      tile_coords(tile - b * p.tiles_per_batch, p.m_tiles, p.n_tiles, mb, nb);
+      tile_coords(tile - b * p.tiles_per_batch, p.m_tiles, p.n_tiles, mb, nb, GROUP);
       if (!tc::mbar_wait(tfull_bar(abuf), aphase, abort_flag, kWaitNs, p.status)) break;
       tc::tc_fence_after();
-      const int row0 = mb * BM + quarter * 32;
+      const int row0 = mb * TILE_M + (int)rank * BM + quarter * 32;
       const int row = row0 + lane;
       const bool row_ok = row < p.M;
       const size_t yrow = (size_t)b * (size_t)p.M + (size_t)row;  // output row of [batch*M, N]
@@ -431,7 +494,10 @@ gemm_w8a8_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
       }
       tc::tc_fence_before();
       __syncwarp();
-      if (lane == 0) tc::mbar_arrive(tempty_bar(abuf));
+      if (lane == 0) {
+        if constexpr (PAIR) tc::mbar_arrive_cluster(tc::mapa_shared(tempty_bar(abuf), 0));
+        else tc::mbar_arrive(tempty_bar(abuf));
+      }
       abuf ^= 1u;
       if (abuf == 0) aphase ^= 1u;
     }
@@ -454,9 +520,13 @@ gemm_w8a8_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
 
   tc::tc_fence_before();
   __syncthreads();
+  // neither CTA of a pair leaves while the other may still reach its
+  // barriers or shared memory
+  if constexpr (PAIR) tc::cluster_sync();
   if (warp == 1) {
     tc::tc_fence_after();
-    tc::tmem_dealloc(tmem_base, TMEM_COLS);
+    if constexpr (PAIR) tc::tmem_dealloc_pair(tmem_base, TMEM_COLS);
+    else tc::tmem_dealloc(tmem_base, TMEM_COLS);
   }
 }
 
@@ -855,6 +925,46 @@ cudaError_t launch_tc(const CUtensorMap& ta, const CUtensorMap& tb, const CUtens
                     dim3(C::THREADS), C::SMEM, st, ta, tb, ty, p);
 }
 
+// The CTA-pair kernel: `pairs` clusters of two CTAs.  The number of pairs
+// that can be resident at once is queried once per device and tile width;
+// a persistent launch never asks for more.
+template <bool BF16, int TBN>
+cudaError_t launch_tc_pair(const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& ty,
+                           const Params& p, int pairs, cudaStream_t st) {
+  using C = TcCfg<TBN, 2, 4, true>;
+  auto kern = gemm_w8a8_tc_kernel<BF16, TBN, false, 2, 4, false, true>;
+  static std::once_flag once[64];
+  static cudaError_t attr_err[64];
+  static int max_pairs[64];
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess || dev < 0 || dev >= 64) return e != cudaSuccess ? e : cudaErrorInvalidDevice;
+  std::call_once(once[dev], [&] {
+    attr_err[dev] = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)C::SMEM);
+    if (attr_err[dev] != cudaSuccess) return;
+    cudaLaunchConfig_t cfg{};
+    cfg.gridDim = dim3(2 * (unsigned)(sm_count() / 2));
+    cfg.blockDim = dim3(C::THREADS);
+    cfg.dynamicSmemBytes = C::SMEM;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    int n = 0;
+    attr_err[dev] = cudaOccupancyMaxActiveClusters(&n, kern, &cfg);
+    max_pairs[dev] = n;
+  });
+  if (attr_err[dev] != cudaSuccess) return attr_err[dev];
+  if (max_pairs[dev] < 1) return cudaErrorInvalidConfiguration;
+  if (pairs > max_pairs[dev]) pairs = max_pairs[dev];
+  return launch_pdl_cluster(kern, dim3(2 * pairs), dim3(C::THREADS), C::SMEM, st, 2u, ta, tb, ty,
+                            p);
+}
+
 // Tile width for the large-M kernel: the per-tile time grows with the width,
 // and a partly filled last wave costs a whole tile time, so take the width
 // with the smaller (waves x width) -- plus a fixed per-tile cost.
@@ -899,6 +1009,28 @@ cudaError_t launch_tiles(const CUtensorMap& ta, const CUtensorMap& tb, const CUt
   }
   return cudaErrorInvalidValue;
 }
+
+// Tile width for the CTA-pair kernel (256-row tiles, one per pair of SMs),
+// by the same wave cost as pick_tile_n.
+int pick_tile_n_pair(int64_t M, int64_t N, int sms) {
+  const int64_t mt = (M + 2 * BM - 1) / (2 * BM);
+  const int64_t units = sms / 2;
+  int best = 256;
+  int64_t best_cost = -1;
+  for (int tbn : {256, 192}) {
+    const int64_t tiles = mt * ((N + tbn - 1) / tbn);
+    const int64_t waves = (tiles + units - 1) / units;
+    const int64_t cost = waves * (tbn + 16);
+    if (best_cost < 0 || cost < best_cost) { best = tbn; best_cost = cost; }
+  }
+  return best;
+}
+
+// The plain GEMM takes CTA pairs for every M the large-M kernel serves,
+// except short K (at most four k-blocks), where the epilogue and not the
+// operand traffic sets the pace and the single-CTA kernel's twelve
+// epilogue warps serve it better.
+bool use_pair(int64_t M, int64_t K) { return M > 128 && (K + BK - 1) / BK > 4; }
 
 constexpr int64_t kSmallMaxM = 128;
 
@@ -1026,17 +1158,21 @@ struct LargeSetup {
   CUtensorMap ta, tb, ty;
   Params p;
   int tbn, grid;
+  bool pair;  // grid counts CTA pairs
 };
-bool setup_large(const GemmArgs& a, unsigned int* sw, LargeSetup* L) {
-  L->tbn = pick_tile_n(a.M, a.N, sm_count());
+bool setup_large(const GemmArgs& a, unsigned int* sw, LargeSetup* L, bool allow_pair) {
+  L->pair = allow_pair && use_pair(a.M, a.K);
+  L->tbn = L->pair ? pick_tile_n_pair(a.M, a.N, sm_count()) : pick_tile_n(a.M, a.N, sm_count());
+  const int tile_m = L->pair ? 2 * BM : BM;
+  const int b_rows = L->pair ? L->tbn / 2 : L->tbn;
   if (!make_tmap(&L->ta, a.xq, (uint64_t)a.K, (uint64_t)a.M, BM) ||
-      !make_tmap(&L->tb, a.wq, (uint64_t)a.K, (uint64_t)a.N, (uint32_t)L->tbn))
+      !make_tmap(&L->tb, a.wq, (uint64_t)a.K, (uint64_t)a.N, (uint32_t)b_rows))
     return false;
   memset(&L->ty, 0, sizeof L->ty);
   Params& p = L->p;
   p = Params{};
   p.M = (int)a.M; p.N = (int)a.N; p.K = (int)a.K;
-  p.m_tiles = (int)((a.M + BM - 1) / BM);
+  p.m_tiles = (int)((a.M + tile_m - 1) / tile_m);
   p.n_tiles = (int)((a.N + L->tbn - 1) / L->tbn);
   p.num_tiles = p.m_tiles * p.n_tiles;
   p.tiles_per_batch = p.num_tiles;
@@ -1048,7 +1184,7 @@ bool setup_large(const GemmArgs& a, unsigned int* sw, LargeSetup* L) {
   p.y = a.y;
   p.acc = a.acc_out;
   p.status = sw;
-  L->grid = sm_count();
+  L->grid = L->pair ? sm_count() / 2 : sm_count();
   if (L->grid > p.num_tiles) L->grid = p.num_tiles;
   return true;
 }
@@ -1081,13 +1217,23 @@ sq_status launch_gemm(const GemmArgs& a, cudaStream_t st) {
     return SQ_OK;
   }
   LargeSetup L;
-  if (!setup_large(a, sw, &L))
+  if (!setup_large(a, sw, &L, true))
     return fail(SQ_ERR_CUDA, "sq_gemm_w8a8: cuTensorMapEncodeTiled failed");
   // TMA stores need 16-byte row pitches; other widths store directly
   const bool bf16 = a.yt == SQ_BF16;
   L.p.tma_store = (a.N % (bf16 ? 8 : 4)) == 0 &&
                   make_tmap_out(&L.ty, a.y, (uint64_t)a.N, (uint64_t)a.M, bf16);
-  const cudaError_t e = launch_tiles<false>(L.ta, L.tb, L.ty, L.p, L.grid, L.tbn, bf16, st);
+  cudaError_t e;
+  if (L.pair) {
+    if (L.tbn == 256)
+      e = bf16 ? launch_tc_pair<true, 256>(L.ta, L.tb, L.ty, L.p, L.grid, st)
+               : launch_tc_pair<false, 256>(L.ta, L.tb, L.ty, L.p, L.grid, st);
+    else
+      e = bf16 ? launch_tc_pair<true, 192>(L.ta, L.tb, L.ty, L.p, L.grid, st)
+               : launch_tc_pair<false, 192>(L.ta, L.tb, L.ty, L.p, L.grid, st);
+  } else {
+    e = launch_tiles<false>(L.ta, L.tb, L.ty, L.p, L.grid, L.tbn, bf16, st);
+  }
   if (e != cudaSuccess) return fail(SQ_ERR_CUDA, "sq_gemm_w8a8: %s", cudaGetErrorString(e));
   return SQ_OK;
 }
@@ -1102,7 +1248,7 @@ sq_status launch_gemm_err(const GemmArgs& a, const float* y_ref, double* part, i
   if (!sw) return fail(SQ_ERR_CUDA, "sq_alpha_sweep: device status word unavailable");
   if (!gemm_err_ok(a.M, a.N)) return fail(SQ_ERR_UNSUPPORTED, "sq_alpha_sweep: error-mode GEMM shape");
   LargeSetup L;
-  if (!setup_large(a, sw, &L))
+  if (!setup_large(a, sw, &L, false))
     return fail(SQ_ERR_CUDA, "sq_alpha_sweep: cuTensorMapEncodeTiled failed");
   L.p.tma_store = 0;  // nothing is stored
   L.p.err_ref = y_ref;
