@@ -33,7 +33,8 @@ on bounded samples of the same workload, each step extrapolated linearly to
 the full workload.
 `--profile-call NAME` only runs the named call of the step `--steps` times
 after the warm-up steps (for an ncu capture of one kernel) and prints no
-line; `--tokens T` shrinks the runtime token count for such a capture.
+line; `--tokens T` and `--cal-tokens T` shrink the runtime and calibration
+token counts for such a capture.
 """
 from __future__ import annotations
 
@@ -95,6 +96,8 @@ def parse():
                     help="run only this call (after the warm-up steps) --steps times; no line")
     ap.add_argument("--tokens", type=int, default=None,
                     help="runtime tokens of the workload's linear (profiling of smaller cases)")
+    ap.add_argument("--cal-tokens", type=int, default=None,
+                    help="calibration tokens of the workload's linear (profiling of smaller cases)")
     return ap.parse_args()
 
 
@@ -105,6 +108,8 @@ def pick_linear(args, workload=None):
         lin = next(l for l in wl.linears if l.name == args.linear)
     if args.tokens and workload is None:
         lin = dataclasses.replace(lin, T=int(args.tokens))
+    if args.cal_tokens and workload is None:
+        lin = dataclasses.replace(lin, T_cal=int(args.cal_tokens))
     return wl, lin
 
 

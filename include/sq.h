@@ -322,10 +322,13 @@ sq_status sq_gemm_w8a8_bias(const int8_t* xq, const int8_t* wq, int64_t M,
  * device memory that the library reserves on every GPU that loads it, held
  * until the process exits.
  *
- *   - Shapes whose sq_gemm_workspace_bytes(M,N,K) exceeds 8 MiB are refused
- *     with SQ_ERR_WORKSPACE before anything is launched (at 148 SMs that is
- *     roughly M > 52 tokens on the stream-K path); shapes off that path need
- *     no scratch and are always served.
+ *   - A shape is refused with SQ_ERR_WORKSPACE, before anything is
+ *     launched, exactly when sq_gemm_workspace_bytes(M,N,K) > 8,388,608.
+ *     On the stream-K path that size is the tile counters (4 bytes per 128
+ *     output channels, rounded up to 256) plus G * 2 * M * 512 bytes, G =
+ *     min(SM count, 128-channel tiles x 128-byte k-blocks); with G = 148 the
+ *     largest M served is 55.  Shapes off that path need no scratch and are
+ *     always served.
  *   - The first call on a device looks up the array's device address with
  *     cudaGetSymbolAddress, so make that first call before any stream capture
  *     begins on that device.

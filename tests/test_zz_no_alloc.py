@@ -91,3 +91,32 @@ def test_noalloc_refuses_shapes_beyond_its_scratch(sq):
     assert "static scratch" in sq._lib.last_error()
     sq.sq_sync_status()
     assert bool((y == 3.0).all())  # nothing was launched
+
+
+def test_noalloc_boundary_on_the_stream_k_path(sq):
+    """At the edge of the 8 MiB array: on a stream-K shape whose units cover
+    every SM (1000 output channels, K = 12288), the largest token count whose
+    scratch fits (55 at 148 SMs: 256 + 148 * 2 * 55 * 128 * 4 bytes) is
+    served -- twice, bit-exact against the workspace entry point -- and one
+    token more is refused before any launch."""
+    N, K = 1000, 12288
+    fits = [m for m in range(9, 129)
+            if 0 < sq.sq_gemm_workspace_bytes(m, N, K) <= STATIC_SCRATCH_BYTES]
+    M = max(fits)
+    assert sq.sq_gemm_workspace_bytes(M + 1, N, K) > STATIC_SCRATCH_BYTES
+    xq, wq, act, ws = _inputs(M + 1, N, K, 11)
+    y_ref = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
+    a_ref = torch.empty((M, N), dtype=torch.int32, device="cuda")
+    sq.sq_gemm_w8a8(xq[:M], wq, act[:M], ws, y_ref, acc_out=a_ref, workspace=sq.Workspace())
+    sq.sq_sync_status()
+    for _ in range(2):
+        y = torch.full((M, N), float("nan"), dtype=torch.bfloat16, device="cuda")
+        acc = torch.zeros((M, N), dtype=torch.int32, device="cuda")
+        assert _noalloc(sq, xq[:M], wq, act[:M], ws, y, acc) == 0, sq._lib.last_error()
+        sq.sq_sync_status()
+        assert torch.equal(acc, a_ref)
+        assert torch.equal(y.view(torch.int16), y_ref.view(torch.int16))
+    y = torch.full((M + 1, N), 3.0, dtype=torch.bfloat16, device="cuda")
+    assert _noalloc(sq, xq, wq, act, ws, y, None) == 8  # SQ_ERR_WORKSPACE
+    sq.sq_sync_status()
+    assert bool((y == 3.0).all())
