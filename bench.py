@@ -66,7 +66,11 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 CALLS = ["calib_absmax", "smooth_scales", "fuse_weights_q8", "ln_smooth_quant_act", "gemm_w8a8"]
 # DRAM bytes (read + write) of one launch of the step's GEMM, from an ncu
 # capture of the current kernel (None until one exists for the workload)
-GEMM_DRAM_TRAFFIC = {}
+GEMM_DRAM_TRAFFIC = {
+    "large_prefill_k8192": (2978473216, "ncu, one launch of gemm_w8a8_tc_kernel<1,256,0,2,4,0,1> "
+                            "(CTA pairs) at 16384 x 28672 x 8192: dram__bytes_read.sum 2056.2 MB + "
+                            "dram__bytes_write.sum 922.3 MB"),
+}
 
 
 def load_peaks():

@@ -113,12 +113,12 @@ __device__ __forceinline__ void load_cols32(const float* src, int col0, int N, f
     const float4* s4 = reinterpret_cast<const float4*>(src + col0);
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
-      const float4 t = __ldg(s4 + i);
+      const float4 t = __ldcg(s4 + i);
       v[4 * i] = t.x; v[4 * i + 1] = t.y; v[4 * i + 2] = t.z; v[4 * i + 3] = t.w;
     }
   } else {
 #pragma unroll
-    for (int i = 0; i < 32; ++i) v[i] = col0 + i < N ? __ldg(src + col0 + i) : 0.0f;
+    for (int i = 0; i < 32; ++i) v[i] = col0 + i < N ? __ldcg(src + col0 + i) : 0.0f;
   }
 }
 
@@ -137,7 +137,7 @@ __device__ __forceinline__ void dequant_chunk(const Params& p, int b, int col0,
                                               float (&yv)[32]) {
   float ws[32];
   if (BATCH && p.w_per_tensor) {
-    const float w = __ldg(p.w_scale + b);
+    const float w = __ldcg(p.w_scale + b);
 #pragma unroll
     for (int i = 0; i < 32; ++i) ws[i] = w;
   } else {
@@ -414,8 +414,8 @@ gemm_w8a8_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
       const int row = row0 + lane;
       const bool row_ok = row < p.M;
       const size_t yrow = (size_t)b * (size_t)p.M + (size_t)row;  // output row of [batch*M, N]
-      const float as = p.per_token ? (row_ok ? __ldg(p.act_scale + yrow) : 0.0f)
-                                   : __ldg(p.act_scale + b);
+      const float as = p.per_token ? (row_ok ? __ldcg(p.act_scale + yrow) : 0.0f)
+                                   : __ldcg(p.act_scale + b);
       const uint32_t taddr = tmem_base + abuf * BN + ((uint32_t)(quarter * 32) << 16);
 #pragma unroll 1
       for (int c = chunk0; c < BN / 32; c += EPI_W / 4) {
@@ -594,13 +594,13 @@ __device__ __forceinline__ void tmem_ld_n(uint32_t taddr, uint32_t (&r)[CH]) {
 template <bool BF16, int CH>
 __device__ __forceinline__ void small_store(const SmallParams& p, int n, int t0, const int32_t (&v)[CH]) {
   if (n >= p.N) return;
-  const float ws = __ldg(p.w_scale + n);
-  const float bn = p.bias ? __ldg(p.bias + n) : 0.0f;
+  const float ws = __ldcg(p.w_scale + n);
+  const float bn = p.bias ? __ldcg(p.bias + n) : 0.0f;
 #pragma unroll
   for (int i = 0; i < CH; ++i) {
     const int t = t0 + i;
     if (t < p.M) {
-      const float as = __ldg(p.act_scale + (p.per_token ? t : 0));
+      const float as = __ldcg(p.act_scale + (p.per_token ? t : 0));
       float y = dequant((uint32_t)v[i], as, ws);
       if (p.bias) y = __fadd_rn(y, bn);
       const size_t o = (size_t)t * (size_t)p.N + (size_t)n;

@@ -175,7 +175,7 @@ strip_quant_kernel(const T* __restrict__ x, int64_t T_, int64_t K, int64_t rows_
 #pragma unroll
   for (int e = 0; e < 8; ++e) m8[e] = 1.0f;
   if (live && mul) load8(mul + chunk * 8, m8);
-  const float inv = PEAK ? 0.0f : __fdiv_rn(1.0f, __ldg(scale));
+  const float inv = PEAK ? 0.0f : __fdiv_rn(1.0f, __ldcg(scale));
   const bool count = n_clipped != nullptr;
   unsigned clipped = 0;
   float pk = 0.0f;
@@ -389,7 +389,7 @@ row_kernel(RowArgs a) {
   };
 
   float static_inv = 0.0f;
-  if (MODE == ROW_STATIC) static_inv = __fdiv_rn(1.0f, __ldg(a.scale));
+  if (MODE == ROW_STATIC) static_inv = __fdiv_rn(1.0f, __ldcg(a.scale));
   unsigned clipped = 0;
   int parity = 0;
   float peak = 0.0f;  // ROW_PEAK: this thread's running max of |y| (NaN skipped)
@@ -746,7 +746,7 @@ output_error_kernel(const float* __restrict__ y, const float* __restrict__ r, in
   double num = 0.0, den = 0.0;
   for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n;
        i += (int64_t)gridDim.x * blockDim.x) {
-    const double a = (double)__ldg(y + i), b = (double)__ldg(r + i);
+    const double a = (double)__ldcg(y + i), b = (double)__ldcg(r + i);
     const double d = a - b;
     num += d * d;
     den += b * b;

@@ -234,10 +234,10 @@ __device__ __forceinline__ void stage_params(const RowArgs& a, float* pg, float*
       bv[u] = 0.0f;
       if (k < K) {
         if (LN) {
-          gv[u] = __ldg(a.g + k);
-          if (a.b) bv[u] = __ldg(a.b + k);
+          gv[u] = __ldcg(a.g + k);
+          if (a.b) bv[u] = __ldcg(a.b + k);
         } else if (has_mul) {
-          gv[u] = __ldg(a.mul + k);
+          gv[u] = __ldcg(a.mul + k);
         }
       }
     }
@@ -351,7 +351,7 @@ __global__ void __launch_bounds__(kThreads, NB) rowpipe_kernel(const Pipe P) {
 #pragma unroll
     for (int i = 0; i < NC; ++i) cmax[i] = 0.0f;
     float pk[4] = {0.0f, 0.0f, 0.0f, 0.0f};  // ROW_PEAK: running max of |y| (NaN skipped)
-    const float static_inv = MODE == ROW_STATIC ? __fdiv_rn(1.0f, __ldg(a.scale)) : 0.0f;
+    const float static_inv = MODE == ROW_STATIC ? __fdiv_rn(1.0f, __ldcg(a.scale)) : 0.0f;
     const bool count = P.count != 0;
     int parity = 0;
     const int nch = (int)nchunk;  // < 2^14 here: rows fit in shared memory

@@ -22,10 +22,17 @@ template <typename T> struct Raw8;
 template <> struct Raw8<float> { float4 a, b; };
 template <> struct Raw8<uint16_t> { uint4 a; };
 
-// Streaming (read-once) loads: do not keep the line in L1.
+// Loads of data that an earlier kernel of the stream may have written.
+// Every kernel here is launched with programmatic dependent launch: it may
+// start while the kernels before it still run, and only its
+// griddepcontrol.wait orders it after them.  The read-only (.nc) path and
+// L1 are not kept coherent with those writes, so such data -- activations,
+// 1/s, steps, folded parameters, weight scales -- is read at L2 (.cg).
+
+// Streaming (read-once) loads, at L2.
 __device__ __forceinline__ uint4 ld_stream_u4(const void* p) {
   uint4 r;
-  asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
+  asm volatile("ld.global.cg.v4.u32 {%0,%1,%2,%3}, [%4];"
                : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w) : "l"(p));
   return r;
 }
@@ -39,13 +46,13 @@ __device__ __forceinline__ void load_raw(const uint16_t* p, Raw8<uint16_t>& r) {
   r.a = ld_stream_u4(p);
 }
 
-// Cached loads (rows read more than once).
+// Rows read more than once (also at L2).
 __device__ __forceinline__ void load_raw_cached(const float* p, Raw8<float>& r) {
-  r.a = __ldg(reinterpret_cast<const float4*>(p));
-  r.b = __ldg(reinterpret_cast<const float4*>(p) + 1);
+  r.a = __ldcg(reinterpret_cast<const float4*>(p));
+  r.b = __ldcg(reinterpret_cast<const float4*>(p) + 1);
 }
 __device__ __forceinline__ void load_raw_cached(const uint16_t* p, Raw8<uint16_t>& r) {
-  r.a = __ldg(reinterpret_cast<const uint4*>(p));
+  r.a = __ldcg(reinterpret_cast<const uint4*>(p));
 }
 
 __device__ __forceinline__ void unpack(const Raw8<float>& r, float (&v)[8]) {
@@ -95,10 +102,10 @@ __device__ __forceinline__ unsigned int peak_bits(float a) {
   return a != a ? 0u : __float_as_uint(a);
 }
 
-// 8 consecutive fp32 parameters (gamma, beta, multipliers), L1-cached.
+// 8 consecutive fp32 parameters (gamma, beta, multipliers), at L2.
 __device__ __forceinline__ void load8(const float* p, float (&v)[8]) {
-  float4 a = __ldg(reinterpret_cast<const float4*>(p));
-  float4 b = __ldg(reinterpret_cast<const float4*>(p) + 1);
+  float4 a = __ldcg(reinterpret_cast<const float4*>(p));
+  float4 b = __ldcg(reinterpret_cast<const float4*>(p) + 1);
   v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
   v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
 }
