@@ -374,12 +374,13 @@ def kernel_table(lin, per, hbm, int8_peak):
 def measure_int8_peak(sq, torch, dev, clocks_cls):
     """The dense INT8 tensor-core ceiling of this GPU, measured two ways:
     (1) the tcgen05.mma kind::i8 issue rate with the operands in shared
-    memory and no other work (sq_probe_mma_i8, one CTA per SM), in bursts of
+    memory and no other work, one CTA per SM (sq_probe_mma_i8) and on CTA
+    pairs (sq_probe_mma_i8_pair, the GEMM's instruction form), in bursts of
     about 2 ms with idle gaps -- the way the step's GEMM runs in the timed
     region -- and, for context, back to back for ~30 ms launches, where the
     power cap lowers the clock; (2) cuBLAS's INT8 GEMM (torch._int_mm) at
     8192^3.  Best of several launches each, CUDA events on the launching
-    stream, NVML clock sampled during each.  The larger of the burst probe
+    stream, NVML clock sampled during each.  The largest of the burst probes
     and cuBLAS is the roofline's peak."""
     sms = torch.cuda.get_device_properties(dev).multi_processor_count
 
@@ -402,18 +403,30 @@ def measure_int8_peak(sq, torch, dev, clocks_cls):
         return best
 
     out = {}
-    for name, kblocks, reps, gap in (("tcgen05_i8_probe", 8000, 10, 0.05),
-                                     ("tcgen05_i8_probe_sustained", 100_000, 5, 0.0)):
+    pairs = sms // 2
+    for name, kblocks, reps, gap, pair in (
+            ("tcgen05_i8_probe", 8000, 10, 0.05, False),
+            ("tcgen05_i8_pair_probe", 8000, 10, 0.05, True),
+            ("tcgen05_i8_probe_sustained", 100_000, 5, 0.0, False)):
         clocks = clocks_cls(torch.cuda.current_device())
+        if pair:
+            fn = lambda: sq.sq_probe_mma_i8_pair(kblocks, pairs)  # noqa: E731
+            ops = 16777216.0 * kblocks * pairs
+            mma = "256x256x32 kind::i8 on CTA pairs (cta_group::2), operands in smem"
+        else:
+            fn = lambda: sq.sq_probe_mma_i8(kblocks, sms)  # noqa: E731
+            ops = 8388608.0 * kblocks * sms
+            mma = "128x256x32 kind::i8, one accumulator, operands in smem"
         with clocks:
-            ms = ev_time(lambda: sq.sq_probe_mma_i8(kblocks, sms), reps, 2, gap)
+            ms = ev_time(fn, reps, 2, gap)
         st = sq.sq_sync_status()
-        tops = 8388608.0 * kblocks * sms / (ms * 1e-3) / 1e12
+        tops = ops / (ms * 1e-3) / 1e12
         out[name] = {"tops": round(tops, 1), "ms": round(ms, 3), "ctas": sms,
-                     "kblocks_per_cta": kblocks, "idle_gap_s": gap,
-                     "mma": "128x256x32 kind::i8, one accumulator, operands in smem",
+                     "kblocks_per_cta": kblocks, "idle_gap_s": gap, "mma": mma,
                      "clocks": clocks.summary(), "status": st}
-    probe_tops = out["tcgen05_i8_probe"]["tops"]
+    probe_tops = max(out["tcgen05_i8_probe"]["tops"], out["tcgen05_i8_pair_probe"]["tops"])
+    probe_name = ("tcgen05_i8_pair_probe" if out["tcgen05_i8_pair_probe"]["tops"] >=
+                  out["tcgen05_i8_probe"]["tops"] else "tcgen05_i8_probe")
     n = 8192
     g = torch.Generator(device=dev).manual_seed(5)
     a = torch.randint(-127, 128, (n, n), dtype=torch.int8, device=dev, generator=g)
@@ -428,7 +441,7 @@ def measure_int8_peak(sq, torch, dev, clocks_cls):
         out["cublas_int8_gemm_8192"] = {"error": str(e)[:200]}
     del a, b
     out["peak_tops"] = round(max(probe_tops, cub), 1)
-    out["peak_from"] = "tcgen05_i8_probe" if probe_tops >= cub else "cublas_int8_gemm_8192"
+    out["peak_from"] = probe_name if probe_tops >= cub else "cublas_int8_gemm_8192"
     out["vendor_dense_tops"] = VENDOR_INT8_TOPS
     return out
 
@@ -440,6 +453,7 @@ def profile_only(args, sq, torch, layer, flush):
     torch.cuda.synchronize()
     for i in range(args.steps):
         if args.profile_call == "int8_probe":
+            sq.sq_probe_mma_i8_pair(2000, torch.cuda.get_device_properties(0).multi_processor_count // 2)
             sq.sq_probe_mma_i8(2000, torch.cuda.get_device_properties(0).multi_processor_count)
         else:
             layer.call(args.profile_call)

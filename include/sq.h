@@ -439,6 +439,17 @@ sq_status sq_selftest_bounded_wait(int64_t limit_ns, sq_stream stream);
  */
 sq_status sq_probe_mma_i8(int64_t kblocks, int grid, sq_stream stream);
 
+/*
+ * sq_probe_mma_i8_pair -- the same measurement for the instruction form the
+ * large-M GEMM uses: `pairs` clusters of two CTAs, the even CTA of each
+ * issuing kblocks x 4 tcgen05.mma.cta_group::2.kind::i8 steps of
+ * 256 x 256 x 32 that read A and B from both CTAs' shared memory into each
+ * CTA's TMEM.  Work: 16,777,216 * kblocks * pairs int8 ops (the same per SM
+ * as sq_probe_mma_i8).  kblocks in [1, 2^30], pairs in [1, 32767], else
+ * SQ_ERR_INVALID_ARG; the final wait is bounded.
+ */
+sq_status sq_probe_mma_i8_pair(int64_t kblocks, int pairs, sq_stream stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -208,6 +208,8 @@ def test_selftest_checks(lib):
     assert L.sq_probe_mma_i8(0, 148, None) == lib.SQ_ERR_INVALID_ARG
     assert L.sq_probe_mma_i8((1 << 30) + 1, 148, None) == lib.SQ_ERR_INVALID_ARG
     assert L.sq_probe_mma_i8(16, 0, None) == lib.SQ_ERR_INVALID_ARG
+    assert L.sq_probe_mma_i8_pair(0, 74, None) == lib.SQ_ERR_INVALID_ARG
+    assert L.sq_probe_mma_i8_pair(16, 0, None) == lib.SQ_ERR_INVALID_ARG
 
 
 def test_binding_fails_loudly_without_library(tmp_path, monkeypatch):

@@ -28,7 +28,7 @@ __all__ = [
     "sq_sync_status", "sq_selftest_bounded_wait", "SQError", "Workspace",
     "sq_calib_absmax_rms", "sq_rms_smooth_quant_act", "sq_fold_into_producer",
     "sq_alpha_sweep_workspace_bytes", "sq_alpha_sweep", "sq_bmm_w8a8",
-    "sq_weight_colmax", "sq_smooth_scales_peaks", "sq_probe_mma_i8",
+    "sq_weight_colmax", "sq_smooth_scales_peaks", "sq_probe_mma_i8", "sq_probe_mma_i8_pair",
 ]
 
 
@@ -247,3 +247,12 @@ def sq_probe_mma_i8(kblocks: int, grid: int, stream=None):
     per k-block).  Returns the op count; the caller times the launch."""
     check(lib.sq_probe_mma_i8(int(kblocks), int(grid), _stream(stream)), "sq_probe_mma_i8")
     return 8388608 * int(kblocks) * int(grid)
+
+
+def sq_probe_mma_i8_pair(kblocks: int, pairs: int, stream=None):
+    """Launch the CTA-pair INT8 tensor-core rate probe: `pairs` clusters of two
+    CTAs issuing kblocks x 4 tcgen05.mma.cta_group::2 steps of 256 x 256 x 32
+    (16,777,216 ops per k-block per pair).  Returns the op count."""
+    check(lib.sq_probe_mma_i8_pair(int(kblocks), int(pairs), _stream(stream)),
+          "sq_probe_mma_i8_pair")
+    return 16777216 * int(kblocks) * int(pairs)

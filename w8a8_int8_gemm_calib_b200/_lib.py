@@ -37,7 +37,7 @@ EXPORTS = [
     "sq_selftest_bounded_wait", "sq_gemm_w8a8_noalloc", "sq_gemm_w8a8_bias",
     "sq_calib_absmax_rms", "sq_rms_smooth_quant_act", "sq_fold_into_producer",
     "sq_alpha_sweep_workspace_bytes", "sq_alpha_sweep", "sq_bmm_w8a8",
-    "sq_weight_colmax", "sq_smooth_scales_peaks", "sq_probe_mma_i8",
+    "sq_weight_colmax", "sq_smooth_scales_peaks", "sq_probe_mma_i8", "sq_probe_mma_i8_pair",
 ]
 
 
@@ -79,13 +79,14 @@ def _load() -> ctypes.CDLL:
     L.sq_last_error.restype = ctypes.c_char_p
     L.sq_selftest_bounded_wait.argtypes = [i64, p]
     L.sq_probe_mma_i8.argtypes = [i64, i, p]
+    L.sq_probe_mma_i8_pair.argtypes = [i64, i, p]
     L.sq_gemm_w8a8_noalloc.argtypes = [p, p, i64, i64, i64, p, i, p, p, i, p, p]
     for fn in ("sq_calib_absmax", "sq_smooth_scales", "sq_fuse_weights_q8",
                "sq_ln_smooth_quant_act", "sq_gemm_w8a8", "sq_sync_status",
                "sq_selftest_bounded_wait", "sq_gemm_w8a8_noalloc", "sq_gemm_w8a8_bias",
                "sq_calib_absmax_rms", "sq_rms_smooth_quant_act", "sq_fold_into_producer",
                "sq_alpha_sweep", "sq_bmm_w8a8", "sq_weight_colmax", "sq_smooth_scales_peaks",
-               "sq_probe_mma_i8"):
+               "sq_probe_mma_i8", "sq_probe_mma_i8_pair"):
         getattr(L, fn).restype = st
     return L
 

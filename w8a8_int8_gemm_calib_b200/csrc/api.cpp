@@ -588,4 +588,14 @@ sq_status sq_probe_mma_i8(int64_t kblocks, int grid, sq_stream stream) {
   return e == cudaSuccess ? SQ_OK : cuda_fail(e, "sq_probe_mma_i8");
 }
 
+sq_status sq_probe_mma_i8_pair(int64_t kblocks, int pairs, sq_stream stream) {
+  g_last_error[0] = 0;
+  if (kblocks < 1 || kblocks > ((int64_t)1 << 30))
+    return fail(SQ_ERR_INVALID_ARG, "sq_probe_mma_i8_pair: kblocks must be in [1, 2^30]");
+  if (pairs < 1 || pairs > 32767)
+    return fail(SQ_ERR_INVALID_ARG, "sq_probe_mma_i8_pair: pairs must be in [1, 32767]");
+  cudaError_t e = launch_mma_pair_probe(kblocks, pairs, (cudaStream_t)stream);
+  return e == cudaSuccess ? SQ_OK : cuda_fail(e, "sq_probe_mma_i8_pair");
+}
+
 }  // extern "C"

@@ -149,5 +149,6 @@ cudaError_t launch_wait_selftest(int64_t limit_ns, cudaStream_t st);
 
 // ---------------------------------------------------------------- measurement
 cudaError_t launch_mma_probe(int64_t kblocks, int grid, cudaStream_t st);
+cudaError_t launch_mma_pair_probe(int64_t kblocks, int pairs, cudaStream_t st);
 
 }  // namespace sq
