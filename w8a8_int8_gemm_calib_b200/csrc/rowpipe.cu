@@ -340,6 +340,10 @@ __global__ void __launch_bounds__(kThreads, NB) rowpipe_kernel(const Pipe P) {
     const int q = tid / ST, j = tid % ST;
     const int v = j >> 5, lane = j & 31;
     const float kf = (float)K;
+    // a LayerNorm subtracts the mean; an RMSNorm has none (x - 0 = x, the
+    // shift is left out)
+    const bool shift = LN && !a.rms;
+    const bool has_beta = LN && a.b != nullptr;
     // x / K for a power-of-two K is x * (1/K) exactly (both are the correctly
     // rounded value of the same exact quotient): a multiply instead of a
     // division subroutine
@@ -399,16 +403,24 @@ __global__ void __launch_bounds__(kThreads, NB) rowpipe_kernel(const Pipe P) {
 
       float2 negmu2 = make_float2(0.0f, 0.0f), rstd2 = make_float2(0.0f, 0.0f);
       // y of one chunk in place: ((x - mu) * rstd) * g + b from x - mu, or
-      // x * m, or x
+      // x * m, or x.  Without a beta (RMSNorm, or a LayerNorm given none) the
+      // addition of +0 is left out: it could only turn a -0 into +0, which
+      // changes no peak and no code.
       auto ytrans = [&](int c, float2 (&x)[4]) {
         if constexpr (LN) {
-          float2 g8[4], b8[4];
+          float2 g8[4];
           lds8(pg, c, khalf, g8);
-          lds8(pb, c, khalf, b8);
+          if (has_beta) {
+            float2 b8[4];
+            lds8(pb, c, khalf, b8);
 #pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const float2 t = mul2(mul2(x[e], rstd2), g8[e]);
-            x[e] = make_float2(__fadd_rn(t.x, b8[e].x), __fadd_rn(t.y, b8[e].y));
+            for (int e = 0; e < 4; ++e) {
+              const float2 t = mul2(mul2(x[e], rstd2), g8[e]);
+              x[e] = make_float2(__fadd_rn(t.x, b8[e].x), __fadd_rn(t.y, b8[e].y));
+            }
+          } else {
+#pragma unroll
+            for (int e = 0; e < 4; ++e) x[e] = mul2(mul2(x[e], rstd2), g8[e]);
           }
         } else {
           if (has_mul) {
@@ -425,7 +437,7 @@ __global__ void __launch_bounds__(kThreads, NB) rowpipe_kernel(const Pipe P) {
       // recompute the level from the stored row.
       auto for_level = [&](int lvl, auto&& f) {
         auto lift = [&](int c, float2 (&x)[4]) {
-          if (LN && lvl >= 1) {
+          if (LN && lvl >= 1 && shift) {
 #pragma unroll
             for (int e = 0; e < 4; ++e) x[e] = add2(x[e], negmu2);
           }
@@ -500,7 +512,7 @@ __global__ void __launch_bounds__(kThreads, NB) rowpipe_kernel(const Pipe P) {
         for_level(0, [&](int m, int, float2 (&x)[4]) {
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
-            x[e] = add2(x[e], negmu2);  // now x - mu
+            if (shift) x[e] = add2(x[e], negmu2);  // now x - mu
             p[m % G] = __fmaf_rn(x[e].x, x[e].x, p[m % G]);
             p[m % G] = __fmaf_rn(x[e].y, x[e].y, p[m % G]);
           }
