@@ -63,7 +63,9 @@ typedef enum {
   SQ_ERR_UNSUPPORTED = 5, /* no sm_100 device, or a size this build cannot serve */
   SQ_ERR_CUDA = 6,        /* a CUDA runtime call failed */
   SQ_ERR_TIMEOUT = 7,     /* device side: a bounded wait ran out (from sq_sync_status) */
-  SQ_ERR_WORKSPACE = 8    /* workspace NULL or smaller than sq_gemm_workspace_bytes() */
+  SQ_ERR_WORKSPACE = 8,   /* workspace NULL or smaller than sq_gemm_workspace_bytes() */
+  SQ_ERR_BOUNDS = 9       /* device side, bounds-checked builds only: an index outside its
+                             tensor was caught and that access skipped (from sq_sync_status) */
 } sq_status;
 
 typedef enum { SQ_F32 = 0, SQ_BF16 = 1 } sq_dtype;
@@ -424,6 +426,27 @@ const char* sq_last_error(void);
  * sq_sync_status() then reports it.  Used by the fault-detection tests.
  */
 sq_status sq_selftest_bounded_wait(int64_t limit_ns, sq_stream stream);
+
+/*
+ * sq_debug_bounds_enabled -- 1 if this library was built with device-side
+ * bounds checks (`build.py --debug-bounds`, which writes
+ * libsq_b200_debug.so), else 0.  In such a build every kernel checks each
+ * global-memory offset it computes by hand (TMA copies are clipped by the
+ * hardware) against its tensor's extent before the access; an offset
+ * outside records SQ_ERR_BOUNDS in the status word and the access is
+ * skipped -- nothing traps.  The checks cost time; the outputs are
+ * otherwise those of the release build.
+ */
+int sq_debug_bounds_enabled(void);
+
+/*
+ * sq_selftest_bounds_check -- exercises that path without any out-of-range
+ * access: one thread checks an offset equal to its tensor's extent and
+ * touches no memory.  In a bounds-checked build the check records
+ * SQ_ERR_BOUNDS, which sq_sync_status() then reports; otherwise nothing is
+ * recorded.
+ */
+sq_status sq_selftest_bounds_check(sq_stream stream);
 
 /*
  * sq_probe_mma_i8 -- measurement support (no counterpart on the pages): the

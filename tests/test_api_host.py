@@ -34,7 +34,7 @@ def test_exports_every_declared_symbol(lib):
 
 
 def test_status_strings(lib):
-    for code in range(9):
+    for code in range(10):
         assert lib.status_string(code).startswith("SQ_")
     assert lib.status_string(42) == "SQ_ERR_UNKNOWN"
 
@@ -240,3 +240,22 @@ def test_gemm_decode_routing_on_the_host(lib):
     assert f(129, 512, 4096) == 0
     # 1000 channels: 8 tile counters (256 bytes) + 148 SMs x 2 slots x 1 token x 128 x 4
     assert f(1, 1000, 12288) == 256 + sms * 2 * 1 * 128 * 4
+
+
+def test_bounds_checked_build(lib):
+    """The release library reports no bounds checks; the bounds-checked
+    build (built here if it is missing) reports them and exports the same
+    entry points."""
+    import importlib.util
+
+    assert lib.lib.sq_debug_bounds_enabled() == 0
+    spec = importlib.util.spec_from_file_location(
+        "sq_build", os.path.join(ROOT, "w8a8_int8_gemm_calib_b200", "build.py"))
+    b = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(b)
+    path = b.LIB_DEBUG if os.path.exists(b.LIB_DEBUG) else b.build(debug_bounds=True)
+    dbg = ctypes.CDLL(path)
+    dbg.sq_debug_bounds_enabled.restype = ctypes.c_int
+    assert dbg.sq_debug_bounds_enabled() == 1
+    for n in declared_functions():
+        assert hasattr(dbg, n), f"{n} missing from the bounds-checked build"

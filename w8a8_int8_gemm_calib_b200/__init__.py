@@ -29,6 +29,7 @@ __all__ = [
     "sq_calib_absmax_rms", "sq_rms_smooth_quant_act", "sq_fold_into_producer",
     "sq_alpha_sweep_workspace_bytes", "sq_alpha_sweep", "sq_bmm_w8a8",
     "sq_weight_colmax", "sq_smooth_scales_peaks", "sq_probe_mma_i8", "sq_probe_mma_i8_pair",
+    "sq_debug_bounds_enabled", "sq_selftest_bounds_check",
 ]
 
 
@@ -256,3 +257,15 @@ def sq_probe_mma_i8_pair(kblocks: int, pairs: int, stream=None):
     check(lib.sq_probe_mma_i8_pair(int(kblocks), int(pairs), _stream(stream)),
           "sq_probe_mma_i8_pair")
     return 16777216 * int(kblocks) * int(pairs)
+
+
+def sq_debug_bounds_enabled() -> bool:
+    """True for the bounds-checked build (libsq_b200_debug.so)."""
+    return bool(lib.sq_debug_bounds_enabled())
+
+
+def sq_selftest_bounds_check(stream=None):
+    """Launch the bounds-check self-test (one thread checks an offset at
+    its tensor's end, touching no memory); sq_sync_status() then raises
+    SQ_ERR_BOUNDS in the bounds-checked build and nothing otherwise."""
+    check(lib.sq_selftest_bounds_check(_stream(stream)), "sq_selftest_bounds_check")

@@ -12,7 +12,9 @@ import ctypes
 import os
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_HERE, "libsq_b200.so")
+# SQ_B200_LIB may name another build of the same library, such as the
+# bounds-checked libsq_b200_debug.so (build.py --debug-bounds)
+LIB_PATH = os.environ.get("SQ_B200_LIB") or os.path.join(_HERE, "libsq_b200.so")
 
 SQ_OK = 0
 SQ_ERR_INVALID_ARG = 1
@@ -23,6 +25,7 @@ SQ_ERR_UNSUPPORTED = 5
 SQ_ERR_CUDA = 6
 SQ_ERR_TIMEOUT = 7
 SQ_ERR_WORKSPACE = 8
+SQ_ERR_BOUNDS = 9
 
 SQ_F32 = 0
 SQ_BF16 = 1
@@ -38,6 +41,7 @@ EXPORTS = [
     "sq_calib_absmax_rms", "sq_rms_smooth_quant_act", "sq_fold_into_producer",
     "sq_alpha_sweep_workspace_bytes", "sq_alpha_sweep", "sq_bmm_w8a8",
     "sq_weight_colmax", "sq_smooth_scales_peaks", "sq_probe_mma_i8", "sq_probe_mma_i8_pair",
+    "sq_debug_bounds_enabled", "sq_selftest_bounds_check",
 ]
 
 
@@ -80,13 +84,16 @@ def _load() -> ctypes.CDLL:
     L.sq_selftest_bounded_wait.argtypes = [i64, p]
     L.sq_probe_mma_i8.argtypes = [i64, i, p]
     L.sq_probe_mma_i8_pair.argtypes = [i64, i, p]
+    L.sq_debug_bounds_enabled.argtypes = []
+    L.sq_debug_bounds_enabled.restype = i
+    L.sq_selftest_bounds_check.argtypes = [p]
     L.sq_gemm_w8a8_noalloc.argtypes = [p, p, i64, i64, i64, p, i, p, p, i, p, p]
     for fn in ("sq_calib_absmax", "sq_smooth_scales", "sq_fuse_weights_q8",
                "sq_ln_smooth_quant_act", "sq_gemm_w8a8", "sq_sync_status",
                "sq_selftest_bounded_wait", "sq_gemm_w8a8_noalloc", "sq_gemm_w8a8_bias",
                "sq_calib_absmax_rms", "sq_rms_smooth_quant_act", "sq_fold_into_producer",
                "sq_alpha_sweep", "sq_bmm_w8a8", "sq_weight_colmax", "sq_smooth_scales_peaks",
-               "sq_probe_mma_i8", "sq_probe_mma_i8_pair"):
+               "sq_probe_mma_i8", "sq_probe_mma_i8_pair", "sq_selftest_bounds_check"):
         getattr(L, fn).restype = st
     return L
 

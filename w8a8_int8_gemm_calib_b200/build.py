@@ -1,7 +1,13 @@
 """Build the sm_100a library libsq_b200.so in-tree with nvcc.
 
 Usage: python w8a8_int8_gemm_calib_b200/build.py [--force] [--verbose] [--ptxas]
+                                                [--debug-bounds]
 (run it as a script: importing the package would load the existing library)
+
+--debug-bounds builds libsq_b200_debug.so instead: the same kernels with
+device-side bounds checks on every hand-computed global-memory offset
+(SQ_DEBUG_BOUNDS; a check that fails records SQ_ERR_BOUNDS and skips the
+access).  The package loads it when SQ_B200_LIB names its path.
 """
 from __future__ import annotations
 
@@ -14,6 +20,8 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 CSRC = os.path.join(HERE, "csrc")
 OBJ = os.path.join(HERE, "_build")
 LIB = os.path.join(HERE, "libsq_b200.so")
+OBJ_DEBUG = os.path.join(HERE, "_build_debug")
+LIB_DEBUG = os.path.join(HERE, "libsq_b200_debug.so")
 INCLUDE = os.path.join(os.path.dirname(HERE), "include")
 
 SOURCES = ["api.cpp", "status.cu", "rowops.cu", "rowpipe.cu", "gemm.cu", "probe.cu"]
@@ -39,18 +47,21 @@ def _stale(target: str, deps: list[str]) -> bool:
     return any(os.path.getmtime(d) > t for d in deps)
 
 
-def build(force: bool = False, verbose: bool = False, ptxas_verbose: bool = False) -> str:
-    os.makedirs(OBJ, exist_ok=True)
+def build(force: bool = False, verbose: bool = False, ptxas_verbose: bool = False,
+          debug_bounds: bool = False) -> str:
+    obj_dir, lib = (OBJ_DEBUG, LIB_DEBUG) if debug_bounds else (OBJ, LIB)
+    defines = ["-DSQ_DEBUG_BOUNDS"] if debug_bounds else []
+    os.makedirs(obj_dir, exist_ok=True)
     hdrs = [os.path.join(CSRC, h) for h in HEADERS] + [os.path.join(INCLUDE, "sq.h"),
                                                         os.path.abspath(__file__)]
     jobs = []
     objs = []
     for src in SOURCES:
         s = os.path.join(CSRC, src)
-        o = os.path.join(OBJ, src + ".o")
+        o = os.path.join(obj_dir, src + ".o")
         objs.append(o)
         if force or _stale(o, [s] + hdrs):
-            cmd = [nvcc(), *ARCH, *NVCC_FLAGS, *EXTRA_FLAGS.get(src, []), "-c", s, "-o", o]
+            cmd = [nvcc(), *ARCH, *NVCC_FLAGS, *defines, *EXTRA_FLAGS.get(src, []), "-c", s, "-o", o]
             if ptxas_verbose and src.endswith(".cu"):
                 cmd += ["-Xptxas", "-v"]
             jobs.append(cmd)
@@ -67,18 +78,17 @@ def build(force: bool = False, verbose: bool = False, ptxas_verbose: bool = Fals
                 sys.stderr.write(r.stdout + r.stderr)
             if r.returncode != 0:
                 raise RuntimeError(f"nvcc failed: {' '.join(cmd)}")
-    if force or jobs or _stale(LIB, objs):
-        tmp = LIB + f".tmp{os.getpid()}"
+    if force or jobs or _stale(lib, objs):
+        tmp = lib + f".tmp{os.getpid()}"
         cmd = [nvcc(), *ARCH, "-shared", "-o", tmp, *objs, "-lcudart_static", "-lrt",
                "-lpthread", "-ldl"]
         if verbose:
             print(" ".join(cmd), flush=True)
         subprocess.check_call(cmd)
-        os.replace(tmp, LIB)
-    return LIB
+        os.replace(tmp, lib)
+    return lib
 
 
 if __name__ == "__main__":
-    build(force="--force" in sys.argv, verbose="--verbose" in sys.argv,
-          ptxas_verbose="--ptxas" in sys.argv)
-    print(LIB)
+    print(build(force="--force" in sys.argv, verbose="--verbose" in sys.argv,
+                ptxas_verbose="--ptxas" in sys.argv, debug_bounds="--debug-bounds" in sys.argv))

@@ -564,6 +564,7 @@ const char* sq_status_string(sq_status s) {
     case SQ_ERR_CUDA: return "SQ_ERR_CUDA";
     case SQ_ERR_TIMEOUT: return "SQ_ERR_TIMEOUT";
     case SQ_ERR_WORKSPACE: return "SQ_ERR_WORKSPACE";
+    case SQ_ERR_BOUNDS: return "SQ_ERR_BOUNDS";
   }
   return "SQ_ERR_UNKNOWN";
 }
@@ -576,6 +577,20 @@ sq_status sq_selftest_bounded_wait(int64_t limit_ns, sq_stream stream) {
     return fail(SQ_ERR_INVALID_ARG, "sq_selftest_bounded_wait: limit_ns must be in [1, 1e9]");
   cudaError_t e = launch_wait_selftest(limit_ns, (cudaStream_t)stream);
   return e == cudaSuccess ? SQ_OK : cuda_fail(e, "sq_selftest_bounded_wait");
+}
+
+int sq_debug_bounds_enabled(void) {
+#ifdef SQ_DEBUG_BOUNDS
+  return 1;
+#else
+  return 0;
+#endif
+}
+
+sq_status sq_selftest_bounds_check(sq_stream stream) {
+  g_last_error[0] = 0;
+  cudaError_t e = launch_bounds_selftest((cudaStream_t)stream);
+  return e == cudaSuccess ? SQ_OK : cuda_fail(e, "sq_selftest_bounds_check");
 }
 
 sq_status sq_probe_mma_i8(int64_t kblocks, int grid, sq_stream stream) {

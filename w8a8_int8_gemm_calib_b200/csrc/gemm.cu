@@ -83,6 +83,7 @@ struct Params {
   int group;            // tile raster: row tiles per band (each band sweeps every column)
   int w_per_tensor;     // batched: one weight step per batch (w_scale[b])
   int tma_store;  // outputs leave through shared memory and TMA stores
+  int64_t y_elems;  // elements of y (and acc): batch * M * N
   const float* act_scale;
   int per_token;
   const float* w_scale;
@@ -161,6 +162,7 @@ __device__ __forceinline__ void store_chunk(const Params& p, size_t yrow, int co
                                             const uint32_t (&r)[32], const float (&yv)[32]) {
   const bool full = col0 + 32 <= p.N;
   const size_t base = yrow * (size_t)p.N + (size_t)col0;
+  if (!in_bounds((int64_t)base, min(32, p.N - col0), p.y_elems, p.status)) return;
   if (BF16) {
     __nv_bfloat16* y = reinterpret_cast<__nv_bfloat16*>(p.y) + base;
     if (full && (p.N % 8) == 0) {
@@ -429,7 +431,7 @@ gemm_w8a8_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
         if constexpr (ERR) {
           // (y - y_ref)^2 and y_ref^2 in fp64, y the fp32 output the store
           // path would write; columns past N hold y = 0 and read ref = 0
-          if (row_ok) {
+          if (row_ok && in_bounds((int64_t)(yrow * p.N), p.N, p.y_elems, p.status)) {
             float rv[32];
             load_cols32(p.err_ref + yrow * (size_t)p.N, col0, p.N, rv);
 #pragma unroll
@@ -459,7 +461,8 @@ gemm_w8a8_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
             wv[i + 1] = __float_as_uint(y1);
           }
         }
-        if (p.acc && row_ok && col0 < p.N) {
+        if (p.acc && row_ok && col0 < p.N &&
+            in_bounds((int64_t)(yrow * p.N + col0), min(32, p.N - col0), p.y_elems, p.status)) {
           int32_t* a = p.acc + yrow * p.N + col0;
 #pragma unroll
           for (int i = 0; i < 32; ++i)
@@ -604,6 +607,7 @@ __device__ __forceinline__ void small_store(const SmallParams& p, int n, int t0,
       float y = dequant((uint32_t)v[i], as, ws);
       if (p.bias) y = __fadd_rn(y, bn);
       const size_t o = (size_t)t * (size_t)p.N + (size_t)n;
+      if (!in_bounds((int64_t)o, 1, (int64_t)p.M * p.N, p.status)) continue;
       if (BF16) reinterpret_cast<__nv_bfloat16*>(p.y)[o] = __float2bfloat16_rn(y);
       else reinterpret_cast<float*>(p.y)[o] = y;
       if (p.acc) p.acc[o] = v[i];
@@ -752,6 +756,7 @@ gemm_w8a8_smallm_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_co
     // ------------------------------------------------------------ epilogue
     const int quarter = warp & 3;
     const int rloc = quarter * 32 + lane;  // output channel within the tile
+    const int64_t slot_elems = (int64_t)p.grid * 2 * p.M * SM_BM;  // the partial-tile slots
     uint32_t abuf = 0, aphase = 0;
     for (int64_t u = ub; u < ue;) {
       const int tile = (int)(u / p.nk);
@@ -778,7 +783,9 @@ gemm_w8a8_smallm_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_co
         } else {
 #pragma unroll
           for (int i = 0; i < C::CH; ++i)
-            if (c0 + i < p.M) slot[(int64_t)(c0 + i) * SM_BM + rloc] = (int32_t)r[i];
+            if (c0 + i < p.M &&
+                in_bounds((slot - p.slots) + (int64_t)(c0 + i) * SM_BM + rloc, 1, slot_elems, p.status))
+              slot[(int64_t)(c0 + i) * SM_BM + rloc] = (int32_t)r[i];
         }
       }
       tc::tc_fence_before();
@@ -793,7 +800,9 @@ gemm_w8a8_smallm_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_co
         __threadfence();
         epi_bar();
         if (threadIdx.x == 64) {
-          const unsigned prev = atomicAdd(p.counters + tile, 1u);
+          const unsigned prev = in_bounds(tile, 1, p.n_tiles, p.status)
+                                    ? atomicAdd(p.counters + tile, 1u)
+                                    : 0u;
           *last_flag = prev == (unsigned)(gl - gf);
         }
         epi_bar();
@@ -811,7 +820,9 @@ gemm_w8a8_smallm_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_co
               const int32_t* sl = p.slots + (g * 2 + wg) * (int64_t)p.M * SM_BM;
 #pragma unroll
               for (int i = 0; i < C::CH; ++i)
-                if (c0 + i < p.M) v[i] += __ldcg(sl + (int64_t)(c0 + i) * SM_BM + rloc);
+                if (c0 + i < p.M &&
+                    in_bounds((sl - p.slots) + (int64_t)(c0 + i) * SM_BM + rloc, 1, slot_elems, p.status))
+                  v[i] += __ldcg(sl + (int64_t)(c0 + i) * SM_BM + rloc);
             }
             small_store<BF16, C::CH>(p, n, c0, v);
           }
@@ -1201,6 +1212,7 @@ bool setup_large(const GemmArgs& a, unsigned int* sw, LargeSetup* L, bool allow_
   p.bias = a.bias;
   p.y = a.y;
   p.acc = a.acc_out;
+  p.y_elems = a.M * a.N;
   p.status = sw;
   L->grid = L->pair ? sm_count() / 2 : sm_count();
   if (L->grid > p.num_tiles) L->grid = p.num_tiles;
@@ -1306,6 +1318,7 @@ sq_status launch_bmm(const BmmArgs& a, cudaStream_t st) {
   p.bias = nullptr;
   p.y = a.y;
   p.acc = a.acc_out;
+  p.y_elems = a.batch * a.M * a.N;
   p.status = sw;
   CUtensorMap ty;
   memset(&ty, 0, sizeof ty);

@@ -48,7 +48,7 @@ __device__ __forceinline__ float warp_max(float p) {
 template <typename T>
 __global__ void __launch_bounds__(kColWarps * 32)
 colmax_kernel(const T* __restrict__ x, int64_t T_, int64_t K, int64_t rows_per_slab,
-              unsigned int* __restrict__ out) {
+              unsigned int* __restrict__ out, unsigned int* status) {
   __shared__ float part[kColWarps][256];
   pdl_launch_dependents();
   pdl_wait();
@@ -68,7 +68,11 @@ colmax_kernel(const T* __restrict__ x, int64_t T_, int64_t K, int64_t rows_per_s
     for (; r + (U - 1) * kColWarps < r1; r += U * kColWarps) {
       Raw8<T> raw[U];
 #pragma unroll
-      for (int u = 0; u < U; ++u) load_raw(base + (r + u * kColWarps) * K, raw[u]);
+      for (int u = 0; u < U; ++u) {
+        raw[u] = Raw8<T>{};
+        if (in_bounds(chunk * 8 + (r + u * kColWarps) * K, 8, T_ * K, status))
+          load_raw(base + (r + u * kColWarps) * K, raw[u]);
+      }
 #pragma unroll
       for (int u = 0; u < U; ++u) {
         float v[8];
@@ -78,8 +82,8 @@ colmax_kernel(const T* __restrict__ x, int64_t T_, int64_t K, int64_t rows_per_s
       }
     }
     for (; r < r1; r += kColWarps) {
-      Raw8<T> raw;
-      load_raw(base + r * K, raw);
+      Raw8<T> raw{};
+      if (in_bounds(chunk * 8 + r * K, 8, T_ * K, status)) load_raw(base + r * K, raw);
       float v[8];
       unpack(raw, v);
 #pragma unroll
@@ -95,7 +99,7 @@ colmax_kernel(const T* __restrict__ x, int64_t T_, int64_t K, int64_t rows_per_s
 #pragma unroll
   for (int w = 1; w < kColWarps; ++w) v = fmaxf(v, part[w][col]);
   const int64_t k = (int64_t)blockIdx.x * 256 + col;
-  if (k < K) atomicMax(out + k, __float_as_uint(v));
+  if (k < K && in_bounds(k, 1, K, status)) atomicMax(out + k, __float_as_uint(v));
 }
 
 // Slabs of rows per column strip so that the grid is one wave of resident
@@ -144,9 +148,9 @@ cudaError_t launch_colmax(const void* x, sq_dtype xt, int64_t T, int64_t K, floa
   dim3 grid((unsigned)strips, (unsigned)((T + rows - 1) / rows));
   if (xt == SQ_BF16)
     return launch_pdl(colmax_kernel<uint16_t>, grid, dim3(kColWarps * 32), 0, st,
-                      (const uint16_t*)x, T, K, rows, (unsigned int*)out);
+                      (const uint16_t*)x, T, K, rows, (unsigned int*)out, status_word());
   return launch_pdl(colmax_kernel<float>, grid, dim3(kColWarps * 32), 0, st, (const float*)x, T,
-                    K, rows, (unsigned int*)out);
+                    K, rows, (unsigned int*)out, status_word());
 }
 
 // ============================================================ strip quantizer
@@ -162,7 +166,7 @@ template <typename T, bool PEAK>
 __global__ void __launch_bounds__(kColWarps * 32)
 strip_quant_kernel(const T* __restrict__ x, int64_t T_, int64_t K, int64_t rows_per_slab,
                    const float* __restrict__ mul, const float* scale, int8_t* __restrict__ q,
-                   unsigned long long* n_clipped, unsigned int* peak) {
+                   unsigned long long* n_clipped, unsigned int* peak, unsigned int* status) {
   pdl_launch_dependents();
   pdl_wait();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -193,7 +197,7 @@ strip_quant_kernel(const T* __restrict__ x, int64_t T_, int64_t K, int64_t rows_
       uint32_t b[8];
 #pragma unroll
       for (int e = 0; e < 8; ++e) b[e] = qbits(v[e], inv, count, clipped);
-      store_codes(q + r * K + chunk * 8, b);
+      if (in_bounds(r * K + chunk * 8, 8, T_ * K, status)) store_codes(q + r * K + chunk * 8, b);
     }
   };
   if (live) {
@@ -203,13 +207,17 @@ strip_quant_kernel(const T* __restrict__ x, int64_t T_, int64_t K, int64_t rows_
     for (; r + (U - 1) * kColWarps < r1; r += U * kColWarps) {
       Raw8<T> raw[U];
 #pragma unroll
-      for (int u = 0; u < U; ++u) load_raw(base + (r + u * kColWarps) * K, raw[u]);
+      for (int u = 0; u < U; ++u) {
+        raw[u] = Raw8<T>{};
+        if (in_bounds(chunk * 8 + (r + u * kColWarps) * K, 8, T_ * K, status))
+          load_raw(base + (r + u * kColWarps) * K, raw[u]);
+      }
 #pragma unroll
       for (int u = 0; u < U; ++u) work(raw[u], r + u * kColWarps);
     }
     for (; r < r1; r += kColWarps) {
-      Raw8<T> raw;
-      load_raw(base + r * K, raw);
+      Raw8<T> raw{};
+      if (in_bounds(chunk * 8 + r * K, 8, T_ * K, status)) load_raw(base + r * K, raw);
       work(raw, r);
     }
   }
@@ -233,7 +241,7 @@ cudaError_t launch_strip_quant_t(const RowArgs& a, cudaStream_t st) {
   dim3 grid((unsigned)strips, (unsigned)((a.T + rows - 1) / rows));
   return launch_pdl(strip_quant_kernel<T, PEAK>, grid, dim3(kColWarps * 32), 0, st,
                     (const T*)a.x, a.T, a.K, rows, a.mul, (const float*)a.scale, a.q,
-                    a.n_clipped, reinterpret_cast<unsigned int*>(a.peak));
+                    a.n_clipped, reinterpret_cast<unsigned int*>(a.peak), status_word());
 }
 
 cudaError_t launch_strip_quant(const RowArgs& a, sq_dtype xt, RowMode mode, cudaStream_t st) {
@@ -274,7 +282,9 @@ __device__ __forceinline__ void slice_bar(int slice) {
 // Calls f(i, c, v[8]) for every chunk the thread owns, in increasing c.
 template <int MAXC, typename T, typename F>
 __device__ __forceinline__ void for_chunks(const Raw8<T> (&raw)[MAXC > 0 ? MAXC : 1],
-                                           const T* xr, int j, int64_t nchunk, F&& f) {
+                                           const T* xr, int j, int64_t nchunk, F&& f,
+                                           int64_t row_off = 0, int64_t size = 0,
+                                           unsigned int* status = nullptr) {
   if constexpr (MAXC > 0) {
 #pragma unroll
     for (int i = 0; i < MAXC; ++i) {
@@ -288,8 +298,8 @@ __device__ __forceinline__ void for_chunks(const Raw8<T> (&raw)[MAXC > 0 ? MAXC 
   } else {
     int i = 0;
     for (int64_t c = j; c < nchunk; c += kSliceThreads, ++i) {
-      Raw8<T> r;
-      load_raw_cached(xr + c * 8, r);
+      Raw8<T> r{};
+      if (in_bounds(row_off + c * 8, 8, size, status)) load_raw_cached(xr + c * 8, r);
       float v[8];
       unpack(r, v);
       f(i, c, v);
@@ -397,20 +407,25 @@ row_kernel(RowArgs a) {
   const int64_t stride = (int64_t)gridDim.x * kSlices;
   int64_t row = (int64_t)blockIdx.x * kSlices + slice;
   Raw8<T> cur[CM];
-  if (row < a.T) load_row<MAXC>(cur, x + row * K, j, nchunk);
+  if (row < a.T && in_bounds(row * K, K, a.T * K, a.status))
+    load_row<MAXC>(cur, x + row * K, j, nchunk);
   while (row < a.T) {
     const int64_t nrow = row + stride;
     Raw8<T> nxt[PF ? CM : 1];
     if constexpr (PF) {
-      if (nrow < a.T) load_row<MAXC>(nxt, x + nrow * K, j, nchunk);
+      if (nrow < a.T && in_bounds(nrow * K, K, a.T * K, a.status))
+        load_row<MAXC>(nxt, x + nrow * K, j, nchunk);
     }
     const T* xr = x + row * K;
+    // the thread's chunks of this row (re-read from global memory when they
+    // are not held in registers, the row's extent checked in debug builds)
+    auto chunks = [&](auto&& f) { for_chunks<MAXC>(cur, xr, j, nchunk, f, row * K, a.T * K, a.status); };
 
     float mu = 0.0f, rstd = 0.0f;
     if constexpr (LN) {
       if (!a.rms) {  // RMSNorm: no mean (mu = 0, beta NULL)
         float p = 0.0f;
-        for_chunks<MAXC>(cur, xr, j, nchunk, [&](int, int64_t, const float (&v)[8]) {
+        chunks([&](int, int64_t, const float (&v)[8]) {
 #pragma unroll
           for (int e = 0; e < 8; ++e) p = __fadd_rn(p, v[e]);
         });
@@ -422,7 +437,7 @@ row_kernel(RowArgs a) {
         mu = __fdiv_rn(s0, kf);
       }
       float q = 0.0f;
-      for_chunks<MAXC>(cur, xr, j, nchunk, [&](int, int64_t, const float (&v)[8]) {
+      chunks([&](int, int64_t, const float (&v)[8]) {
 #pragma unroll
         for (int e = 0; e < 8; ++e) {
           const float d = __fsub_rn(v[e], mu);
@@ -447,7 +462,7 @@ row_kernel(RowArgs a) {
     };
 
     if constexpr (MODE == ROW_COLMAX) {
-      for_chunks<MAXC>(cur, xr, j, nchunk, [&](int i, int64_t c, const float (&v)[8]) {
+      chunks([&](int i, int64_t c, const float (&v)[8]) {
         float g8[8], b8[8];
         params(i, c, g8, b8);
 #pragma unroll
@@ -457,12 +472,13 @@ row_kernel(RowArgs a) {
             cmax[i * 8 + e] = fmaxf(cmax[i * 8 + e], y);
           } else {
             if (use_smem) atomicMax(&colmax_s[c * 8 + e], peak_bits(y));
-            else atomicMax((unsigned int*)a.colmax + c * 8 + e, peak_bits(y));
+            else if (in_bounds(c * 8 + e, 1, K, a.status))
+              atomicMax((unsigned int*)a.colmax + c * 8 + e, peak_bits(y));
           }
         }
       });
     } else if constexpr (MODE == ROW_PEAK) {
-      for_chunks<MAXC>(cur, xr, j, nchunk, [&](int i, int64_t c, const float (&v)[8]) {
+      chunks([&](int i, int64_t c, const float (&v)[8]) {
         float g8[8], b8[8];
         params(i, c, g8, b8);
 #pragma unroll
@@ -472,7 +488,7 @@ row_kernel(RowArgs a) {
       float inv = static_inv;
       if constexpr (MODE == ROW_DYNAMIC) {
         float m = 0.0f;
-        for_chunks<MAXC>(cur, xr, j, nchunk, [&](int i, int64_t c, const float (&v)[8]) {
+        chunks([&](int i, int64_t c, const float (&v)[8]) {
           float g8[8], b8[8];
           params(i, c, g8, b8);
 #pragma unroll
@@ -485,10 +501,10 @@ row_kernel(RowArgs a) {
                   fmaxf(red[slice][parity][2][2], red[slice][parity][2][3]));
         const float delta = __fdiv_rn(fmaxf(m, 1e-7f), 127.0f);
         inv = __fdiv_rn(1.0f, delta);
-        if (j == 0) a.scale[row] = delta;
+        if (j == 0 && in_bounds(row, 1, a.T, a.status)) a.scale[row] = delta;
       }
       int8_t* qr = a.q + row * K;
-      for_chunks<MAXC>(cur, xr, j, nchunk, [&](int i, int64_t c, const float (&v)[8]) {
+      chunks([&](int i, int64_t c, const float (&v)[8]) {
         float g8[8], b8[8];
         params(i, c, g8, b8);
         int q[8];
@@ -497,7 +513,8 @@ row_kernel(RowArgs a) {
         uint2 pk;
         pk.x = pack4(q[0], q[1], q[2], q[3]);
         pk.y = pack4(q[4], q[5], q[6], q[7]);
-        *reinterpret_cast<uint2*>(qr + c * 8) = pk;
+        if (in_bounds(row * K + c * 8, 8, a.T * K, a.status))
+          *reinterpret_cast<uint2*>(qr + c * 8) = pk;
       });
     }
     parity ^= 1;
@@ -507,7 +524,8 @@ row_kernel(RowArgs a) {
 #pragma unroll
         for (int i = 0; i < CM; ++i) cur[i] = nxt[i];
       } else {
-        if (row < a.T) load_row<MAXC>(cur, x + row * K, j, nchunk);
+        if (row < a.T && in_bounds(row * K, K, a.T * K, a.status))
+          load_row<MAXC>(cur, x + row * K, j, nchunk);
       }
     }
   }
@@ -528,7 +546,7 @@ row_kernel(RowArgs a) {
     if (use_smem) {
       __syncthreads();
       for (int64_t k = threadIdx.x; k < K; k += blockDim.x)
-        atomicMax((unsigned int*)a.colmax + k, colmax_s[k]);
+        if (in_bounds(k, 1, K, a.status)) atomicMax((unsigned int*)a.colmax + k, colmax_s[k]);
     }
   }
   if constexpr (MODE == ROW_PEAK) {
@@ -611,7 +629,9 @@ static cudaError_t dispatch_mode(const RowArgs& a, RowMode mode, cudaStream_t st
   return cudaErrorInvalidValue;
 }
 
-cudaError_t launch_row(const RowArgs& a, sq_dtype xt, RowMode mode, cudaStream_t st) {
+cudaError_t launch_row(const RowArgs& args, sq_dtype xt, RowMode mode, cudaStream_t st) {
+  RowArgs a = args;
+  a.status = status_word();
   // no LayerNorm and one step for the whole call: a plain element stream
   const bool folds = a.fold_g_out || a.fold_b_out;
   if (!a.g && !folds && (mode == ROW_STATIC || mode == ROW_PEAK))

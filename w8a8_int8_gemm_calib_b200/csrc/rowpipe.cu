@@ -202,7 +202,10 @@ __device__ __forceinline__ void produce_rows(const Pipe& P, uint32_t ring_u32, u
     tc::mbar_arrive_expect_tx(full_bar(s), RB);
     for (uint32_t off = 0; off < RB; off += kCopyPiece) {
       const uint32_t n = RB - off < kCopyPiece ? RB - off : kCopyPiece;
-      tc::bulk_load(ring_u32 + (uint32_t)s * RB + off, src + i * (int64_t)RB + off, n, full_bar(s));
+      // a copy outside x is skipped: its row's barrier then never completes
+      // and the consumers give up at their bounded wait
+      if (in_bounds((r0 + i) * (int64_t)RB + off, n, P.a.T * (int64_t)RB, P.status))
+        tc::bulk_load(ring_u32 + (uint32_t)s * RB + off, src + i * (int64_t)RB + off, n, full_bar(s));
     }
     issued |= 1u << s;
     issued_par = (issued_par & ~(1u << s)) | ((uint32_t)(u & 1) << s);
@@ -552,7 +555,7 @@ __global__ void __launch_bounds__(kThreads, NB) rowpipe_kernel(const Pipe P) {
             b[2 * e] = qbits(x[e].x, static_inv, count, clipped);
             b[2 * e + 1] = qbits(x[e].y, static_inv, count, clipped);
           }
-          store_codes(qr + c * 8, b);
+          if (in_bounds(row * K + c * 8, 8, a.T * K, P.status)) store_codes(qr + c * 8, b);
         });
       } else {
         // peak magnitude with NaN propagated: a finite result means every
@@ -592,7 +595,7 @@ __global__ void __launch_bounds__(kThreads, NB) rowpipe_kernel(const Pipe P) {
         }
         const float delta = __fdiv_rn(fmaxf(mx, 1e-7f), 127.0f);
         const float inv = __fdiv_rn(1.0f, delta);
-        if (j == 0) a.scale[row] = delta;
+        if (j == 0 && in_bounds(row, 1, a.T, P.status)) a.scale[row] = delta;
         int8_t* qr = a.q + row * K;
         if (clean) {
           // |y * inv| <= 127*(1 + 2^-23) < 127.5 for every element of a
@@ -606,7 +609,7 @@ __global__ void __launch_bounds__(kThreads, NB) rowpipe_kernel(const Pipe P) {
               b[2 * e] = __float_as_uint(__fadd_rn(r.x, kRoundMagic));
               b[2 * e + 1] = __float_as_uint(__fadd_rn(r.y, kRoundMagic));
             }
-            store_codes(qr + c * 8, b);
+            if (in_bounds(row * K + c * 8, 8, a.T * K, P.status)) store_codes(qr + c * 8, b);
           });
         } else {
           for_level(2, [&](int, int c, float2 (&y)[4]) {
@@ -616,7 +619,7 @@ __global__ void __launch_bounds__(kThreads, NB) rowpipe_kernel(const Pipe P) {
               b[2 * e] = qbits(y[e].x, inv, count, clipped);
               b[2 * e + 1] = qbits(y[e].y, inv, count, clipped);
             }
-            store_codes(qr + c * 8, b);
+            if (in_bounds(row * K + c * 8, 8, a.T * K, P.status)) store_codes(qr + c * 8, b);
           });
         }
       }
@@ -646,7 +649,8 @@ __global__ void __launch_bounds__(kThreads, NB) rowpipe_kernel(const Pipe P) {
   if constexpr (MODE == ROW_COLMAX) {
     if (tid < kConsumers && R > 0)
       for (int64_t k = tid; k < K; k += kConsumers)
-        atomicMax(reinterpret_cast<unsigned int*>(a.colmax) + k, colmax_s[k]);
+        if (in_bounds(k, 1, K, P.status))
+          atomicMax(reinterpret_cast<unsigned int*>(a.colmax) + k, colmax_s[k]);
   }
   if (P.count && tid < kConsumers) {
 #pragma unroll

@@ -8,9 +8,27 @@ namespace sq {
 
 // Device status codes written to the status word (values of sq_status).
 constexpr unsigned kStatusTimeout = 7u;
+constexpr unsigned kStatusBounds = 9u;
 
 __device__ __forceinline__ void set_status(unsigned int* status, unsigned code) {
   if (status) atomicCAS(status, 0u, code);
+}
+
+// Bounds check of a hand-computed global-memory offset: the access of
+// elements [off, off + n) of a tensor of `size` elements may go ahead.  In
+// a build with SQ_DEBUG_BOUNDS an offset outside records SQ_ERR_BOUNDS and
+// the caller skips the access; otherwise the check is compiled away.
+__device__ __forceinline__ bool in_bounds(int64_t off, int64_t n, int64_t size,
+                                          unsigned int* status) {
+#ifdef SQ_DEBUG_BOUNDS
+  if (off < 0 || n < 0 || off + n > size) {
+    set_status(status, kStatusBounds);
+    return false;
+  }
+#else
+  (void)off; (void)n; (void)size; (void)status;
+#endif
+  return true;
 }
 
 // bf16 -> fp32 is exact: the bf16 pattern is the upper half of the fp32 one.

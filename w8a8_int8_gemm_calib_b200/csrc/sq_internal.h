@@ -57,6 +57,7 @@ struct RowArgs {
   const float* fold_b;
   float* fold_g_out;
   float* fold_b_out;
+  unsigned int* status;  // the device status word (set by launch_row)
 };
 
 cudaError_t launch_row(const RowArgs& a, sq_dtype xt, RowMode mode,
@@ -146,6 +147,7 @@ sq_status launch_gemm_noalloc(GemmArgs a, cudaStream_t st);
 
 // ---------------------------------------------------------------- self test
 cudaError_t launch_wait_selftest(int64_t limit_ns, cudaStream_t st);
+cudaError_t launch_bounds_selftest(cudaStream_t st);
 
 // ---------------------------------------------------------------- measurement
 cudaError_t launch_mma_probe(int64_t kblocks, int grid, cudaStream_t st);

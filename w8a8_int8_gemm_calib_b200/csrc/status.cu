@@ -74,6 +74,19 @@ __global__ void wait_selftest_kernel(int64_t limit_ns, unsigned int* status) {
   asm volatile("mbarrier.inval.shared::cta.b64 [%0];" ::"r"(addr) : "memory");
 }
 
+// One thread checks an offset equal to its (4-element) tensor's extent and
+// touches no memory: a bounds-checked build records SQ_ERR_BOUNDS.
+__global__ void bounds_selftest_kernel(unsigned int* status) {
+  if (threadIdx.x == 0) (void)in_bounds(4, 1, 4, status);
+}
+
+cudaError_t launch_bounds_selftest(cudaStream_t st) {
+  unsigned int* sw = status_word();
+  if (!sw) return cudaErrorInvalidDevice;
+  bounds_selftest_kernel<<<1, 32, 0, st>>>(sw);
+  return cudaGetLastError();
+}
+
 cudaError_t launch_wait_selftest(int64_t limit_ns, cudaStream_t st) {
   unsigned int* sw = status_word();
   if (!sw) return cudaErrorInvalidDevice;
