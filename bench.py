@@ -882,8 +882,15 @@ def run_gemm_bias(sq, torch, layer, lin, flush, int8_peak, reps=20):
 
 
 def run_e2e(sq, torch, layer, lin, d, dev, steps, world, barrier):
-    """Same step through the public API, inputs copied from pinned host memory
-    every step and the output read back."""
+    """The same step through the public API, every step uploading all of its
+    inputs from pinned host memory and reading its whole output back, run
+    the way a serving loop would: two sets of device buffers, the uploads on
+    one copy stream and the read-backs on another, so that step i's output
+    travels to the host while step i+1's inputs travel to the device (PCIe
+    moves both directions at once) and the kernels run in between.  Events
+    order each buffer's reuse: an upload waits until the step that last used
+    its buffers has computed, a step waits for its upload and for the
+    read-back of the output it will overwrite."""
     def pinned(a):
         if a is None:
             return None
@@ -893,35 +900,55 @@ def run_e2e(sq, torch, layer, lin, d, dev, steps, world, barrier):
 
     hx_cal, hx, hw = pinned(d["x_cal"]), pinned(d["x"]), pinned(d["w"])
     hg, hb = pinned(d["gamma"]), pinned(d["beta"])
-    hy = torch.empty(layer.y.shape, dtype=layer.y.dtype).pin_memory()
+    layers = [layer, Layer(sq, torch, lin, d, dev)]
+    hy = [torch.empty(layer.y.shape, dtype=layer.y.dtype).pin_memory() for _ in layers]
     h2d = sum(t.numel() * t.element_size() for t in (hx_cal, hx, hw, hg, hb) if t is not None)
-    d2h = hy.numel() * hy.element_size()
+    d2h = hy[0].numel() * hy[0].element_size()
+    s_comp = torch.cuda.current_stream()
+    s_up, s_down = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+    computed = [torch.cuda.Event() for _ in layers]
+    uploaded = [torch.cuda.Event() for _ in layers]
+    read_back = [torch.cuda.Event() for _ in layers]
 
-    def one():
-        layer.x_cal.copy_(hx_cal, non_blocking=True)
-        layer.x.copy_(hx, non_blocking=True)
-        layer.w.copy_(hw, non_blocking=True)
-        if hg is not None:
-            layer.gamma.copy_(hg, non_blocking=True)
-            layer.beta.copy_(hb, non_blocking=True)
-        layer.step()
-        hy.copy_(layer.y, non_blocking=True)
+    def one(i):
+        k = i % 2
+        L = layers[k]
+        with torch.cuda.stream(s_up):
+            s_up.wait_event(computed[k])  # the step that last read these inputs is done
+            L.x_cal.copy_(hx_cal, non_blocking=True)
+            L.x.copy_(hx, non_blocking=True)
+            L.w.copy_(hw, non_blocking=True)
+            if hg is not None:
+                L.gamma.copy_(hg, non_blocking=True)
+                L.beta.copy_(hb, non_blocking=True)
+            uploaded[k].record(s_up)
+        s_comp.wait_event(uploaded[k])
+        s_comp.wait_event(read_back[k])  # the output this step overwrites is on the host
+        L.step()
+        computed[k].record(s_comp)
+        with torch.cuda.stream(s_down):
+            s_down.wait_event(computed[k])
+            hy[k].copy_(L.y, non_blocking=True)
+            read_back[k].record(s_down)
 
-    for _ in range(2):
-        one()
+    for i in range(2):
+        one(i)
     barrier()
     s = torch.cuda.Event(enable_timing=True)
     e = torch.cuda.Event(enable_timing=True)
-    s.record()
-    for _ in range(steps):
-        one()
-    e.record()
+    s.record(s_up)
+    for i in range(steps):
+        one(i)
+    e.record(s_down)
     barrier()
     ms = max_over_ranks(s.elapsed_time(e) / steps, world, dev)
     ops = 2.0 * lin.T * lin.N * lin.K
+    del layers[1]
     return {"value": round(throughput_tops(ops, 1, world, ms), 3), "unit": "TOPS",
             "ms_per_step": round(ms, 4), "h2d_bytes_per_step": int(h2d),
-            "d2h_bytes_per_step": int(d2h)}
+            "d2h_bytes_per_step": int(d2h),
+            "pipelining": "two device buffer sets; uploads, kernels and read-backs on three "
+                          "streams, step i's read-back beside step i+1's upload"}
 
 
 # ---------------------------------------------------------------- CPU oracle
