@@ -24,7 +24,7 @@ OBJ_DEBUG = os.path.join(HERE, "_build_debug")
 LIB_DEBUG = os.path.join(HERE, "libsq_b200_debug.so")
 INCLUDE = os.path.join(os.path.dirname(HERE), "include")
 
-SOURCES = ["api.cpp", "status.cu", "rowops.cu", "rowpipe.cu", "gemm.cu", "probe.cu"]
+SOURCES = ["api.cpp", "status.cu", "rowops.cu", "rowpipe.cu", "rowreg.cu", "gemm.cu", "probe.cu"]
 # The row pipeline's packed fp32 multiplies and adds must stay separately
 # rounded (the INT8 codes are bit-exact against the oracle); its one intended
 # fused multiply-add is an explicit intrinsic, which this flag leaves alone.

@@ -159,25 +159,6 @@ __device__ __forceinline__ float2 mul2(float2 a, float2 b) {
   return r;
 }
 
-// Maxima with NaN propagated: NaN if any operand is NaN.  The three-operand
-// form takes |a| and |b| as operand modifiers (one instruction for two
-// elements); the warp form is one redux over the 32 lanes' magnitudes.
-__device__ __forceinline__ float max_nan(float a, float b) {
-  float r;
-  asm("max.NaN.f32 %0, %1, %2;" : "=f"(r) : "f"(a), "f"(b));
-  return r;
-}
-__device__ __forceinline__ float max_nan3(float a, float b, float c) {
-  float r;
-  asm("max.NaN.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
-  return r;
-}
-__device__ __forceinline__ float warp_maxabs_nan(float v) {
-  float r;
-  asm volatile("redux.sync.max.abs.NaN.f32 %0, %1, 0xffffffff;" : "=f"(r) : "f"(v));
-  return r;
-}
-
 // Producer (one thread): streams rows r0 .. r0+R-1 of P.a.x into the ring,
 // row i into slot i mod S, each slot refilled once its consumers released it
 // (empty barrier).  On a time-out it lets every copy already issued land

@@ -120,6 +120,25 @@ __device__ __forceinline__ unsigned int peak_bits(float a) {
   return a != a ? 0u : __float_as_uint(a);
 }
 
+// Maxima with NaN propagated: NaN if any operand is NaN.  The three-operand
+// form takes |a| and |b| as operand modifiers (one instruction for two
+// elements); the warp form is one redux over the 32 lanes' magnitudes.
+__device__ __forceinline__ float max_nan(float a, float b) {
+  float r;
+  asm("max.NaN.f32 %0, %1, %2;" : "=f"(r) : "f"(a), "f"(b));
+  return r;
+}
+__device__ __forceinline__ float max_nan3(float a, float b, float c) {
+  float r;
+  asm("max.NaN.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
+__device__ __forceinline__ float warp_maxabs_nan(float v) {
+  float r;
+  asm volatile("redux.sync.max.abs.NaN.f32 %0, %1, 0xffffffff;" : "=f"(r) : "f"(v));
+  return r;
+}
+
 // 8 consecutive fp32 parameters (gamma, beta, multipliers), at L2.
 __device__ __forceinline__ void load8(const float* p, float (&v)[8]) {
   float4 a = __ldcg(reinterpret_cast<const float4*>(p));
@@ -150,9 +169,9 @@ __device__ __forceinline__ void fold_columns(const float* s, const float* g, con
                                              int nt) {
   if (!g_out && !b_out) return;
   for (int64_t k = (int64_t)blockIdx.x * nt + t; k < K; k += (int64_t)gridDim.x * nt) {
-    const float sk = s[k];
-    if (g_out) g_out[k] = __fdiv_rn(g[k], sk);
-    if (b_out) b_out[k] = __fdiv_rn(b[k], sk);
+    const float sk = __ldcg(s + k);
+    if (g_out) g_out[k] = __fdiv_rn(__ldcg(g + k), sk);
+    if (b_out) b_out[k] = __fdiv_rn(__ldcg(b + k), sk);
   }
 }
 
