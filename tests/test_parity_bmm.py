@@ -62,13 +62,13 @@ def test_bmm(sq, orc, B, M, N, K, out, per_token, per_channel):
     assert_bits_equal(y, y_want, "y")
 
 
-@pytest.mark.parametrize("B,M,N,K", [(3, 130, 200, 240), (3, 130, 200, 512),
-                                     (3, 130, 200, 528), (2, 1024, 2048, 64)])
+@pytest.mark.parametrize("B,M,N,K", [(3, 130, 200, 240), (3, 130, 200, 256), (3, 130, 200, 272),
+                                     (3, 130, 200, 512), (3, 130, 200, 528), (2, 1024, 2048, 64)])
 @pytest.mark.parametrize("out", ["f32", "bf16"])
 def test_bmm_short_k_epilogue(sq, orc, B, M, N, K, out):
     """Head-sized K: three epilogue warps per accumulator quarter up to four
     k-blocks (K = 528 is back on one), with the largest accumulators the
-    codes allow beside random rows.  130 x 200 per batch picks the
+    codes allow beside random rows (2^22 at K = 256).  130 x 200 per batch picks the
     128-column tile (four chunks over three warps), 1024 x 2048 the
     256-column one."""
     r = np.random.default_rng(K + M)

@@ -84,14 +84,15 @@ def test_gemm_extremes(sq, orc):
     assert_bits_equal(y, y_want, "y")
 
 
-@pytest.mark.parametrize("M,N,K", [(200, 264, 240), (200, 264, 512), (200, 264, 528),
-                                   (2048, 2048, 128)])
+@pytest.mark.parametrize("M,N,K", [(200, 264, 240), (200, 264, 256), (200, 264, 272),
+                                   (200, 264, 512), (200, 264, 528), (2048, 2048, 128)])
 def test_gemm_short_k_epilogue(sq, orc, M, N, K):
     """Short K (at most four 128-byte k-blocks) runs the epilogue on three
     warps per accumulator quarter, each taking every third 32-column chunk;
     K = 528 is the first width back on one warp per quarter.  The largest
-    accumulators the codes allow (-128 x -128 x K) sit beside random rows.
-    2048 x 2048 picks the 256-column tile, the others the 192-column one."""
+    accumulators the codes allow (-128 x -128 x K) sit beside random rows:
+    2^22 at K = 256, past the 2^22 bound of fp32 integer tricks at K = 272
+    (the conversion must stay exact there too).  2048 x 2048 picks the 256-column tile, the others the 192-column one."""
     r = np.random.default_rng(K + N)
     xq = r.integers(-128, 128, (M, K)).astype(np.int8)
     wq = r.integers(-128, 128, (N, K)).astype(np.int8)

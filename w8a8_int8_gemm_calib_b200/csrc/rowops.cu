@@ -632,7 +632,7 @@ static cudaError_t dispatch_mode(const RowArgs& a, RowMode mode, cudaStream_t st
 cudaError_t launch_row(const RowArgs& args, sq_dtype xt, RowMode mode, cudaStream_t st) {
   RowArgs a = args;
   a.status = status_word();
-  // bf16 rows without a LayerNorm: whole rows in registers
+  // static steps on bf16 rows without a LayerNorm: whole rows in registers
   if (rowreg_fits(a.K, xt, mode, a.g != nullptr)) return launch_rowreg(a, mode, st);
   // no LayerNorm and one step for the whole call: a plain element stream
   const bool folds = a.fold_g_out || a.fold_b_out;

@@ -63,8 +63,8 @@ struct RowArgs {
 cudaError_t launch_row(const RowArgs& a, sq_dtype xt, RowMode mode,
                        cudaStream_t st);
 
-// Rows held in registers (rowreg.cu): the bf16 row quantizers without a
-// LayerNorm (weight fold, per-token, static, peak pass) up to 20480 columns.
+// Rows held in registers (rowreg.cu): the static quantizer of bf16 rows
+// without a LayerNorm, up to 20480 columns.
 bool rowreg_fits(int64_t K, sq_dtype xt, RowMode mode, bool ln);
 cudaError_t launch_rowreg(const RowArgs& a, RowMode mode, cudaStream_t st);
 
