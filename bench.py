@@ -95,6 +95,8 @@ def parse():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-small-m", action="store_true",
                     help="skip the decode-shaped (small-M) GEMM measurement")
+    ap.add_argument("--no-sustained", action="store_true",
+                    help="skip the one-second back-to-back GEMM / cuBLAS / probe comparison")
     ap.add_argument("--no-extras", action="store_true",
                     help="skip the secondary workload, the HBM rows and the next rows")
     ap.add_argument("--profile-call", default=None, choices=CALLS + ["int8_probe"],
@@ -144,6 +146,7 @@ class ClockSampler:
 
     def __init__(self, index):
         self.samples = []
+        self.power = []
         self.reasons = set()
         self.max_mhz = None
         self._stop = threading.Event()
@@ -163,6 +166,7 @@ class ClockSampler:
         while not self._stop.is_set():
             try:
                 self.samples.append(self.nv.nvmlDeviceGetClockInfo(self.h, self.nv.NVML_CLOCK_SM))
+                self.power.append(self.nv.nvmlDeviceGetPowerUsage(self.h) / 1000.0)
                 r = self.nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
                 for bit, name in self.REASONS.items():
                     if r & bit and name != "gpu_idle":
@@ -185,8 +189,11 @@ class ClockSampler:
     def summary(self):
         if not self._ok or not self.samples:
             return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": ["unavailable"]}
-        return {"sm_mhz": statistics.median(self.samples), "sm_max_mhz": self.max_mhz,
-                "reasons": sorted(self.reasons), "samples": len(self.samples)}
+        out = {"sm_mhz": statistics.median(self.samples), "sm_max_mhz": self.max_mhz,
+               "reasons": sorted(self.reasons), "samples": len(self.samples)}
+        if self.power:
+            out["power_w_median"] = round(statistics.median(self.power), 1)
+        return out
 
 
 # ---------------------------------------------------------------- our arm
@@ -558,6 +565,8 @@ def run_ours(args):
             "alpha_sweep": settled(lambda: run_alpha_sweep(sq, torch, layer, lin, flush)),
             "attention_bmm": settled(
                 lambda: run_attention_bmm(sq, torch, layer.x.device, flush, int8_peak))}
+    if not args.no_extras and not args.no_sustained:
+        extras["sustained_power_cap"] = run_sustained(sq, torch, layer, lin)
 
     traffic = GEMM_DRAM_TRAFFIC.get(wl.name, (None, None))
     line = {
@@ -627,6 +636,54 @@ def time_graph_calls(torch, fn, flush, reps):
         t.append(e0.elapsed_time(e1))
     del graph
     return statistics.mean(t)
+
+
+def run_sustained(sq, torch, layer, lin, seconds=1.0):
+    """The step's GEMM, cuBLAS's INT8 GEMM on the same operands (torch._int_mm,
+    int32 out) and the tcgen05 probe, each back to back for about `seconds`
+    so that the board's power cap engages, with the SM clock and the board
+    power sampled.  int8 ops per clock per SM compares the three at whatever
+    clock the cap leaves each; the tensor cores' ceiling is 16384 (8192
+    multiply-adds per clock per SM)."""
+    sms = torch.cuda.get_device_properties(layer.x.device).multi_processor_count
+    ops = 2.0 * lin.T * lin.N * lin.K
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        layer.call("gemm_w8a8")
+    xq, wq = layer.xq, layer.wq
+    entries = (("gemm_w8a8", lambda: graph.replay(), ops),
+               ("cublas_int_mm_same_shape", lambda: torch._int_mm(xq, wq.t()), ops),
+               ("tcgen05_i8_probe", lambda: sq.sq_probe_mma_i8(8000, sms), 8388608.0 * 8000 * sms))
+    out = {}
+    for name, fn, n_ops in entries:
+        try:
+            e0 = torch.cuda.Event(enable_timing=True)
+            e1 = torch.cuda.Event(enable_timing=True)
+            e0.record()
+            fn()
+            e1.record()
+            torch.cuda.synchronize()
+            n = max(20, int(seconds * 1e3 / e0.elapsed_time(e1)))
+            time.sleep(SETTLE_S)
+            cs = ClockSampler(torch.cuda.current_device())
+            with cs:
+                e0.record()
+                for _ in range(n):
+                    fn()
+                e1.record()
+                torch.cuda.synchronize()
+            ms = e0.elapsed_time(e1) / n
+            tops = n_ops / (ms * 1e-3) / 1e12
+            c = cs.summary()
+            per_clk = (round(tops * 1e12 / (c["sm_mhz"] * 1e6 * sms))
+                       if c.get("sm_mhz") else None)
+            out[name] = {"launches": n, "ms_per_launch": round(ms, 4), "tops": round(tops, 1),
+                         "int8_ops_per_clock_per_sm": per_clk, "clocks": c}
+        except Exception as e:  # noqa: BLE001 - reported; the rest still stands
+            out[name] = {"error": str(e)[:200]}
+    del graph
+    sq.sq_sync_status()
+    return out
 
 
 def run_secondary(args, sq, torch, dev, flush, hbm, int8_peak):
