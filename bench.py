@@ -557,6 +557,7 @@ def run_ours(args):
             SECONDARY_WORKLOAD: settled(
                 lambda: run_secondary(args, sq, torch, dev, flush, hbm, int8_peak))}
         extras["hbm_rows"] = settled(lambda: run_hbm_rows(sq, torch, dev, flush, hbm))
+        extras["gemm_13b_layer"] = settled(lambda: run_13b_gemms(sq, torch, dev, flush, int8_peak))
         extras["next_rows"] = {
             "o2_per_tensor_dynamic_quant": settled(lambda: run_o2(sq, torch, layer, lin, flush)),
             "gemm_bias_epilogue": settled(
@@ -737,6 +738,32 @@ def run_hbm_rows(sq, torch, dev, flush, hbm):
                                    "hbm_frac": round(nb / (ms * 1e-3) / 1e9 / hbm, 3)}
     sq.sq_sync_status()
     return res
+
+
+def run_13b_gemms(sq, torch, dev, flush, int8_peak):
+    """The four GEMMs of the 13B layer (4096 tokens, hidden 5120: QKV, out,
+    fc1, fc2), per-token steps, bf16 out, each one CUDA-graph replay after an
+    L2 flush; TOPS against the measured INT8 peak."""
+    g = torch.Generator(device=dev).manual_seed(23)
+    out = {}
+    for lin in synth.workloads()["13b_layer_t4096"].linears:
+        if not lin.name.endswith("_a0.5"):
+            continue
+        M, N, K = lin.T, lin.N, lin.K
+        xq = torch.randint(-127, 128, (M, K), dtype=torch.int8, device=dev, generator=g)
+        wq = torch.randint(-127, 128, (N, K), dtype=torch.int8, device=dev, generator=g)
+        act = torch.rand(M, device=dev, generator=g) * 0.01 + 1e-4
+        ws = torch.rand(N, device=dev, generator=g) * 0.01 + 1e-4
+        y = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+        wsp = sq.Workspace(dev)
+        ms = time_call(torch, lambda: sq.sq_gemm_w8a8(xq, wq, act, ws, y, per_token=True,
+                                                     workspace=wsp), flush)
+        tops = 2.0 * M * N * K / (ms * 1e-3) / 1e12
+        out[lin.name.split("_")[0]] = {"shape": f"{M}x{N}x{K}", "us": round(ms * 1e3, 2),
+                                       "tops": round(tops, 1), "int8_frac": round(tops / int8_peak, 3)}
+        del xq, wq, y
+    sq.sq_sync_status()
+    return out
 
 
 def run_small_m(sq, torch, dev, flush, reps=20):
