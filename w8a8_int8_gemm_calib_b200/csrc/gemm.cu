@@ -129,26 +129,29 @@ __device__ __forceinline__ float dequant(uint32_t acc, float as, float ws) {
   return __fmul_rn(__int2float_rn((int)acc), __fmul_rn(as, ws));
 }
 
-// The 32 outputs of one row from columns col0..col0+31 of batch b:
-// (float)acc * (as * ws[n]) (+ bias[n]); ws per output channel (batch b's
-// row of w_scale) or, for a batch with one weight step, w_scale[b].
+// The weight steps (and bias) of the 32 columns col0..col0+31 of batch b:
+// ws per output channel (batch b's row of w_scale) or, for a batch with one
+// weight step, wt = w_scale[b].  They are loaded before the chunk's
+// accumulators, so that their L2 latency overlaps the TMEM load (measured:
+// 16384 x 28672 x 8192 2382 -> 2264 us, attention scores 94.2 -> 92.2 us).
 template <bool BATCH>
-__device__ __forceinline__ void dequant_chunk(const Params& p, int b, int col0,
-                                              const uint32_t (&r)[32], float as,
-                                              float (&yv)[32]) {
-  float ws[32];
+__device__ __forceinline__ void load_scales(const Params& p, int b, int col0, float wt,
+                                            float (&ws)[32], float (&bs)[32]) {
   if (BATCH && p.w_per_tensor) {
-    const float w = __ldcg(p.w_scale + b);
 #pragma unroll
-    for (int i = 0; i < 32; ++i) ws[i] = w;
+    for (int i = 0; i < 32; ++i) ws[i] = wt;
   } else {
     load_cols32(p.w_scale + (BATCH ? (size_t)b * (size_t)p.N : (size_t)0), col0, p.N, ws);
   }
+  if (p.bias) load_cols32(p.bias, col0, p.N, bs);
+}
+// The 32 outputs of one row: (float)acc * (as * ws[n]) (+ bias[n])
+__device__ __forceinline__ void dequant_loaded(const Params& p, const uint32_t (&r)[32], float as,
+                                               const float (&ws)[32], const float (&bs)[32],
+                                               float (&yv)[32]) {
 #pragma unroll
   for (int i = 0; i < 32; ++i) yv[i] = dequant(r[i], as, ws[i]);
-  if (p.bias) {  // never with a batch
-    float bs[32];
-    load_cols32(p.bias, col0, p.N, bs);
+  if (p.bias) {
 #pragma unroll
     for (int i = 0; i < 32; ++i) yv[i] = __fadd_rn(yv[i], bs[i]);
   }
@@ -419,15 +422,18 @@ gemm_w8a8_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
       const float as = p.per_token ? (row_ok ? __ldcg(p.act_scale + yrow) : 0.0f)
                                    : __ldcg(p.act_scale + b);
       const uint32_t taddr = tmem_base + abuf * BN + ((uint32_t)(quarter * 32) << 16);
+      const float wt = (BATCH && p.w_per_tensor) ? __ldcg(p.w_scale + b) : 0.0f;
 #pragma unroll 1
       for (int c = chunk0; c < BN / 32; c += EPI_W / 4) {
+        const int col0 = nb * BN + c * 32;
+        float ws[32], bs[32];
+        load_scales<BATCH>(p, b, col0, wt, ws, bs);  // in flight during the TMEM load
         uint32_t r[32];
         tc::tmem_ld32(taddr + c * 32, r);
         tc::tmem_ld_wait();
-        const int col0 = nb * BN + c * 32;
         // dequantize this lane's 32 outputs (row `row`, columns col0..+31)
         float yv[32];
-        dequant_chunk<BATCH>(p, b, col0, r, as, yv);
+        dequant_loaded(p, r, as, ws, bs, yv);
         if constexpr (ERR) {
           // (y - y_ref)^2 and y_ref^2 in fp64, y the fp32 output the store
           // path would write; columns past N hold y = 0 and read ref = 0
