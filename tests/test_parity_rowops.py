@@ -155,6 +155,36 @@ def test_quant_act(sq, orc, dtype, mode, per_token, T, K):
     assert int(host(ncl)[0]) == ncl_want
 
 
+# The static step on bf16 rows without a norm runs whole rows held in
+# registers: 512 threads of one chunk (K <= 4096) or two (K <= 8192), two rows
+# a step, or 640 threads of four chunks (K <= 20480); wider rows take the
+# column strips.  Each width at and just past its boundary, with row counts
+# below, at and past the grid, odd (a last step of one row), and with
+# saturating outliers counted.
+ROWREG_STATIC = [(1, 4096), (149, 4096), (150, 4112), (297, 8192), (147, 8208),
+                 (300, 20480), (5, 20496)]
+
+
+@pytest.mark.parametrize("mode", ["inv_s", "plain"])
+@pytest.mark.parametrize("T,K", ROWREG_STATIC)
+def test_quant_act_static_rows_in_registers(sq, orc, mode, T, K):
+    x = _x(41, T, K, "bf16", relu=(mode == "plain"))
+    r = np.random.default_rng(T * 7 + K)
+    inv = r.uniform(0.02, 2.0, K).astype(np.float32) if mode == "inv_s" else None
+    dstatic = np.float32(0.04)
+    xq_want, _, ncl_want = orc.quant_act(x, None, None, 1e-5, inv, per_token=False,
+                                         static_delta=dstatic)
+    xq = torch.empty((T, K), dtype=torch.int8, device="cuda")
+    act = torch.tensor([dstatic], dtype=torch.float32, device="cuda")
+    ncl = torch.zeros(1, dtype=torch.int64, device="cuda")
+    sq.sq_ln_smooth_quant_act(dev(x), xq, act, None, None, 1e-5, dev(inv), per_token=False,
+                              n_clipped=ncl)
+    sq.sq_sync_status()
+    assert_bits_equal(host(xq), xq_want, "xq")
+    assert int(host(ncl)[0]) == ncl_want
+    assert ncl_want > 0  # the outliers saturate
+
+
 def test_quant_act_edge_values(sq, orc):
     """All-zero rows, +-inf and exact ties at the rounding boundary."""
     K = 64
